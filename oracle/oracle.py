@@ -1,0 +1,550 @@
+"""Plain, slow CPU oracle of one selected-token denoising step.
+
+TEST INFRASTRUCTURE.  This module is the yardstick the CUDA library is
+checked against.  It is imported only by ``tests/``, by
+``__graft_entry__.smoke()`` and by the CPU-baseline legs of ``bench.py``;
+the library never calls it and it never calls the library.  It shares no
+code with the CUDA path: it is numpy in float64, with an optional bf16
+storage emulation (round-to-nearest-even at the points where the bf16
+path stores a tensor).
+
+Sources (web pages; cited by title and section):
+  [ES-de]  "ES-dLLM: Efficient Inference for Diffusion Large Language Models
+           by Early-Skipping", gist.science German technical summary.
+           §1 problem statement, §2.A importance-score equation, §2.B partial
+           cache update / early skip, §4 results (cache size per sample).
+  [ES-nl]  same paper, gist.science Dutch technical summary, "Methodologie"
+           items 1-3 (importance score, early skipping, partial cache update).
+  [DyLLM]  "DyLLM: Efficient Diffusion LLM Inference via Saliency-based
+           Token Selection and Partial Attention", gist.science French
+           technical summary, §1 problem (bidirectional attention, FFN and
+           attention dominate), §2.A saliency by cosine similarity and
+           threshold tau, §2.B partial attention.
+  [SF-de]  "Accelerating Diffusion Large Language Models with SlowFast
+           Sampling", gist.science German technical summary, §2 (top-k
+           confidence unmasking in the exploratory phase).
+
+What the pages leave open and the reading taken here (each is listed again
+in the design notes):
+  * The model is a pre-RMSNorm transformer block with rotate-half RoPE,
+    bidirectional (unmasked) softmax attention, grouped KV heads and a
+    SwiGLU FFN; no biases; untied LM head.  [DyLLM §1] only says
+    "bidirectional" and "FFN"; the shape is the 8B/7B-class layout.
+  * The variation score is taken on the input of the score layer l_s,
+    against that row's value at its last recompute (the hidden-reference
+    cache).  Default kind is 1 - cosine [DyLLM §2.A]; the ES L1 form of
+    [ES-de §2.A] is the alternative.  Rows bitwise equal to their reference
+    score exactly 0.
+  * Importance I = alpha*c + (1-alpha)*v [ES-de §2.A]; c is the cached
+    confidence for masked positions and 0 for unmasked ones.
+  * Top-k ranks by (I descending, position ascending); -0 counts as +0;
+    NaN ranks below everything.  Index lists are returned in ascending
+    position order.
+  * Threshold selection keeps the rows whose score is strictly above tau
+    (with alpha = 0 and the cosine kind this is cos < 1 - tau, the
+    [DyLLM §2.A] rule), capped at k_cap by the same total order.
+  * Selected rows are recomputed through layers l_s..L-1; their new K/V
+    rows overwrite the cache before the layer's attention runs; every
+    other row keeps its cached K/V [ES-de §2.B].
+  * Confidence is the max softmax probability, 1 / sum_j exp(z_j - z_max);
+    argmax ties go to the lowest token id.  Only selected rows that are
+    still masked get new logits; other masked rows keep their cached
+    confidence (c^(t-1) of [ES-de §2.A]).
+  * Unmasking reveals, in the first generation block that still holds a
+    masked position, the n masked positions of highest confidence
+    (ties: lower position first) [SF-de §2].
+
+Parity pins: every public function here is pinned by tests under
+``tests/test_oracle_*.py`` (closed forms, textbook/library special cases,
+brute force on tiny inputs, and invariants the pages state).  The quality
+of the approximate method itself (accuracy on a benchmark) is not pinned:
+that needs trained weights.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import List, Optional
+
+import numpy as np
+
+F32 = "f32"
+BF16 = "bf16"
+
+SCORE_COS = 0
+SCORE_ES_L1 = 1
+SELECT_TOPK = 0
+SELECT_THRESH = 1
+
+
+# ---------------------------------------------------------------------------
+# storage precision
+# ---------------------------------------------------------------------------
+
+def bf16_round(x) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 value (ties to even).
+
+    bfloat16 keeps float32's 8 exponent bits and 7 explicit mantissa bits.
+    Normal numbers are rounded directly on the float64 bit pattern (52 -> 7
+    mantissa bits, no intermediate float32 rounding); values below the
+    smallest normal float32 are rounded on the fixed 2^-133 subnormal grid.
+    Values beyond the bf16 range become +-inf; NaN stays NaN.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty_like(x)
+    bits = x.view(np.uint64)
+    tiny = np.abs(x) < 2.0 ** -126
+    # normal range: round mantissa bits 52 -> 7 with ties to even
+    keep = np.uint64(45)
+    lsb = (bits >> keep) & np.uint64(1)
+    bias = (np.uint64(1) << np.uint64(44)) - np.uint64(1) + lsb
+    rounded = ((bits + bias) >> keep) << keep
+    out_n = rounded.view(np.float64)
+    # bf16 max finite = (2 - 2^-7) * 2^127; anything that rounded past it is inf
+    over = np.abs(out_n) > (2.0 - 2.0 ** -7) * 2.0 ** 127
+    out_n = np.where(over, np.copysign(np.inf, x), out_n)
+    out[...] = out_n
+    # subnormal range of bf16: multiples of 2^-133, round half to even
+    if np.any(tiny):
+        q = 2.0 ** -133
+        out[tiny] = np.round(x[tiny] / q) * q
+    nan = np.isnan(x)
+    if np.any(nan):
+        out[nan] = np.nan
+    return out
+
+
+def store(x, dtype: str) -> np.ndarray:
+    """Value of ``x`` after it is written to a tensor of the path's storage dtype."""
+    if dtype == BF16:
+        return bf16_round(x)
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# model definition
+# ---------------------------------------------------------------------------
+
+@dataclass
+class ModelCfg:
+    n_layers: int
+    d: int
+    n_heads: int
+    n_kv_heads: int
+    head_dim: int
+    ffn: int
+    vocab: int
+    rope_theta: float = 5.0e5
+    rms_eps: float = 1.0e-5
+    mask_id: int = -1          # -1 means vocab - 1
+    dtype: str = BF16
+
+    def __post_init__(self):
+        if self.mask_id < 0:
+            self.mask_id = self.vocab - 1
+
+
+@dataclass
+class LayerW:
+    attn_norm: np.ndarray   # [d]
+    wq: np.ndarray          # [Hq*hd, d]
+    wk: np.ndarray          # [Hkv*hd, d]
+    wv: np.ndarray          # [Hkv*hd, d]
+    wo: np.ndarray          # [d, Hq*hd]
+    ffn_norm: np.ndarray    # [d]
+    w_gate: np.ndarray      # [F, d]
+    w_up: np.ndarray        # [F, d]
+    w_down: np.ndarray      # [d, F]
+
+
+@dataclass
+class ModelW:
+    embed: np.ndarray       # [V, d]
+    layers: List[LayerW]
+    final_norm: np.ndarray  # [d]
+    lm_head: np.ndarray     # [V, d]
+
+
+@dataclass
+class Policy:
+    score_layer: int = 0
+    alpha: float = 0.5
+    kind: int = SCORE_COS
+    mode: int = SELECT_TOPK
+    k: int = 0
+    tau: float = 0.0
+    n_unmask: int = 1
+    gen_start: int = 0
+    block_len: int = 32
+
+
+@dataclass
+class State:
+    """Everything that persists between denoising steps (all float64 / int64)."""
+    tokens: np.ndarray                  # [B, N] int
+    k: List[np.ndarray]                 # per layer [B, N, Hkv, hd]
+    v: List[np.ndarray]                 # per layer [B, N, Hkv, hd]
+    h_ref: np.ndarray                   # [B, N, d] hidden at the score layer, last recompute
+    conf: np.ndarray                    # [B, N] cached confidence
+    pred: np.ndarray                    # [B, N] cached argmax token
+
+    def copy(self) -> "State":
+        return State(self.tokens.copy(), [a.copy() for a in self.k],
+                     [a.copy() for a in self.v], self.h_ref.copy(),
+                     self.conf.copy(), self.pred.copy())
+
+
+def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
+    B, N = tokens.shape
+    kv = (B, N, cfg.n_kv_heads, cfg.head_dim)
+    return State(np.array(tokens, dtype=np.int64).copy(),
+                 [np.zeros(kv) for _ in range(cfg.n_layers)],
+                 [np.zeros(kv) for _ in range(cfg.n_layers)],
+                 np.zeros((B, N, cfg.d)), np.zeros((B, N)),
+                 np.zeros((B, N), dtype=np.int64))
+
+
+# ---------------------------------------------------------------------------
+# transformer sub-blocks
+# ---------------------------------------------------------------------------
+
+def rms_norm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis: x / sqrt(mean(x^2) + eps) * g."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)
+
+
+def rope_inv_freq(head_dim: int, theta: float) -> np.ndarray:
+    """theta^(-2j/hd) for j = 0 .. hd/2-1 (the pair (j, j+hd/2) turns at this rate)."""
+    j = np.arange(head_dim // 2, dtype=np.float64)
+    return theta ** (-2.0 * j / head_dim)
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half rotary embedding.
+
+    ``x`` is [R, H, hd]; ``pos`` is [R] (the row's token index).  The pair
+    (x_j, x_{j+hd/2}) is turned by the angle pos * theta^(-2j/hd).
+    ``theta == 0`` disables the rotation.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    if theta == 0.0:
+        return x.copy()
+    hd = x.shape[-1]
+    half = hd // 2
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * rope_inv_freq(hd, theta)[None, :]
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    a, b = x[..., :half], x[..., half:]
+    return np.concatenate([a * c - b * s, b * c + a * s], axis=-1)
+
+
+def softmax_rows(s: np.ndarray) -> np.ndarray:
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """Bidirectional softmax attention of R query rows over all N keys.
+
+    q [R, Hq, hd]; K, V [N, Hkv, hd]; query head h reads KV head
+    floor(h * Hkv / Hq).  No mask: every query sees every key [DyLLM §1].
+    Returns [R, Hq, hd].
+    """
+    R, Hq, hd = q.shape
+    Hkv = K.shape[1]
+    out = np.empty((R, Hq, hd))
+    scale = 1.0 / math.sqrt(hd)
+    for h in range(Hq):
+        g = (h * Hkv) // Hq
+        p = softmax_rows((q[:, h, :] @ K[:, g, :].T) * scale)
+        out[:, h, :] = p @ V[:, g, :]
+    return out
+
+
+def silu(x: np.ndarray) -> np.ndarray:
+    return x / (1.0 + np.exp(-x))
+
+
+def layer_rows(cfg: ModelCfg, w: LayerW, x: np.ndarray, b_of_row: np.ndarray,
+               pos_of_row: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray) -> np.ndarray:
+    """One transformer layer on a set of rows; updates the layer's K/V cache.
+
+    ``x`` [R, d] are the rows' layer inputs; row r belongs to sequence
+    ``b_of_row[r]`` at position ``pos_of_row[r]``.  The rows' new K/V
+    overwrite the cache before attention, so each selected query sees the
+    fresh K/V of every recomputed row and the cached K/V of the rest
+    [ES-de §2.B].  Returns the layer outputs [R, d] (stored precision).
+    """
+    dt = cfg.dtype
+    Hq, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    R = x.shape[0]
+    n = store(rms_norm(x, w.attn_norm, cfg.rms_eps), dt)
+    q = rope((n @ w.wq.T).reshape(R, Hq, hd), pos_of_row, cfg.rope_theta)
+    k = rope((n @ w.wk.T).reshape(R, Hkv, hd), pos_of_row, cfg.rope_theta)
+    v = (n @ w.wv.T).reshape(R, Hkv, hd)
+    q, k, v = store(q, dt), store(k, dt), store(v, dt)
+    k_cache[b_of_row, pos_of_row] = k
+    v_cache[b_of_row, pos_of_row] = v
+    o = np.empty((R, Hq, hd))
+    for b in np.unique(b_of_row):
+        rows = np.nonzero(b_of_row == b)[0]
+        o[rows] = attention(q[rows], k_cache[b], v_cache[b])
+    o = store(o.reshape(R, Hq * hd), dt)
+    x = store(x + o @ w.wo.T, dt)
+    n2 = store(rms_norm(x, w.ffn_norm, cfg.rms_eps), dt)
+    a = store(silu(n2 @ w.w_gate.T) * (n2 @ w.w_up.T), dt)
+    return store(x + a @ w.w_down.T, dt)
+
+
+# ---------------------------------------------------------------------------
+# scoring, confidence, selection, unmasking
+# ---------------------------------------------------------------------------
+
+def variation(h_cur: np.ndarray, h_ref: np.ndarray, kind: int) -> np.ndarray:
+    """Per-row variation of the hidden state since the row's last recompute.
+
+    kind SCORE_COS:   1 - cos(h, h_ref) [DyLLM §2.A].
+    kind SCORE_ES_L1: ||h - h_ref||_1 / (sqrt(d) * ||h_ref||_2) [ES-de §2.A].
+    Rows bitwise equal to their reference give exactly 0.  For the cosine a
+    zero-norm row against a non-zero one gives cos = 0 (v = 1); for the L1
+    form a zero reference against a different row gives +inf.
+    """
+    h = np.asarray(h_cur, dtype=np.float64)
+    r = np.asarray(h_ref, dtype=np.float64)
+    d = h.shape[-1]
+    same = np.all(h == r, axis=-1)
+    if kind == SCORE_COS:
+        dot = np.sum(h * r, axis=-1)
+        nn = np.sqrt(np.sum(h * h, axis=-1)) * np.sqrt(np.sum(r * r, axis=-1))
+        with np.errstate(divide="ignore", invalid="ignore"):
+            cos = np.where(nn > 0, dot / np.where(nn > 0, nn, 1.0), 0.0)
+        v = 1.0 - cos
+    elif kind == SCORE_ES_L1:
+        l1 = np.sum(np.abs(h - r), axis=-1)
+        nr = np.sqrt(np.sum(r * r, axis=-1))
+        with np.errstate(divide="ignore", invalid="ignore"):
+            v = np.where(nr > 0, l1 / (math.sqrt(d) * np.where(nr > 0, nr, 1.0)), np.inf)
+    else:
+        raise ValueError("unknown score kind")
+    return np.where(same, 0.0, v)
+
+
+def importance(v: np.ndarray, conf: np.ndarray, masked: np.ndarray, alpha: float) -> np.ndarray:
+    """I = alpha * c + (1 - alpha) * v, with c = cached confidence on masked
+    positions and 0 elsewhere [ES-de §2.A]."""
+    c = np.where(np.asarray(masked, dtype=bool), np.asarray(conf, dtype=np.float64), 0.0)
+    return alpha * c + (1.0 - alpha) * np.asarray(v, dtype=np.float64)
+
+
+def confidence(logits: np.ndarray):
+    """Max softmax probability and argmax of each row of ``logits`` [..., V].
+
+    conf = 1 / sum_j exp(z_j - z_max); ties of the maximum go to the lowest id.
+    """
+    z = np.asarray(logits, dtype=np.float64)
+    zmax = np.max(z, axis=-1, keepdims=True)
+    conf = 1.0 / np.sum(np.exp(z - zmax), axis=-1)
+    pred = np.argmax(z, axis=-1)  # first occurrence = lowest id
+    return conf, pred.astype(np.int64)
+
+
+def _rank_key(value: float, pos: int):
+    """Total order for selection: larger value first, NaN last, lower position first."""
+    v = float(value)
+    if math.isnan(v):
+        return (0, 0.0, -pos)
+    if v == 0.0:
+        v = 0.0  # -0 counts as +0
+    return (1, v, -pos)
+
+
+def select_topk(scores: np.ndarray, k: int) -> np.ndarray:
+    """The k highest-ranked positions of one sequence, ascending by position."""
+    n = len(scores)
+    k = max(0, min(int(k), n))
+    order = sorted(range(n), key=lambda i: _rank_key(scores[i], i), reverse=True)
+    return np.array(sorted(order[:k]), dtype=np.int64)
+
+
+def select_thresh(scores: np.ndarray, tau: float, k_cap: int):
+    """Positions with score > tau (strict), capped at k_cap by the top-k order.
+
+    Returns (idx ascending, number over the threshold before the cap).
+    """
+    over = [i for i in range(len(scores))
+            if not math.isnan(float(scores[i])) and float(scores[i]) > tau]
+    n_over = len(over)
+    if n_over > k_cap:
+        over = sorted(over, key=lambda i: _rank_key(scores[i], i), reverse=True)[:k_cap]
+    return np.array(sorted(over), dtype=np.int64), n_over
+
+
+def select(scores: np.ndarray, mode: int, k: int, tau: float, k_cap: int):
+    """Per-sequence selection over scores [B, N] -> list of ascending index arrays."""
+    out = []
+    for b in range(scores.shape[0]):
+        if mode == SELECT_TOPK:
+            out.append(select_topk(scores[b], min(k, k_cap)))
+        else:
+            out.append(select_thresh(scores[b], tau, k_cap)[0])
+    return out
+
+
+def current_block(tokens_b: np.ndarray, mask_id: int, gen_start: int, block_len: int):
+    """[start, end) of the first generation block that still has a masked position."""
+    N = len(tokens_b)
+    m = np.nonzero(tokens_b[gen_start:] == mask_id)[0]
+    if len(m) == 0:
+        return None
+    first = gen_start + int(m[0])
+    start = gen_start + ((first - gen_start) // block_len) * block_len
+    return start, min(start + block_len, N)
+
+
+def unmask_positions(conf_b, tokens_b, mask_id: int, gen_start: int, block_len: int, n: int):
+    """Positions revealed in one sequence this step, ascending [SF-de §2]."""
+    blk = current_block(tokens_b, mask_id, gen_start, block_len)
+    if blk is None or n <= 0:
+        return np.zeros(0, dtype=np.int64)
+    cand = [p for p in range(blk[0], blk[1]) if tokens_b[p] == mask_id]
+    cand.sort(key=lambda p: _rank_key(conf_b[p], p), reverse=True)
+    return np.array(sorted(cand[:n]), dtype=np.int64)
+
+
+def unmask(conf, pred, tokens, mask_id, gen_start, block_len, n):
+    """Applies the unmask rule to every sequence in place; returns pos [B, n] padded with -1."""
+    B = tokens.shape[0]
+    pos = -np.ones((B, max(n, 0)), dtype=np.int64)
+    for b in range(B):
+        p = unmask_positions(conf[b], tokens[b], mask_id, gen_start, block_len, n)
+        tokens[b, p] = pred[b, p]
+        pos[b, :len(p)] = p
+    return pos
+
+
+def apply_unmask(pred, tokens, pos):
+    """Reveals given positions (-1 entries are ignored); used with forced decisions."""
+    for b in range(tokens.shape[0]):
+        p = pos[b][pos[b] >= 0]
+        tokens[b, p] = pred[b, p]
+
+
+# ---------------------------------------------------------------------------
+# the standalone score call (confidence from logits, then importance)
+# ---------------------------------------------------------------------------
+
+def score_call(h_cur, h_ref, conf, pred, masked, alpha, kind,
+               logits=None, logit_pos=None):
+    """Confidence refresh from logits (if given) followed by importance scores.
+
+    logits [B, Mm, V] belong to positions logit_pos [B, Mm]; their max-softmax
+    confidence and argmax overwrite conf/pred there first.  Returns
+    (scores [B, N], conf, pred) as new arrays.
+    """
+    conf = np.array(conf, dtype=np.float64)
+    pred = np.array(pred, dtype=np.int64)
+    if logits is not None:
+        c, p = confidence(logits)
+        for b in range(conf.shape[0]):
+            conf[b, logit_pos[b]] = c[b]
+            pred[b, logit_pos[b]] = p[b]
+    v = variation(h_cur, h_ref, kind)
+    return importance(v, conf, masked, alpha), conf, pred
+
+
+# ---------------------------------------------------------------------------
+# one denoising step
+# ---------------------------------------------------------------------------
+
+@dataclass
+class StepOut:
+    idx: List[np.ndarray]          # per sequence, ascending
+    scores: Optional[np.ndarray]   # [B, N] or None for a dense step
+    unmasked: np.ndarray           # [B, n] padded with -1
+    final_rows: List[np.ndarray] = field(default_factory=list)  # per sequence [k_b, d]
+
+
+def embed(W: ModelW, tokens: np.ndarray) -> np.ndarray:
+    return np.asarray(W.embed, dtype=np.float64)[tokens]
+
+
+def dense_layers(cfg: ModelCfg, W: ModelW, st: State, h: np.ndarray, upto: int) -> np.ndarray:
+    """Layers 0 .. upto-1 on every row (writes every row's K/V there)."""
+    B, N, d = h.shape
+    b_of = np.repeat(np.arange(B), N)
+    p_of = np.tile(np.arange(N), B)
+    x = h.reshape(B * N, d)
+    for l in range(upto):
+        x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l])
+    return x.reshape(B, N, d)
+
+
+def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
+         forced_idx=None, forced_unmask=None, k_cap: Optional[int] = None) -> StepOut:
+    """One denoising step, in place on ``st``.
+
+    1. embed the tokens; run layers below the score layer on every row;
+    2. score every row and select (skipped when ``dense``: all rows);
+    3. store the selected rows' score-layer hidden into the reference cache;
+    4. recompute the selected rows through the remaining layers, updating
+       their K/V rows in each layer's cache [ES-de §2.B, ES-nl Methodologie 3];
+    5. logits -> confidence / argmax for selected rows that are masked;
+    6. unmask in the current block [SF-de §2].
+    ``forced_idx`` / ``forced_unmask`` replace the decisions of steps 2 / 6.
+    """
+    B, N = st.tokens.shape
+    ls = pol.score_layer
+    masked = st.tokens == cfg.mask_id
+    h = embed(W, st.tokens)
+    h = dense_layers(cfg, W, st, h, ls)
+    scores = None
+    if dense:
+        idx = [np.arange(N, dtype=np.int64) for _ in range(B)]
+    elif forced_idx is not None:
+        idx = [np.asarray(a, dtype=np.int64) for a in forced_idx]
+    else:
+        v = variation(h, st.h_ref, pol.kind)
+        scores = importance(v, st.conf, masked, pol.alpha)
+        kc = k_cap if k_cap is not None else (pol.k if pol.mode == SELECT_TOPK else N)
+        idx = select(scores, pol.mode, pol.k, pol.tau, kc)
+    b_of = np.concatenate([np.full(len(a), b, dtype=np.int64) for b, a in enumerate(idx)])
+    p_of = np.concatenate(idx) if len(idx) else np.zeros(0, dtype=np.int64)
+    x = h[b_of, p_of]
+    st.h_ref[b_of, p_of] = x
+    for l in range(ls, cfg.n_layers):
+        if len(b_of):
+            x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l])
+    sel_masked = masked[b_of, p_of]
+    if np.any(sel_masked):
+        n = store(rms_norm(x[sel_masked], W.final_norm, cfg.rms_eps), cfg.dtype)
+        c, p = confidence(n @ np.asarray(W.lm_head, dtype=np.float64).T)
+        st.conf[b_of[sel_masked], p_of[sel_masked]] = c
+        st.pred[b_of[sel_masked], p_of[sel_masked]] = p
+    if forced_unmask is not None:
+        pos = np.asarray(forced_unmask, dtype=np.int64)
+        apply_unmask(st.pred, st.tokens, pos)
+    else:
+        pos = unmask(st.conf, st.pred, st.tokens, cfg.mask_id, pol.gen_start,
+                     pol.block_len, pol.n_unmask)
+    rows = []
+    off = 0
+    for a in idx:
+        rows.append(x[off:off + len(a)].copy())
+        off += len(a)
+    return StepOut(idx, scores, pos, rows)
+
+
+def dense_forward(cfg: ModelCfg, W: ModelW, tokens: np.ndarray) -> np.ndarray:
+    """Full recomputation of every row through every layer (the vanilla pass);
+    returns the final hidden rows [B, N, d]."""
+    st = empty_state(cfg, tokens)
+    return dense_layers(cfg, W, st, embed(W, st.tokens), cfg.n_layers)
+
+
+def kv_cache_bytes(n_layers: int, n_tokens: int, n_kv_heads: int, head_dim: int,
+                   bytes_per_elem: int = 2) -> int:
+    """Bytes of the per-layer K and V caches of one sequence."""
+    return 2 * n_layers * n_tokens * n_kv_heads * head_dim * bytes_per_elem
