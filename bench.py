@@ -1,0 +1,411 @@
+"""Benchmark of the selected-token denoising step on B200.
+
+Default workload: the 8B-shaped model (32 layers, d 4096, 32 heads x 128,
+SwiGLU 12288, vocab 126464, bf16, random-init N(0, 0.02) weights) over 32
+sequences of 1536 tokens (512 random prompt ids + 1024 [MASK], blocks of 64).
+After an untimed dense first step, each timed step is one partial denoising
+step: score all rows, keep 20 % (308 per sequence), recompute them through
+the 32 layers against the full cached K/V, refresh confidence on the masked
+ones and reveal 16 tokens per sequence.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  Under torchrun every rank runs its own 32
+sequences on its own GPU (replicated weights, no collective in the step);
+the timed region is bracketed by a barrier and a device synchronize and the
+reported time is the maximum over ranks.  ``--impl reference`` times the CPU
+oracle (plain float64 numpy) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import dllm_synth as SY  # noqa: E402
+
+METRIC = "tokens/s & denoise steps/s at 8B shape, bs 1/32; % of HBM / bf16 TC roofline"
+SHAPE = SY.DENSE8B_B32_N1536
+BS1 = SY.DENSE8B_B1_N768
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-bs1", action="store_true", help="skip the batch-1 measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="(debug) override the layer count")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons while timing."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str):
+        self.uuid = uuid
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        try:
+            rows = [l.strip().split(", ") for l in open(self.path) if l.strip()]
+        except Exception:
+            return None
+        mine = [r for r in rows if len(r) >= 10 and (not self.uuid or self.uuid in r[1])]
+        if not mine:
+            mine = [r for r in rows if len(r) >= 10 and r[0] == "0"]
+        if not mine:
+            return None
+        sm = [float(r[2]) for r in mine if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in mine if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in mine for i in range(4) if r[6 + i] == "Active"})
+        under = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(under) if under else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(mine)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- our path
+
+def setup(S, shape, rank, layers=0):
+    import torch
+    if layers:
+        shape = SY.with_(shape, n_layers=layers)
+    W = SY.model_weights(shape, seed=0, device="cuda")
+    model = S.Model(S.cfg_from_shape(shape), W)
+    tokens = SY.prompt_tokens(shape, seed=1 + rank, device="cuda")
+    cache = S.Cache(model.cfg, shape.batch, shape.seq_len)
+    pol = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k, n_unmask=shape.n_unmask,
+                        gen_start=shape.prompt_len, block_len=shape.block_len)
+    ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+    torch.cuda.synchronize()
+    return shape, W, model, tokens, cache, pol, ws
+
+
+def time_steps(S, model, cache, tokens, pol, ws, K, stream):
+    import torch
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        S.dllm_step(model, cache, tokens, pol, False, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def bs1_measure(S, W, steps, warmup):
+    """Batch-1 8B step (768 tokens, blocks of 32, 8 revealed/step) at 10/25/50 %."""
+    import torch
+    out = {}
+    model = S.Model(S.cfg_from_shape(BS1), W)
+    stream = torch.cuda.current_stream()
+    for ratio in (0.10, 0.25, 0.50):
+        shape = SY.with_(BS1, ratio=ratio)
+        tokens = SY.prompt_tokens(shape, seed=7, device="cuda")
+        cache = S.Cache(model.cfg, 1, shape.seq_len)
+        pol = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k,
+                            n_unmask=shape.n_unmask, gen_start=shape.prompt_len,
+                            block_len=shape.block_len)
+        ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, 1, shape.seq_len, pol))
+        S.dllm_step(model, cache, tokens, pol, True, ws)
+        for _ in range(warmup):
+            S.dllm_step(model, cache, tokens, pol, False, ws)
+        torch.cuda.synchronize()
+        K = min(steps, 20)
+        ms = time_steps(S, model, cache, tokens, pol, ws, K, stream) / K
+        out[f"r{int(ratio * 100)}"] = {"k": shape.k, "ms_per_step": round(ms, 4),
+                                       "steps_per_s": round(1000.0 / ms, 2),
+                                       "tokens_per_s": round(shape.n_unmask * 1000.0 / ms, 1)}
+        del cache, ws
+    return out
+
+
+def cpu_baseline_sample(W, cache, tokens, shape):
+    """The oracle on one sequence, one layer and that sequence's LM-head rows,
+    scaled to a full step: per step = 32 sequences x (32 layers x t_layer + t_lm)."""
+    import numpy as np
+    import torch
+    import oracle as O
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    L = W["layers"][0]
+    ow = O.LayerW(**{k: f64(v) for k, v in L.items()})
+    cfg = O.ModelCfg(shape.n_layers, shape.d, shape.n_heads, shape.n_kv_heads, shape.head_dim,
+                     shape.ffn, shape.vocab, shape.rope_theta, shape.rms_eps, shape.mask_id,
+                     shape.dtype)
+    k = shape.k
+    rows = np.arange(shape.seq_len - k, shape.seq_len)  # stand-in for the selected rows
+    x = f64(W["embed"][tokens[0, rows].long()])
+    kb, vb = f64(cache.k[0][0:1]), f64(cache.v[0][0:1])
+    t0 = time.perf_counter()
+    xo = O.layer_rows(cfg, ow, x, np.zeros(k, dtype=np.int64), rows, kb, vb)
+    t_layer = time.perf_counter() - t0
+    n_lm = k - shape.n_unmask
+    lm = f64(W["lm_head"])
+    fn = f64(W["final_norm"])
+    t0 = time.perf_counter()
+    n = O.store(O.rms_norm(xo[:n_lm], fn, cfg.rms_eps), cfg.dtype)
+    O.confidence(n @ lm.T)
+    t_lm = time.perf_counter() - t0
+    per_step = shape.batch * (shape.n_layers * t_layer + t_lm)
+    tps = shape.batch * shape.n_unmask / per_step
+    return {"value": tps, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"1 of {shape.batch} sequences, layer 1 of {shape.n_layers} ({k} rows) + "
+                      f"LM head on {n_lm} rows; scaled to a full step "
+                      f"({t_layer:.2f} s/layer, {t_lm:.2f} s LM head measured)",
+            "s_per_step_extrapolated": per_step}
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    import sparse_token_recompute_b200 as S  # raises if the CUDA library is missing
+
+    hbm, tc_burst, tc_sus, peak_kind = peaks()
+    shape, W, model, tokens, cache, pol, ws = setup(S, SHAPE, rank, args.layers)
+    stream = torch.cuda.current_stream()
+    S.dllm_step(model, cache, tokens, pol, True, ws)           # dense first step (untimed)
+    for _ in range(args.warmup):
+        S.dllm_step(model, cache, tokens, pol, False, ws)
+    torch.cuda.synchronize()
+    st = ws.device_status()
+    if st:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    try:
+        uuid = str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        uuid = ""
+    barrier(world)
+    torch.cuda.synchronize()
+    S.profile_reset()
+    S.profile_enable(True)
+    with Clocks(uuid) as clk:
+        ms = time_steps(S, model, cache, tokens, pol, ws, args.steps, stream)
+    S.profile_enable(False)
+    prof = S.profile_read()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    tok_per_step = shape.batch * shape.n_unmask
+    value = world * tok_per_step * 1000.0 / ms_step
+
+    # end to end through the public API with host token buffers
+    tok_h = torch.empty_like(tokens, device="cpu").pin_memory()
+    tok_h.copy_(tokens)
+    pos_h = torch.empty(shape.batch, shape.n_unmask, dtype=torch.int32).pin_memory()
+    pos_d = torch.empty(shape.batch, shape.n_unmask, dtype=torch.int32, device="cuda")
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        S.dllm_step_host(model, cache, tok_h, pol, False, ws, tokens, pos_d, pos_h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+    barrier(world)
+
+    # roofline of the dominant kernel: the tensor-core GEMM of the layer projections
+    M = shape.batch * shape.k
+    q = shape.n_heads * shape.head_dim
+    kv = shape.n_kv_heads * shape.head_dim
+    p_layer = shape.d * (q + 2 * kv) + q * shape.d + 2 * shape.d * shape.ffn + shape.ffn * shape.d
+    flops_step = 2.0 * M * p_layer * shape.n_layers
+    gemm_names = ("gemm_qkv", "gemm_resid", "gemm_swiglu")
+    gemm_ms = sum(prof.get(n, [0, 0.0])[1] for n in gemm_names)
+    gemm_launches = sum(prof.get(n, [0, 0.0])[0] for n in gemm_names)
+    achieved = flops_step * args.steps / (gemm_ms / 1000.0) / 1e12 if gemm_ms else None
+    launches = int(sum(v[0] for v in prof.values()))
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: random-init weights N(0,0.02), uniform random prompt ids, "
+                "all-[MASK] generation region",
+        "config": {"workload": f"8B-shaped partial denoising step, {shape.batch} x "
+                               f"{shape.seq_len} tokens ({shape.prompt_len} prompt + "
+                               f"{shape.gen_len} generated, blocks of {shape.block_len}), "
+                               f"{int(shape.ratio * 100)}% recompute ({shape.k} rows/seq), "
+                               f"{shape.n_unmask} tokens revealed/seq/step, 32 layers",
+                   "global_batch": world * shape.batch, "seq_len": shape.seq_len,
+                   "parallelism": f"dp{world} (replicated weights, sequences sharded)",
+                   "l2": "inputs larger than L2: ~16 GB weights + ~26 GB K/V caches per step"},
+        "steps_per_s": round(1000.0 / ms_step, 3),
+        "roofline": {
+            "kernel": "gemm_tc (tcgen05 layer projections: QKV+RoPE+KV scatter, O+residual, "
+                      "gate/up+SwiGLU, down+residual)",
+            "bound": "tensor", "achieved": round(achieved, 1) if achieved else None,
+            "peak": tc_sus, "unit": "TFLOP/s",
+            "frac": round(achieved / tc_sus, 4) if achieved else None,
+            "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long step)",
+            "flops_per_step": flops_step, "launches": gemm_launches,
+            "avg_launch_ms": round(gemm_ms / max(gemm_launches, 1), 4), "traffic": None},
+        "e2e": {"value": round(world * tok_per_step * 1000.0 / ms_e2e, 2), "unit": "tokens/s",
+                "ms_per_step": round(ms_e2e, 4),
+                "h2d_bytes_per_step": tokens.numel() * 4,
+                "d2h_bytes_per_step": tokens.numel() * 4 + pos_d.numel() * 4},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "kernels_ms": {k: [v[0], round(v[1], 3)] for k, v in sorted(prof.items())},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline_sample(W, cache, tokens, shape)
+    if not args.no_bs1 and not args.layers:
+        del cache, ws
+        torch.cuda.empty_cache()
+        result["bs1"] = bs1_measure(S, W, args.steps, args.warmup)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle as O
+    shape = SHAPE
+    # one layer's weights and one sequence's caches at the real shape, drawn on the host
+    W1 = SY.model_weights(SY.with_(shape, n_layers=1, vocab=shape.vocab), seed=0, device="cpu")
+    times = []
+    k = shape.k
+    cfg = O.ModelCfg(shape.n_layers, shape.d, shape.n_heads, shape.n_kv_heads, shape.head_dim,
+                     shape.ffn, shape.vocab, shape.rope_theta, shape.rms_eps, shape.mask_id,
+                     shape.dtype)
+    f64 = lambda t: t.detach().to(torch.float64).numpy()
+    L = W1["layers"][0]
+    ow = O.LayerW(**{kk: f64(v) for kk, v in L.items()})
+    kvs = (1, shape.seq_len, shape.n_kv_heads, shape.head_dim)
+    kb = f64(SY.normal(kvs, 1.0, 5, "cpu", "bf16"))
+    vb = f64(SY.normal(kvs, 1.0, 6, "cpu", "bf16"))
+    rows = np.arange(shape.seq_len - k, shape.seq_len)
+    x = f64(SY.normal((k, shape.d), 1.0, 7, "cpu", "bf16"))
+    lm = f64(W1["lm_head"])
+    fn = f64(W1["final_norm"])
+    n_lm = k - shape.n_unmask
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        xo = O.layer_rows(cfg, ow, x, np.zeros(k, dtype=np.int64), rows, kb.copy(), vb.copy())
+        t1 = time.perf_counter()
+        n = O.store(O.rms_norm(xo[:n_lm], fn, cfg.rms_eps), cfg.dtype)
+        O.confidence(n @ lm.T)
+        t2 = time.perf_counter()
+        if i >= args.warmup:
+            times.append(shape.batch * (shape.n_layers * (t1 - t0) + (t2 - t1)))
+    s_step = statistics.mean(times)
+    value = shape.batch * shape.n_unmask / s_step
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"per step: 1 of {shape.batch} sequences through 1 of {shape.n_layers} layers "
+              f"({k} rows) + LM head on {n_lm} rows, scaled by {shape.batch} sequences x "
+              f"{shape.n_layers} layers")
+    out = {"metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s_step * 1000, 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": {"workload": "8B-shaped partial denoising step, 32 x 1536 tokens, 20% "
+                                  "recompute (CPU oracle, sampled)",
+                      "global_batch": shape.batch, "seq_len": shape.seq_len,
+                      "parallelism": "cpu"},
+           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores,
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,288 @@
+/*
+ * dllm.h - C ABI of the selected-token denoising step for masked-diffusion
+ * language models, sm_100a (NVIDIA B200).
+ *
+ * One denoising step scores every token by how far its hidden state moved
+ * since the row was last recomputed and by its cached confidence, keeps the
+ * top-k (or over-threshold) positions, recomputes only those rows through
+ * the transformer layers (their queries attend to the full cached K/V), and
+ * writes the new K/V / hidden / confidence rows back into the caches.
+ *
+ * Sources, cited by page title and section:
+ *   [ES-de]  "ES-dLLM: Efficient Inference for Diffusion Large Language
+ *            Models by Early-Skipping", German technical summary: section 2.A
+ *            (importance score I = alpha*c + (1-alpha)*variation, alpha 0.5),
+ *            section 2.B (top-k rows processed, K/V/hidden caches updated for
+ *            selected rows in place, skipped rows reuse cached values).
+ *   [DyLLM]  "DyLLM: Efficient Diffusion LLM Inference via Saliency-based
+ *            Token Selection and Partial Attention", French technical
+ *            summary: section 1 (bidirectional attention over the whole
+ *            sequence each step), section 2.A (cosine similarity against the
+ *            previous step, salient if below a threshold tau), section 2.B
+ *            (rows of salient tokens recomputed exactly).
+ *   [SF-de]  "Accelerating Diffusion Large Language Models with SlowFast
+ *            Sampling", German technical summary, section 2 (the most
+ *            confident masked tokens of a window are revealed each step).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer argument is device memory owned by the caller unless the
+ *     argument is documented as host memory.  The library never allocates
+ *     device memory: scratch comes from a caller buffer of at least the size
+ *     the matching *_workspace_size() call returns (256-byte aligned).
+ *   - Every call is asynchronous on the given CUDA stream (NULL: the legacy
+ *     default stream) and returns before the GPU work finishes.
+ *   - Arguments are validated before anything is launched; on an error
+ *     nothing is launched and outputs are untouched.
+ *   - Faults the GPU detects (a wait that ran past its limit, more candidates
+ *     than an index list holds) set bits in a status word inside the
+ *     workspace; dllm_get_device_status() reads and clears it.
+ *   - Tensors are dense row-major; weights are [out, in] (y = x W^T).
+ *   - Storage dtype DLLM_BF16 computes with fp32 accumulation and stores
+ *     bf16; DLLM_F32 stores fp32 (small models, exact-arithmetic checks).
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef DLLM_H
+#define DLLM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* dllm_stream_t;
+
+typedef enum {
+  DLLM_OK = 0,
+  DLLM_ERR_INVALID_ARG = 1,      /* null pointer, negative size, bad enum      */
+  DLLM_ERR_UNSUPPORTED_SHAPE = 2,/* a size this build cannot run (see below)   */
+  DLLM_ERR_WORKSPACE = 3,        /* workspace missing, misaligned or too small */
+  DLLM_ERR_CUDA = 4,             /* a CUDA runtime call failed                 */
+  DLLM_ERR_CAPACITY = 5,         /* more rows than the index capacity          */
+  DLLM_ERR_DEVICE = 6            /* the device status word is non-zero         */
+} dllm_status;
+
+typedef enum { DLLM_F32 = 0, DLLM_BF16 = 1 } dllm_dtype;
+
+/* variation measure: 1 - cos(h, h_ref) [DyLLM 2.A] or
+ * ||h - h_ref||_1 / (sqrt(d) ||h_ref||_2) [ES-de 2.A] */
+typedef enum { DLLM_SCORE_COS = 0, DLLM_SCORE_ES_L1 = 1 } dllm_score_kind;
+
+/* top-k [ES-de 2.B] or every score strictly above tau [DyLLM 2.A] */
+typedef enum { DLLM_SELECT_TOPK = 0, DLLM_SELECT_THRESH = 1 } dllm_select_mode;
+
+/* device status word bits */
+#define DLLM_DEV_TIMEOUT 1
+#define DLLM_DEV_CAPACITY 2
+#define DLLM_DEV_BAD_INDEX 4
+#define DLLM_DEV_BAD_SHAPE 8
+
+typedef struct {
+  int n_layers;
+  int d;            /* model width                                  */
+  int n_heads;      /* query heads                                  */
+  int n_kv_heads;   /* key/value heads (divides n_heads)            */
+  int head_dim;     /* 64 or 128                                    */
+  int ffn;          /* SwiGLU hidden width                          */
+  int vocab;
+  float rope_theta; /* 0 disables the rotary embedding              */
+  float rms_eps;
+  int mask_id;      /* token id of [MASK]                           */
+  int dtype;        /* dllm_dtype of weights, caches and activations */
+} dllm_model_cfg;
+
+/* One pre-RMSNorm transformer block.  Device pointers, dtype of the model. */
+typedef struct {
+  const void* attn_norm; /* [d]                    */
+  const void* wq;        /* [n_heads*head_dim, d]  */
+  const void* wk;        /* [n_kv_heads*head_dim, d] */
+  const void* wv;        /* [n_kv_heads*head_dim, d] */
+  const void* wo;        /* [d, n_heads*head_dim]  */
+  const void* ffn_norm;  /* [d]                    */
+  const void* w_gate;    /* [ffn, d]               */
+  const void* w_up;      /* [ffn, d]               */
+  const void* w_down;    /* [d, ffn]               */
+} dllm_layer_w;
+
+typedef struct {
+  const void* embed;            /* [vocab, d] device                      */
+  const dllm_layer_w* layers;   /* HOST array [n_layers] of device pointers */
+  const void* final_norm;       /* [d] device                             */
+  const void* lm_head;          /* [vocab, d] device                      */
+} dllm_model_w;
+
+/* The state kept between steps.  k/v are HOST arrays of n_layers device
+ * pointers, each cache [B, N, n_kv_heads, head_dim] (K stored after RoPE).
+ * h_ref [B, N, d]: each row's score-layer hidden at its last recompute.
+ * conf [B, N] f32 / pred [B, N] int32: confidence and argmax of each
+ * position's last LM-head evaluation (c^(t-1) of [ES-de 2.A]). */
+typedef struct {
+  void* const* k;
+  void* const* v;
+  void* h_ref;
+  float* conf;
+  int32_t* pred;
+} dllm_cache;
+
+typedef struct {
+  int score_layer;   /* layers below it run on every row; the score is taken on its input */
+  float alpha;       /* I = alpha * c + (1 - alpha) * v                 */
+  int kind;          /* dllm_score_kind                                 */
+  int mode;          /* dllm_select_mode                                */
+  int k;             /* TOPK: rows per sequence; THRESH: capacity       */
+  float tau;         /* THRESH: keep scores > tau                       */
+  int n_unmask;      /* positions revealed per sequence and step        */
+  int gen_start;     /* first generated position                        */
+  int block_len;     /* generation block length                         */
+} dllm_policy;
+
+/* Supported shapes for DLLM_BF16 layer work: d, n_heads*head_dim,
+ * n_kv_heads*head_dim and ffn multiples of 128; head_dim 64 or 128;
+ * vocab a multiple of 8.  DLLM_F32: any d, ffn; head_dim <= 128 even.
+ * Sequence length N <= 16384 for selection and unmasking; block_len <= 1024. */
+
+const char* dllm_status_string(int status);
+int dllm_version(void);
+
+/*
+ * dllm_score - importance score of every row [ES-de 2.A; DyLLM 2.A].
+ *
+ * When logits != NULL, first refreshes the cached confidence of the rows
+ * the logits belong to: for b < B, j < Mm, row logit_pos[b*Mm+j] of
+ * sequence b gets conf = max softmax of logits[b, j, :] (in fp32) and
+ * pred = its argmax (lowest id on ties).  Then for every row i:
+ *   v_i = variation(h_cur[b,i,:], h_ref[b,i,:], kind)   (0 when bitwise equal)
+ *   c_i = masked[b,i] ? conf[b,i] : 0
+ *   scores[b,i] = alpha * c_i + (1 - alpha) * v_i       (fp32)
+ * h_cur, h_ref: [B, N, d] of dtype; logits [B, Mm, V] of dtype;
+ * logit_pos [B, Mm] int32 in [0, N); conf [B, N] f32 in/out;
+ * pred [B, N] int32 out (may be NULL); masked [B, N] uint8; scores [B, N] f32 out.
+ * d must be a multiple of 8 (bf16) or 4 (f32); V a multiple of 8 (bf16) or 4.
+ */
+dllm_status dllm_score(const void* h_cur, const void* h_ref, int B, int N, int d, int dtype,
+                       const void* logits, const int32_t* logit_pos, int Mm, int V, float* conf,
+                       int32_t* pred, const uint8_t* masked, float alpha, int kind,
+                       float* scores, dllm_stream_t stream);
+
+/*
+ * dllm_select - per-sequence compaction of the rows to recompute [ES-de 2.B].
+ *
+ * TOPK: the min(k, N) highest scores of each sequence under the order
+ * (score descending, position ascending; -0 equals +0; NaN below all).
+ * THRESH: every position with score > tau, capped at k_cap by that order.
+ * idx [B, k_cap] int32 receives each sequence's positions in ascending order
+ * (entries past count[b] are left untouched); count [B] int32.
+ * ws: at least dllm_select_workspace_size() bytes, or NULL; when given, a
+ * THRESH selection clipped by k_cap sets DLLM_DEV_CAPACITY in its status word.
+ * Bit-exact and deterministic.  N <= 16384; k_cap >= 1 (TOPK needs k <= k_cap).
+ */
+size_t dllm_select_workspace_size(int B, int N);
+dllm_status dllm_select(const float* scores, int B, int N, int mode, int k, float tau,
+                        int32_t* idx, int32_t* count, int k_cap, void* ws, size_t ws_bytes,
+                        dllm_stream_t stream);
+
+/*
+ * dllm_unmask - reveal the most confident masked positions [SF-de 2].
+ *
+ * For each sequence: the current block is [s, min(s + block_len, N)) with
+ * s = gen_start + floor((p - gen_start) / block_len) * block_len and p the
+ * first masked position >= gen_start.  Among its masked positions the
+ * n_unmask with the highest conf (ties: lower position) get
+ * tokens[b, p] = pred[b, p].  pos_out [B, n_unmask] int32 receives the
+ * revealed positions in ascending order, padded with -1.
+ * Bit-exact.  block_len <= 1024, N <= 16384.
+ */
+dllm_status dllm_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
+                        int mask_id, int gen_start, int block_len, int n_unmask,
+                        int32_t* pos_out, dllm_stream_t stream);
+
+/*
+ * dllm_partial_layer - one transformer layer on the selected rows only
+ * [ES-de 2.B; DyLLM 2.B].
+ *
+ * Rows: sequence b contributes count[b] rows, positions idx[b*k_cap + j]
+ * (ascending, j < count[b]).  They are packed by sequence: compact row r of
+ * sequence b is r = sum_{b'<b} count[b'] + j.
+ * x_in: x_in_is_full = 1 -> [B, N, d], row (b, idx) is gathered;
+ *       x_in_is_full = 0 -> compact [B*k_cap, d].
+ * x_out: compact [B*k_cap, d] (may equal x_in when compact).
+ * Order inside the layer: RMSNorm -> Q,K,V of all selected rows (RoPE at the
+ * row's position) -> their K/V rows overwrite k_cache/v_cache
+ * [B, N, n_kv_heads, head_dim] -> each selected query attends to all N keys
+ * of its sequence (no mask, scale 1/sqrt(head_dim)) -> O projection +
+ * residual -> RMSNorm -> SwiGLU FFN + residual.
+ * Rows that are not selected keep their cached K/V untouched.
+ */
+size_t dllm_partial_layer_workspace_size(const dllm_model_cfg* cfg, int B, int N, int k_cap);
+dllm_status dllm_partial_layer(const dllm_model_cfg* cfg, const dllm_layer_w* w,
+                               const void* x_in, int x_in_is_full, void* x_out,
+                               const int32_t* idx, const int32_t* count, int k_cap, int B,
+                               int N, void* k_cache, void* v_cache, void* ws, size_t ws_bytes,
+                               dllm_stream_t stream);
+
+/*
+ * dllm_step - one whole denoising step [ES-de 2.A-2.B; DyLLM 2; SF-de 2].
+ *
+ * tokens [B, N] int32 in/out.  With dense = 1 every row is recomputed
+ * (first step, or a full refresh).  Otherwise:
+ *  1. h = embedding of tokens; layers below policy.score_layer run on every row;
+ *  2. scores as dllm_score with c = cache.conf, alpha/kind from policy;
+ *  3. selection as dllm_select (k_cap = min(policy.k, N));
+ *  4. cache.h_ref rows of the selection <- their score-layer hidden;
+ *  5. dllm_partial_layer for layers score_layer .. n_layers-1;
+ *  6. for selected rows whose token is [MASK]: final RMSNorm, LM head,
+ *     cache.conf <- max softmax, cache.pred <- argmax (logits never stored);
+ *  7. dllm_unmask with policy.n_unmask / gen_start / block_len.
+ * forced_idx [B, k_cap] + forced_count [B] replace steps 2-3 when non-NULL;
+ * forced_unmask_pos [B, n_unmask] (-1 padded) replaces step 7's choice.
+ * Outputs (each may be NULL): idx_out [B, k_cap], count_out [B],
+ * pos_out [B, n_unmask], scores_out [B, N].
+ * The workspace size covers both dense and partial steps of this shape.
+ */
+size_t dllm_step_workspace_size(const dllm_model_cfg* cfg, int B, int N,
+                                const dllm_policy* policy);
+dllm_status dllm_step(const dllm_model_cfg* cfg, const dllm_model_w* w, const dllm_cache* cache,
+                      int32_t* tokens, int B, int N, const dllm_policy* policy, int dense,
+                      const int32_t* forced_idx, const int32_t* forced_count,
+                      const int32_t* forced_unmask_pos, int32_t* idx_out, int32_t* count_out,
+                      int32_t* pos_out, float* scores_out, void* ws, size_t ws_bytes,
+                      dllm_stream_t stream);
+
+/*
+ * dllm_get_device_status - synchronises `stream`, copies the device status
+ * word of a workspace used by dllm_select / dllm_partial_layer / dllm_step
+ * into *status_out (HOST memory), and clears it.  Returns DLLM_ERR_DEVICE
+ * when the word was non-zero.
+ */
+dllm_status dllm_get_device_status(void* ws, dllm_stream_t stream, int32_t* status_out);
+
+/*
+ * dllm_gemm_bf16 - the tensor-core GEMM the layer path runs on, exposed for
+ * direct checks: C[M, N] = A[M, K] * B[N, K]^T (+ C when accumulate != 0),
+ * bf16 in, fp32 accumulate, bf16 out.  K, N multiples of 8; a multiple of
+ * 64 in K keeps every k-block full.  splits > 1 splits K across CTAs and
+ * reduces in a fixed order (deterministic); needs ws of
+ * dllm_gemm_workspace_size() bytes.
+ */
+size_t dllm_gemm_workspace_size(int M, int N, int K, int splits);
+dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, int M, int N, int K,
+                           int accumulate, int splits, void* ws, size_t ws_bytes,
+                           dllm_stream_t stream);
+
+/*
+ * Kernel timing.  dllm_profile_enable(1) brackets every kernel the library
+ * launches with CUDA events on the launch stream; dllm_profile_read()
+ * synchronises the device, writes a JSON object
+ * {"kernel": [launches, total_ms], ...} into buf (HOST, len bytes) and
+ * returns the bytes needed; dllm_profile_reset() clears the counters.
+ */
+void dllm_profile_enable(int on);
+void dllm_profile_reset(void);
+size_t dllm_profile_read(char* buf, size_t len);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DLLM_H */

@@ -1,0 +1,337 @@
+"""Python binding of libdllm.so, the sm_100a selected-token denoising step.
+
+Argument marshalling only: every step of the path runs in the library's
+CUDA kernels.  Tensors are torch CUDA tensors (device memory and streams);
+they are passed as raw pointers through ctypes.  If the shared library is
+missing, importing this package raises: there is no fallback path.
+
+The functions carry the C names (``dllm_score``, ``dllm_select``,
+``dllm_unmask``, ``dllm_partial_layer``, ``dllm_step`` ...); ``Model``,
+``Cache`` and ``Workspace`` hold the ctypes structs and the torch-owned
+buffers the calls need.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import json
+import os
+from typing import Dict, List, Optional, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdllm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m sparse_token_recompute_b200.build` "
+        "(there is no CPU or eager fallback)")
+
+_lib = C.CDLL(LIB_PATH)
+
+DLLM_OK = 0
+DLLM_F32, DLLM_BF16 = 0, 1
+DLLM_SCORE_COS, DLLM_SCORE_ES_L1 = 0, 1
+DLLM_SELECT_TOPK, DLLM_SELECT_THRESH = 0, 1
+DLLM_DEV_TIMEOUT, DLLM_DEV_CAPACITY, DLLM_DEV_BAD_INDEX, DLLM_DEV_BAD_SHAPE = 1, 2, 4, 8
+
+vp = C.c_void_p
+
+
+class ModelCfg(C.Structure):
+    _fields_ = [("n_layers", C.c_int), ("d", C.c_int), ("n_heads", C.c_int),
+                ("n_kv_heads", C.c_int), ("head_dim", C.c_int), ("ffn", C.c_int),
+                ("vocab", C.c_int), ("rope_theta", C.c_float), ("rms_eps", C.c_float),
+                ("mask_id", C.c_int), ("dtype", C.c_int)]
+
+
+class LayerW(C.Structure):
+    _fields_ = [(n, vp) for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm", "w_gate",
+                                  "w_up", "w_down")]
+
+
+class ModelW(C.Structure):
+    _fields_ = [("embed", vp), ("layers", C.POINTER(LayerW)), ("final_norm", vp),
+                ("lm_head", vp)]
+
+
+class CacheS(C.Structure):
+    _fields_ = [("k", C.POINTER(vp)), ("v", C.POINTER(vp)), ("h_ref", vp), ("conf", vp),
+                ("pred", vp)]
+
+
+class Policy(C.Structure):
+    _fields_ = [("score_layer", C.c_int), ("alpha", C.c_float), ("kind", C.c_int),
+                ("mode", C.c_int), ("k", C.c_int), ("tau", C.c_float), ("n_unmask", C.c_int),
+                ("gen_start", C.c_int), ("block_len", C.c_int)]
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_i, _f, _sz = C.c_int, C.c_float, C.c_size_t
+_status_string = _sig("dllm_status_string", C.c_char_p, [_i])
+_version = _sig("dllm_version", _i, [])
+_score = _sig("dllm_score", _i, [vp, vp, _i, _i, _i, _i, vp, vp, _i, _i, vp, vp, vp, _f, _i,
+                                 vp, vp])
+_select_ws = _sig("dllm_select_workspace_size", _sz, [_i, _i])
+_select = _sig("dllm_select", _i, [vp, _i, _i, _i, _i, _f, vp, vp, _i, vp, _sz, vp])
+_unmask = _sig("dllm_unmask", _i, [vp, vp, vp, _i, _i, _i, _i, _i, _i, vp, vp])
+_layer_ws = _sig("dllm_partial_layer_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i, _i])
+_layer = _sig("dllm_partial_layer", _i, [C.POINTER(ModelCfg), C.POINTER(LayerW), vp, _i, vp,
+                                         vp, vp, _i, _i, _i, vp, vp, vp, _sz, vp])
+_step_ws = _sig("dllm_step_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i,
+                                                  C.POINTER(Policy)])
+_step = _sig("dllm_step", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS), vp,
+                               _i, _i, C.POINTER(Policy), _i, vp, vp, vp, vp, vp, vp, vp, vp,
+                               _sz, vp])
+_devstat = _sig("dllm_get_device_status", _i, [vp, vp, C.POINTER(C.c_int32)])
+_gemm_ws = _sig("dllm_gemm_workspace_size", _sz, [_i, _i, _i, _i])
+_gemm = _sig("dllm_gemm_bf16", _i, [vp, vp, vp, _i, _i, _i, _i, _i, vp, _sz, vp])
+_prof_enable = _sig("dllm_profile_enable", None, [_i])
+_prof_reset = _sig("dllm_profile_reset", None, [])
+_prof_read = _sig("dllm_profile_read", _sz, [C.c_char_p, _sz])
+
+
+class DllmError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def status_string(st: int) -> str:
+    return _status_string(int(st)).decode()
+
+
+def version() -> int:
+    return int(_version())
+
+
+def _check(st: int, where: str):
+    if st != DLLM_OK:
+        raise DllmError(st, where)
+
+
+def ptr(t) -> Optional[int]:
+    """Device (or host) address of a tensor; None stays NULL."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return DLLM_BF16
+    if t.dtype == torch.float32:
+        return DLLM_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ----------------------------------------------------------------- workspace
+
+def _empty_bytes(nbytes: int, device):
+    import torch
+    # 256-byte alignment: torch's caching allocator returns at least 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+class Workspace:
+    """A caller-owned scratch buffer (torch memory) passed to the library."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.buf = _empty_bytes(nbytes, device)
+        self.buf[:256].zero_()
+        self.nbytes = self.buf.numel()
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def device_status(self, stream=None) -> int:
+        v = C.c_int32(0)
+        _devstat(self.ptr, _stream(stream), C.byref(v))
+        return int(v.value)
+
+
+# ----------------------------------------------------------------- thin calls
+
+def dllm_score(h_cur, h_ref, conf, masked, scores, alpha: float, kind: int = DLLM_SCORE_COS,
+               logits=None, logit_pos=None, pred=None, stream=None):
+    B, N, d = h_cur.shape
+    Mm = V = 0
+    if logits is not None:
+        _, Mm, V = logits.shape
+    st = _score(ptr(h_cur), ptr(h_ref), B, N, d, _dtype_code(h_cur), ptr(logits), ptr(logit_pos),
+                Mm, V, ptr(conf), ptr(pred), ptr(masked), float(alpha), int(kind), ptr(scores),
+                _stream(stream))
+    _check(st, "dllm_score")
+
+
+def dllm_select(scores, idx, count, mode: int, k: int, tau: float = 0.0, ws: Workspace = None,
+                stream=None):
+    B, N = scores.shape
+    k_cap = idx.shape[1]
+    st = _select(ptr(scores), B, N, int(mode), int(k), float(tau), ptr(idx), ptr(count), k_cap,
+                 ws.ptr if ws else None, ws.nbytes if ws else 0, _stream(stream))
+    _check(st, "dllm_select")
+
+
+def dllm_select_workspace_size(B: int, N: int) -> int:
+    return int(_select_ws(B, N))
+
+
+def dllm_unmask(conf, pred, tokens, mask_id: int, gen_start: int, block_len: int, n_unmask: int,
+                pos_out=None, stream=None):
+    B, N = tokens.shape
+    st = _unmask(ptr(conf), ptr(pred), ptr(tokens), B, N, int(mask_id), int(gen_start),
+                 int(block_len), int(n_unmask), ptr(pos_out), _stream(stream))
+    _check(st, "dllm_unmask")
+
+
+def dllm_gemm_workspace_size(M, N, K, splits=0) -> int:
+    return int(_gemm_ws(M, N, K, splits))
+
+
+def dllm_gemm_bf16(A, Bm, Cm, accumulate=False, splits=0, ws: Workspace = None, stream=None):
+    M, K = A.shape
+    N = Bm.shape[0]
+    if ws is None:
+        ws = Workspace(dllm_gemm_workspace_size(M, N, K, splits), A.device)
+    st = _gemm(ptr(A), ptr(Bm), ptr(Cm), M, N, K, int(bool(accumulate)), int(splits), ws.ptr,
+               ws.nbytes, _stream(stream))
+    _check(st, "dllm_gemm_bf16")
+    return ws
+
+
+def profile_enable(on: bool = True):
+    _prof_enable(int(bool(on)))
+
+
+def profile_reset():
+    _prof_reset()
+
+
+def profile_read() -> Dict[str, List[float]]:
+    n = _prof_read(None, 0)
+    buf = C.create_string_buffer(int(n))
+    _prof_read(buf, n)
+    return json.loads(buf.value.decode())
+
+
+# ----------------------------------------------------------------- model / cache
+
+def make_cfg(n_layers, d, n_heads, n_kv_heads, head_dim, ffn, vocab, rope_theta, rms_eps,
+             mask_id, dtype) -> ModelCfg:
+    return ModelCfg(n_layers, d, n_heads, n_kv_heads, head_dim, ffn, vocab, float(rope_theta),
+                    float(rms_eps), mask_id, DLLM_BF16 if dtype == "bf16" else DLLM_F32)
+
+
+def cfg_from_shape(s) -> ModelCfg:
+    return make_cfg(s.n_layers, s.d, s.n_heads, s.n_kv_heads, s.head_dim, s.ffn, s.vocab,
+                    s.rope_theta, s.rms_eps, s.mask_id, s.dtype)
+
+
+def layer_struct(L: Dict[str, object]) -> LayerW:
+    return LayerW(*(ptr(L[n]) for n in ("attn_norm", "wq", "wk", "wv", "wo", "ffn_norm",
+                                        "w_gate", "w_up", "w_down")))
+
+
+class Model:
+    """Weights (torch CUDA tensors, dict layout of ``dllm_synth.model_weights``) plus
+    the ctypes structs that point at them."""
+
+    def __init__(self, cfg: ModelCfg, W: Dict[str, object]):
+        self.cfg = cfg
+        self.W = W
+        n = len(W["layers"])
+        self._layers = (LayerW * max(n, 1))(*[layer_struct(L) for L in W["layers"]])
+        self.s = ModelW(ptr(W["embed"]), self._layers, ptr(W["final_norm"]), ptr(W["lm_head"]))
+
+    def layer(self, i: int) -> LayerW:
+        return self._layers[i]
+
+
+class Cache:
+    """Per-layer K/V caches, hidden reference, cached confidence and argmax (torch memory)."""
+
+    def __init__(self, cfg: ModelCfg, B: int, N: int, device="cuda"):
+        import torch
+        dt = torch.bfloat16 if cfg.dtype == DLLM_BF16 else torch.float32
+        kv = (B, N, cfg.n_kv_heads, cfg.head_dim)
+        self.k = [torch.zeros(kv, dtype=dt, device=device) for _ in range(cfg.n_layers)]
+        self.v = [torch.zeros(kv, dtype=dt, device=device) for _ in range(cfg.n_layers)]
+        self.h_ref = torch.zeros(B, N, cfg.d, dtype=dt, device=device)
+        self.conf = torch.zeros(B, N, dtype=torch.float32, device=device)
+        self.pred = torch.zeros(B, N, dtype=torch.int32, device=device)
+        self._refresh()
+
+    def _refresh(self):
+        L = max(len(self.k), 1)
+        self._kp = (vp * L)(*[ptr(t) for t in self.k])
+        self._vp = (vp * L)(*[ptr(t) for t in self.v])
+        self.s = CacheS(self._kp, self._vp, ptr(self.h_ref), ptr(self.conf), ptr(self.pred))
+
+
+def make_policy(score_layer=0, alpha=0.5, kind=DLLM_SCORE_COS, mode=DLLM_SELECT_TOPK, k=1,
+                tau=0.0, n_unmask=1, gen_start=0, block_len=32) -> Policy:
+    return Policy(score_layer, float(alpha), kind, mode, k, float(tau), n_unmask, gen_start,
+                  block_len)
+
+
+def dllm_partial_layer_workspace_size(cfg: ModelCfg, B: int, N: int, k_cap: int) -> int:
+    return int(_layer_ws(C.byref(cfg), B, N, k_cap))
+
+
+def dllm_partial_layer(cfg: ModelCfg, lw: LayerW, x_in, x_out, idx, count, k_cache, v_cache,
+                       ws: Workspace, x_in_is_full: bool, stream=None):
+    B, k_cap = idx.shape
+    N = k_cache.shape[1]
+    st = _layer(C.byref(cfg), C.byref(lw), ptr(x_in), int(bool(x_in_is_full)), ptr(x_out),
+                ptr(idx), ptr(count), k_cap, B, N, ptr(k_cache), ptr(v_cache), ws.ptr, ws.nbytes,
+                _stream(stream))
+    _check(st, "dllm_partial_layer")
+
+
+def dllm_step_workspace_size(cfg: ModelCfg, B: int, N: int, pol: Policy) -> int:
+    return int(_step_ws(C.byref(cfg), B, N, C.byref(pol)))
+
+
+def dllm_step(model: Model, cache: Cache, tokens, pol: Policy, dense: bool, ws: Workspace,
+              forced_idx=None, forced_count=None, forced_unmask_pos=None, idx_out=None,
+              count_out=None, pos_out=None, scores_out=None, stream=None):
+    B, N = tokens.shape
+    st = _step(C.byref(model.cfg), C.byref(model.s), C.byref(cache.s), ptr(tokens), B, N,
+               C.byref(pol), int(bool(dense)), ptr(forced_idx), ptr(forced_count),
+               ptr(forced_unmask_pos), ptr(idx_out), ptr(count_out), ptr(pos_out),
+               ptr(scores_out), ws.ptr, ws.nbytes, _stream(stream))
+    _check(st, "dllm_step")
+
+
+def dllm_step_host(model: Model, cache: Cache, tokens_host, pol: Policy, dense: bool,
+                   ws: Workspace, dev_tokens, dev_pos, pos_host, stream=None):
+    """One step from HOST token buffers: copies tokens in (pinned host -> device),
+    runs dllm_step, copies the updated tokens and revealed positions back."""
+    dev_tokens.copy_(tokens_host, non_blocking=True)
+    dllm_step(model, cache, dev_tokens, pol, dense, ws, pos_out=dev_pos, stream=stream)
+    tokens_host.copy_(dev_tokens, non_blocking=True)
+    pos_host.copy_(dev_pos, non_blocking=True)
+
+
+__all__ = [n for n in dir() if n.startswith(("dllm_", "DLLM_"))] + [
+    "Model", "Cache", "Workspace", "ModelCfg", "LayerW", "Policy", "make_cfg", "cfg_from_shape",
+    "make_policy", "profile_enable", "profile_reset", "profile_read", "status_string", "version",
+    "DllmError", "LIB_PATH"]

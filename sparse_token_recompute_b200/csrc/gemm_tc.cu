@@ -1,0 +1,691 @@
+// Tensor-core GEMM for the selected-row projections, sm_100a.
+//
+//   C[M, N] = A[M, K] * B[N, K]^T     bf16 operands, fp32 accumulation in TMEM
+//
+// A holds the compact (gathered) rows of the selected tokens, B a weight
+// matrix [out, in].  Structure:
+//   * persistent CTAs (one per SM), static round-robin over work units; a
+//     unit is (m-tile of 128 rows, n-tile of BN columns, K split);
+//   * warp 0: TMA producer (128-byte-swizzled boxes of 64 K-elements into a
+//     STAGES-deep ring, one mbarrier pair per stage);
+//   * warp 1: allocates TMEM and issues tcgen05.mma (M=128, N=BN, K=16) from
+//     a single thread; two accumulator buffers of BN fp32 columns so the
+//     epilogue of one unit overlaps the main loop of the next;
+//   * warps 2-5: epilogue, one TMEM lane quadrant each (thread = one row),
+//     fused per use: plain store, residual add, SwiGLU, RoPE + K/V cache
+//     scatter, or the LM-head online softmax statistics;
+//   * split-K units write fp32 partial tiles; the last unit of a tile (by an
+//     atomic ticket) adds the partials in split order, so the result does
+//     not depend on which CTA finishes last.
+// No TMA multicast is used anywhere.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dllm {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int NUM_THREADS = 192;
+constexpr int EPI_THREADS = 128;
+
+__host__ __device__ constexpr int stages_for(int bn) { return bn >= 256 ? 4 : (bn >= 128 ? 6 : 8); }
+__host__ __device__ constexpr int tmem_cols_for(int bn) { return 2 * bn < 32 ? 32 : 2 * bn; }
+__host__ __device__ constexpr size_t smem_bytes_for(int bn) {
+  return (size_t)stages_for(bn) * (BM * BK * 2 + bn * BK * 2) + 1024 + 256;
+}
+
+struct Params {
+  int M_cap;
+  const int* M_dev;
+  int N;  // output columns of the GEMM (SWIGLU: 2F)
+  int K;
+  int tiles_n;
+  int splits;
+  int kb_total;
+  int kb_per_split;
+  int seg0, seg1;  // column boundaries of B segments
+  __nv_bfloat16* out;
+  int ldo;
+  __nv_bfloat16* kc;
+  __nv_bfloat16* vc;
+  const int* row_pos;
+  const int* row_seq;
+  int Nseq;
+  int q_cols, kv_cols, hd;
+  const float2* rope;
+  float* lm_part;
+  int V;
+  float* partials;
+  int* counters;
+  int* status;
+};
+
+__device__ __forceinline__ void decode_unit(int u, int m_tiles, int tiles_n, int splits, int& m,
+                                            int& n, int& s) {
+  s = u % splits;
+  const int t = u / splits;
+  constexpr int G = 16;  // m-tiles per raster group: keeps A and B slices resident in L2
+  const int per_group = G * tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * G;
+  const int gsz = min(m_tiles - first_m, G);
+  const int r = t - g * per_group;
+  m = first_m + r % gsz;
+  n = r / gsz;
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// bounded wait that ignores the abort flag (used while draining after an abort)
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+// ---------------------------------------------------------------- epilogues
+// `ld(c, v)` fills v[0..31] with fp32 columns [c, c+32) of this thread's row
+// in the tile; every lane of the warp must call it (TMEM loads are warp-wide).
+
+template <int BN, int EPI, class Loader>
+__device__ __forceinline__ void epilogue_tile(const Params& p, int row, bool row_ok, int m, int n,
+                                              Loader&& ld) {
+  if constexpr (EPI == EPI_STORE || EPI == EPI_RESID) {
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      ld(c, v);
+      const int col = n * BN + c;
+      if (row_ok) {
+        __nv_bfloat16* o = p.out + (size_t)row * p.ldo + col;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          if (col + j < p.N) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = v[j + i];
+            if constexpr (EPI == EPI_RESID) {
+              float r[8];
+              unpack8(*reinterpret_cast<const uint4*>(o + j), r);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) f[i] += r[i];
+            }
+            *reinterpret_cast<uint4*>(o + j) = pack8(f);
+          }
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_SWIGLU) {
+    const int F = p.N >> 1;
+#pragma unroll 1
+    for (int c = 0; c < BN / 2; c += 32) {
+      float g[32], u[32];
+      ld(c, g);
+      ld(BN / 2 + c, u);
+      const int col = n * (BN / 2) + c;
+      if (row_ok) {
+        __nv_bfloat16* o = p.out + (size_t)row * p.ldo + col;
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          if (col + j < F) {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = silu_f(g[j + i]) * u[j + i];
+            *reinterpret_cast<uint4*>(o + j) = pack8(f);
+          }
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_QKV) {
+    const int n0 = n * BN;
+    int pos = 0, seq = 0;
+    if (row_ok) {
+      pos = p.row_pos[row];
+      seq = p.row_seq[row];
+    }
+    __nv_bfloat16* dst;
+    bool rot;
+    if (n0 < p.q_cols) {
+      dst = p.out + (size_t)row * p.ldo + n0;
+      rot = p.rope != nullptr;
+    } else if (n0 < p.q_cols + p.kv_cols) {
+      dst = p.kc + ((size_t)seq * p.Nseq + pos) * p.kv_cols + (n0 - p.q_cols);
+      rot = p.rope != nullptr;
+    } else {
+      dst = p.vc + ((size_t)seq * p.Nseq + pos) * p.kv_cols + (n0 - p.q_cols - p.kv_cols);
+      rot = false;
+    }
+    if (!rot) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        ld(c, v);
+        if (row_ok) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8)
+            *reinterpret_cast<uint4*>(dst + c + j) = pack8(v + j);
+        }
+      }
+    } else {
+      const int half = p.hd >> 1;
+#pragma unroll 1
+      for (int h0 = 0; h0 < BN; h0 += p.hd) {
+#pragma unroll 1
+        for (int c = 0; c < half; c += 32) {
+          float x1[32], x2[32];
+          ld(h0 + c, x1);
+          ld(h0 + half + c, x2);
+          if (row_ok) {
+            const float2* cs = p.rope + (size_t)pos * half + c;
+            float y1[32], y2[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float2 t = cs[i];
+              y1[i] = x1[i] * t.x - x2[i] * t.y;
+              y2[i] = x2[i] * t.x + x1[i] * t.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              *reinterpret_cast<uint4*>(dst + h0 + c + j) = pack8(y1 + j);
+              *reinterpret_cast<uint4*>(dst + h0 + half + c + j) = pack8(y2 + j);
+            }
+          }
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_LMHEAD) {
+    float mx = -INFINITY, sm = 0.0f;
+    int arg = 0;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      float v[32];
+      ld(c, v);
+      const int col0 = n * BN + c;
+      float cm = -INFINITY;
+      int ca = col0;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        if (col0 + i < p.V && v[i] > cm) {
+          cm = v[i];
+          ca = col0 + i;
+        }
+      }
+      const float nm = fmaxf(mx, cm);
+      if (nm != -INFINITY) {
+        sm = (mx == -INFINITY) ? 0.0f : sm * expf(mx - nm);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (col0 + i < p.V) sm += expf(v[i] - nm);
+      }
+      if (cm > mx) arg = ca;
+      mx = nm;
+    }
+    if (row_ok) {
+      float* o = p.lm_part + ((size_t)row * p.tiles_n + n) * 3;
+      o[0] = mx;
+      o[1] = sm;
+      o[2] = __int_as_float(arg);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- kernel
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ CUtensorMap tmB2, const Params p) {
+  constexpr int STAGES = stages_for(BN);
+  constexpr int A_BYTES = BM * BK * 2;
+  constexpr int B_BYTES = BN * BK * 2;
+  constexpr uint32_t TMEM_COLS = tmem_cols_for(BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain[1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_last = abort_flag + 1;
+  volatile int* epi_abort = abort_flag + 2;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  int M = p.M_cap;
+  if (p.M_dev) {
+    M = *p.M_dev;
+    if (M > p.M_cap || M < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, DEV_BAD_SHAPE);
+      M = M < 0 ? 0 : p.M_cap;
+    }
+  }
+  const int m_tiles = (M + BM - 1) / BM;
+  const int n_units = m_tiles * p.tiles_n * p.splits;
+
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * STAGES + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[2 * STAGES + 2 + a]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * STAGES + 4]);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), EPI_THREADS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *epi_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (EPI == EPI_SWIGLU || EPI == EPI_QKV) tma_prefetch_desc(&tmB1);
+    if (EPI == EPI_QKV) tma_prefetch_desc(&tmB2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0;
+      uint32_t issue_phase = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        int m, n, s;
+        decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
+        const int kb0 = s * p.kb_per_split;
+        const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), A_BYTES + B_BYTES);
+          const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
+          tma_load_2d(a_dst, &tmA, full_bar(stage), kb * BK, m * BM);
+          if constexpr (EPI == EPI_SWIGLU) {
+            tma_load_2d(b_dst, &tmB0, full_bar(stage), kb * BK, n * (BN / 2));
+            tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB1, full_bar(stage), kb * BK, n * (BN / 2));
+          } else if constexpr (EPI == EPI_QKV) {
+            const int n0 = n * BN;
+            if (n0 < p.seg0)
+              tma_load_2d(b_dst, &tmB0, full_bar(stage), kb * BK, n0);
+            else if (n0 < p.seg1)
+              tma_load_2d(b_dst, &tmB1, full_bar(stage), kb * BK, n0 - p.seg0);
+            else
+              tma_load_2d(b_dst, &tmB2, full_bar(stage), kb * BK, n0 - p.seg1);
+          } else {
+            tma_load_2d(b_dst, &tmB0, full_bar(stage), kb * BK, n * BN);
+          }
+          issued |= 1u << stage;
+          if (phase) issue_phase |= 1u << stage; else issue_phase &= ~(1u << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // drain: every load this thread issued must land before the block exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (issue_phase >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        int m, n, s;
+        decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
+        const int kb0 = s * p.kb_per_split;
+        const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_bf16(d_tmem, umma_desc_k_sw128(a_base + k * 32),
+                        umma_desc_k_sw128(b_base + k * 32), idesc,
+                        (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued_any) {
+        tc_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
+    const int r_in_tile = quad * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
+      int m, n, s;
+      decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
+      // warp-uniform outcome: TMEM loads below are warp-collective
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      if (p.splits > 1) {
+        // and block-uniform among the epilogue warps, which meet at named barriers
+        if (!ok) *epi_abort = 1;
+        named_bar_sync(1, EPI_THREADS);
+        if (*epi_abort) break;
+      } else if (!ok) {
+        break;
+      }
+      tc_fence_after();
+      const int row = m * BM + r_in_tile;
+      const bool row_ok = row < M;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      if (p.splits == 1) {
+        epilogue_tile<BN, EPI>(p, row, row_ok, m, n,
+                               [&](int c, float* v) { tmem_ld_32x32b_x32(t_row + c, v); });
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+      } else {
+        const int tile = m * p.tiles_n + n;
+        float* part = p.partials + (((size_t)tile * p.splits + s) * BM + r_in_tile) * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          tmem_ld_32x32b_x32(t_row + c, v);
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(part + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              __stcg(dst + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(tempty_bar(acc));
+        __threadfence();
+        named_bar_sync(1, EPI_THREADS);
+        if (threadIdx.x == 64) {
+          const int old = atomicAdd(&p.counters[tile], 1);
+          *s_last = (old == p.splits - 1) ? 1 : 0;
+        }
+        named_bar_sync(1, EPI_THREADS);
+        if (*s_last) {
+          __threadfence();
+          const float* base = p.partials + ((size_t)tile * p.splits * BM + r_in_tile) * BN;
+          epilogue_tile<BN, EPI>(p, row, row_ok, m, n, [&](int c, float* v) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            if (row_ok) {
+              for (int sp = 0; sp < p.splits; ++sp) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(base + (size_t)sp * BM * BN + c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const float4 t = __ldcg(src + i);
+                  v[4 * i] += t.x;
+                  v[4 * i + 1] += t.y;
+                  v[4 * i + 2] += t.z;
+                  v[4 * i + 3] += t.w;
+                }
+              }
+            }
+          });
+          if (threadIdx.x == 64) p.counters[tile] = 0;
+        }
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// [rows, cols] bf16 row-major, box (64 cols, box_rows rows), 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn || !ptr || rows <= 0 || cols <= 0) return false;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (cols % 8)) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                     const CUtensorMap& b2, const Params& p, int grid, cudaStream_t s) {
+  constexpr size_t smem = smem_bytes_for(BN);
+  static bool attr_set = false;  // per template instance; device-wide attribute
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  gemm_tc_kernel<BN, EPI><<<grid, NUM_THREADS, smem, s>>>(a, b0, b1, b2, p);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_bn(int bn, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                      const CUtensorMap& b2, const Params& p, int grid, cudaStream_t s) {
+  switch (bn) {
+    case 256: return launch_t<256, EPI>(a, b0, b1, b2, p, grid, s);
+    case 128: return launch_t<128, EPI>(a, b0, b1, b2, p, grid, s);
+    default: return launch_t<64, EPI>(a, b0, b1, b2, p, grid, s);
+  }
+}
+
+}  // namespace
+
+int gemm_total_cols(const GemmSpec& g) {
+  int n = 0;
+  for (int i = 0; i < g.n_seg; ++i) n += g.seg_cols[i];
+  return n;
+}
+
+GemmPlan gemm_plan(const GemmSpec& g) {
+  GemmPlan pl{};
+  const int N = gemm_total_cols(g);
+  const int kb_total = (g.K + BK - 1) / BK;
+  pl.m_tiles_cap = (g.M_cap + BM - 1) / BM;
+  const int sms = num_sms();
+  // candidate tile widths: every B segment (and, for QKV, every head) must tile evenly
+  auto bn_ok = [&](int bn) {
+    if (g.epi == EPI_SWIGLU) return (g.seg_cols[0] % (bn / 2)) == 0;
+    if (g.epi == EPI_QKV) {
+      for (int i = 0; i < g.n_seg; ++i)
+        if (g.seg_cols[i] % bn) return false;
+      return bn % g.hd == 0;
+    }
+    return true;
+  };
+  int bn = g.force_bn;
+  int splits = g.force_splits;
+  if (!bn) {
+    const int cands[3] = {256, 128, 64};
+    double best = 1e30;
+    for (int c : cands) {
+      if (!bn_ok(c)) continue;
+      if (g.epi == EPI_LMHEAD && c < 128) continue;  // stats buffers are sized for >= 128
+      const int tiles = pl.m_tiles_cap * ((N + c - 1) / c);
+      for (int sp = 1; sp <= 16; ++sp) {
+        if (g.epi == EPI_LMHEAD && sp > 1) break;
+        if (sp > 1 && kb_total / sp < 4) break;
+        const int units = tiles * sp;
+        const int waves = (units + sms - 1) / sms;
+        const int kb = (kb_total + sp - 1) / sp;
+        // time ~ waves * (mainloop per unit + fixed cost); wide tiles amortise the A reads
+        const double per_unit = (double)kb * (BM * 64.0 + c * 64.0) / 64.0 + 600.0;
+        double t = waves * per_unit;
+        if (sp > 1) t += 2.0 * (double)sp * std::min(g.M_cap, BM * pl.m_tiles_cap) * c / sms * 0.05;
+        if (t < best * 0.999) {
+          best = t;
+          bn = c;
+          splits = sp;
+        }
+      }
+    }
+    if (!bn) bn = 64;
+  }
+  if (!splits) splits = 1;
+  if (splits > kb_total) splits = kb_total;
+  {
+    // no split may be empty: an empty split would publish a stale accumulator
+    const int per = (kb_total + splits - 1) / splits;
+    splits = (kb_total + per - 1) / per;
+  }
+  pl.bn = bn;
+  pl.splits = splits;
+  pl.tiles_n = (g.epi == EPI_SWIGLU) ? (N / 2 + bn / 2 - 1) / (bn / 2) : (N + bn - 1) / bn;
+  pl.units_cap = pl.m_tiles_cap * pl.tiles_n * pl.splits;
+  pl.grid = std::max(1, std::min(pl.units_cap, sms));
+  pl.partial_bytes =
+      splits > 1 ? (size_t)pl.m_tiles_cap * pl.tiles_n * splits * BM * bn * sizeof(float) : 0;
+  pl.counter_bytes = splits > 1 ? (size_t)pl.m_tiles_cap * pl.tiles_n * sizeof(int) : 0;
+  return pl;
+}
+
+cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
+  if (g.M_cap <= 0) return cudaSuccess;
+  const GemmPlan pl = gemm_plan(g);
+  const int N = gemm_total_cols(g);
+  Params p{};
+  p.M_cap = g.M_cap;
+  p.M_dev = g.M_dev;
+  p.N = N;
+  p.K = g.K;
+  p.tiles_n = pl.tiles_n;
+  p.splits = pl.splits;
+  p.kb_total = (g.K + BK - 1) / BK;
+  p.kb_per_split = (p.kb_total + pl.splits - 1) / pl.splits;
+  p.seg0 = g.seg_cols[0];
+  p.seg1 = g.seg_cols[0] + (g.n_seg > 1 ? g.seg_cols[1] : 0);
+  p.out = g.out;
+  p.ldo = g.ldo;
+  p.kc = g.kc;
+  p.vc = g.vc;
+  p.row_pos = g.row_pos;
+  p.row_seq = g.row_seq;
+  p.Nseq = g.Nseq;
+  p.q_cols = g.seg_cols[0];
+  p.kv_cols = g.n_seg > 1 ? g.seg_cols[1] : 0;
+  p.hd = g.hd;
+  p.rope = g.rope;
+  p.lm_part = g.lm_part;
+  p.V = N;
+  p.partials = g.partials;
+  p.counters = g.counters;
+  p.status = g.status;
+  if (pl.splits > 1 && (!g.partials || !g.counters)) return cudaErrorInvalidValue;
+
+  CUtensorMap ta, tb0, tb1, tb2;
+  if (!make_map(&ta, g.A, g.M_cap, g.K, BM)) return cudaErrorInvalidValue;
+  const int bbox = (g.epi == EPI_SWIGLU) ? pl.bn / 2 : pl.bn;
+  if (!make_map(&tb0, g.B[0], g.seg_cols[0], g.K, bbox)) return cudaErrorInvalidValue;
+  tb1 = tb0;
+  tb2 = tb0;
+  if (g.n_seg > 1 && !make_map(&tb1, g.B[1], g.seg_cols[1], g.K, bbox)) return cudaErrorInvalidValue;
+  if (g.n_seg > 2 && !make_map(&tb2, g.B[2], g.seg_cols[2], g.K, bbox)) return cudaErrorInvalidValue;
+
+  static const char* names[5] = {"gemm_store", "gemm_resid", "gemm_swiglu", "gemm_qkv",
+                                 "gemm_lmhead"};
+  ProfScope prof(names[g.epi], s);
+  switch (g.epi) {
+    case EPI_STORE: return launch_bn<EPI_STORE>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);
+    case EPI_RESID: return launch_bn<EPI_RESID>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);
+    case EPI_SWIGLU: return launch_bn<EPI_SWIGLU>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);
+    case EPI_QKV: return launch_bn<EPI_QKV>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);
+    case EPI_LMHEAD: return launch_bn<EPI_LMHEAD>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace dllm

@@ -1,0 +1,139 @@
+// Internal launchers shared by the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace dllm {
+
+int num_sms();
+cudaError_t last_error();
+
+// ----- kernel timing (dllm_profile_*) -----
+void prof_begin(const char* name, cudaStream_t s);
+void prof_end(cudaStream_t s);
+struct ProfScope {
+  cudaStream_t s;
+  ProfScope(const char* name, cudaStream_t st) : s(st) { prof_begin(name, st); }
+  ~ProfScope() { prof_end(s); }
+};
+
+// ----- tcgen05 GEMM -----
+enum EpiKind { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_LMHEAD = 4 };
+
+struct GemmSpec {
+  int epi;
+  // A [M_cap, K] bf16 row-major; rows >= *M_dev are ignored
+  const __nv_bfloat16* A;
+  int M_cap;
+  const int* M_dev;  // may be null: M = M_cap
+  int K;
+  // B segments: columns [0, seg_cols[0]) from B[0], then B[1], then B[2]; each [cols, K].
+  // SWIGLU: B[0] = gate [F, K], B[1] = up [F, K]; output width F.
+  const __nv_bfloat16* B[3];
+  int seg_cols[3];
+  int n_seg;
+  // STORE / RESID / SWIGLU output, QKV query output
+  __nv_bfloat16* out;
+  int ldo;
+  // QKV
+  __nv_bfloat16* kc;
+  __nv_bfloat16* vc;
+  const int* row_pos;
+  const int* row_seq;
+  int Nseq;
+  int hd;
+  const float2* rope;  // [Nseq, hd/2] (cos, sin), null: no rotation
+  // LMHEAD partial softmax stats [M_cap, n_tiles] x (max, sum, argmax)
+  float* lm_part;
+  int lm_tiles;  // out: number of column tiles (set by plan)
+  // split-K scratch
+  float* partials;
+  int* counters;
+  int* status;
+  int force_bn;      // 0: choose
+  int force_splits;  // 0: choose
+};
+
+struct GemmPlan {
+  int bn, splits, tiles_n, m_tiles_cap, units_cap, grid;
+  size_t partial_bytes, counter_bytes;
+};
+
+int gemm_total_cols(const GemmSpec& g);
+GemmPlan gemm_plan(const GemmSpec& g);
+cudaError_t gemm_launch(GemmSpec g, cudaStream_t s);
+
+// ----- row bookkeeping, gather, norms -----
+// row_off[B+1], row_pos[cap], row_seq[cap] from idx [B, k_cap] / count [B]; M_dev = row_off[B]
+void launch_row_map(const int32_t* idx, const int32_t* count, int B, int k_cap, int N,
+                    int* row_off, int* row_pos, int* row_seq, int* status, cudaStream_t s);
+// identity map (all N rows of every sequence)
+void launch_row_map_dense(int B, int N, int* row_off, int* row_pos, int* row_seq,
+                          cudaStream_t s);
+// x[r] = src row (b, pos) where src is [B,N,d] (or embed[tokens] when tokens != null);
+// also h_ref[b,pos] = x[r] when h_ref != null
+template <typename T>
+void launch_gather_rows(const T* src_full, const T* embed, const int32_t* tokens,
+                        const int* row_pos, const int* row_seq, const int* M_dev, int M_cap,
+                        int N, int d, T* x, T* h_ref, int vocab, int* status, cudaStream_t s);
+template <typename T>
+void launch_rmsnorm(const T* x, const T* g, T* out, const int* M_dev, int M_cap, int d, float eps,
+                    cudaStream_t s);
+// final norm on the masked subset: lm_rows[j] = compact row, writes out[j]
+template <typename T>
+void launch_rmsnorm_rows(const T* x, const T* g, T* out, const int* rows, const int* n_rows,
+                         int cap, int d, float eps, cudaStream_t s);
+void launch_rope_table(float2* table, int N, int hd, float theta, cudaStream_t s);
+// lm_rows: compact rows whose (b,pos) token is masked; n_lm = their count
+void launch_masked_rows(const int32_t* tokens, int mask_id, const int* row_pos,
+                        const int* row_seq, const int* M_dev, int M_cap, int N, int* lm_rows,
+                        int* n_lm, cudaStream_t s);
+void launch_lm_merge(const float* lm_part, int tiles, const int* lm_rows, const int* n_lm,
+                     int cap, const int* row_pos, const int* row_seq, int N, float* conf,
+                     int32_t* pred, cudaStream_t s);
+
+// ----- fp32 (DLLM_F32) layer pieces -----
+void launch_gemm_f32(const float* A, const float* B, float* C, const float* R, const int* M_dev,
+                     int M_cap, int N, int K, cudaStream_t s);  // C = A B^T (+ R)
+void launch_qkv_post_f32(const float* q_raw, const float* k_raw, const float* v_raw,
+                         float* q_out, float* kc, float* vc, const int* row_pos,
+                         const int* row_seq, const int* M_dev, int M_cap, int Nseq, int Hq,
+                         int Hkv, int hd, const float2* rope, cudaStream_t s);
+void launch_swiglu_f32(const float* g, const float* u, float* a, const int* M_dev, int M_cap,
+                       int F, cudaStream_t s);
+void launch_attention_f32(const float* q, const float* kc, const float* vc, float* o,
+                          const int* row_seq, const int* M_dev, int M_cap, int Nseq, int Hq,
+                          int Hkv, int hd, cudaStream_t s);
+void launch_confidence_rows_f32(const float* logits, int V, const int* lm_rows, const int* n_lm,
+                                int cap, const int* row_pos, const int* row_seq, int N,
+                                float* conf, int32_t* pred, cudaStream_t s);
+
+// ----- bf16 attention -----
+void launch_attention_bf16(const __nv_bfloat16* q, const __nv_bfloat16* kc,
+                           const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
+                           int B, int k_cap, int Nseq, int Hq, int Hkv, int hd,
+                           cudaStream_t s);
+
+// ----- score / select / unmask -----
+template <typename T>
+void launch_confidence(const T* logits, const int32_t* logit_pos, int B, int Mm, int V, int N,
+                       float* conf, int32_t* pred, cudaStream_t s);
+// h row i = tokens ? embed[tokens[i]] : h_cur[i]; masked flag from `masked` or, when that
+// is null, from mask_tokens[i] == mask_id (no flag when both are null)
+template <typename T>
+void launch_score(const T* h_cur, const T* embed, const int32_t* tokens, const T* h_ref, int B,
+                  int N, int d, const float* conf, const uint8_t* masked,
+                  const int32_t* mask_tokens, int mask_id, float alpha, int kind, float* scores,
+                  int vocab, int* status, cudaStream_t s);
+void launch_select(const float* scores, int B, int N, int mode, int k, float tau, int32_t* idx,
+                   int32_t* count, int k_cap, int* status, cudaStream_t s);
+void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
+                   int mask_id, int gen_start, int block_len, int n_unmask, int32_t* pos_out,
+                   const int32_t* forced, cudaStream_t s);
+void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
+                     int32_t* dst_count, int B, int k_cap, cudaStream_t s);
+
+}  // namespace dllm

@@ -1,0 +1,1042 @@
+// Memory-bound and bookkeeping kernels of the selected-token step (sm_100a):
+// importance scores, max-softmax confidence, radix top-k / threshold
+// compaction, confidence unmasking, compact-row bookkeeping, gather with the
+// hidden-reference scatter, RMSNorm, the RoPE table, the LM-head merge, and
+// the fp32 pieces of the layer for DLLM_F32 models.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace dllm {
+
+namespace {
+
+// ---------------------------------------------------------------- block scan helpers
+
+// inclusive scan of one int per thread across the block (blockDim.x <= 1024)
+__device__ int block_inclusive_scan(int v, int* warp_tot) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) warp_tot[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += u;
+    }
+    if (lane < nw) warp_tot[lane] = t;  // inclusive totals per warp
+  }
+  __syncthreads();
+  const int add = w > 0 ? warp_tot[w - 1] : 0;
+  const int r = v + add;
+  __syncthreads();  // warp_tot may be reused by the caller
+  return r;
+}
+
+__device__ int block_sum_int(int v, int* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  int t = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nw; ++i) t += red[i];
+    red[32] = t;
+  }
+  __syncthreads();
+  t = red[32];
+  __syncthreads();
+  return t;
+}
+
+__device__ int block_min_int(int v, int* red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = red[0];
+    for (int i = 1; i < nw; ++i) t = min(t, red[i]);
+    red[32] = t;
+  }
+  __syncthreads();
+  const int r = red[32];
+  __syncthreads();
+  return r;
+}
+
+// Order-preserving key of a float for "larger first": NaN -> 0 (below all),
+// -0 -> +0, otherwise the standard sign-flip mapping (-inf -> 0x007FFFFF).
+__device__ __forceinline__ uint32_t order_key(float x) {
+  if (isnan(x)) return 0u;
+  if (x == 0.0f) x = 0.0f;
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------- score
+
+template <typename T>
+__device__ __forceinline__ void load_vec8(const T* p, float* f);
+template <>
+__device__ __forceinline__ void load_vec8<__nv_bfloat16>(const __nv_bfloat16* p, float* f) {
+  unpack8(__ldg(reinterpret_cast<const uint4*>(p)), f);
+}
+template <>
+__device__ __forceinline__ void load_vec8<float>(const float* p, float* f) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+// One warp per row.  Accumulates |h|^2, |r|^2, |h-r|^2, |h-r|_1 and bitwise
+// equality; 1 - cos is evaluated as (|h-r|^2 - (|h|-|r|)^2) / (2 |h| |r|),
+// which equals 1 - h.r/(|h||r|) and stays accurate when the rows are close.
+template <typename T>
+__global__ void __launch_bounds__(256) score_kernel(const T* __restrict__ h_cur,
+                                                    const T* __restrict__ embed,
+                                                    const int32_t* __restrict__ tokens,
+                                                    const T* __restrict__ h_ref, int rows, int N,
+                                                    int d, const float* __restrict__ conf,
+                                                    const uint8_t* __restrict__ masked,
+                                                    const int32_t* __restrict__ mask_tokens,
+                                                    int mask_id, float alpha, int kind,
+                                                    float* __restrict__ scores, int vocab,
+                                                    int* status) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const T* hc;
+  if (tokens) {
+    int t = tokens[row];
+    if (t < 0 || t >= vocab) {
+      if (lane == 0) raise_status(status, DEV_BAD_INDEX);
+      t = t < 0 ? 0 : vocab - 1;
+    }
+    hc = embed + (size_t)t * d;
+  } else {
+    hc = h_cur + (size_t)row * d;
+  }
+  const T* hr = h_ref + (size_t)row * d;
+  float nc = 0.f, nr = 0.f, dd = 0.f, l1 = 0.f;
+  int eq = 1;
+  for (int i = lane * 8; i < d; i += 32 * 8) {
+    float a[8], b[8];
+    load_vec8<T>(hc + i, a);
+    load_vec8<T>(hr + i, b);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float df = a[j] - b[j];
+      nc = fmaf(a[j], a[j], nc);
+      nr = fmaf(b[j], b[j], nr);
+      dd = fmaf(df, df, dd);
+      l1 += fabsf(df);
+      eq &= (__float_as_uint(a[j]) == __float_as_uint(b[j]));
+    }
+  }
+  nc = warp_sum(nc);
+  nr = warp_sum(nr);
+  dd = warp_sum(dd);
+  l1 = warp_sum(l1);
+  eq = warp_and(eq);
+  if (lane == 0) {
+    float v;
+    if (eq) {
+      v = 0.0f;
+    } else if (kind == DLLM_SCORE_COS) {
+      const float a = sqrtf(nc), b = sqrtf(nr);
+      const float nn = a * b;
+      if (nn > 0.0f) {
+        const float t = a - b;
+        v = (dd - t * t) / (2.0f * nn);
+        v = fminf(fmaxf(v, 0.0f), 2.0f);
+      } else {
+        v = 1.0f;
+      }
+    } else {
+      v = nr > 0.0f ? l1 / (sqrtf((float)d) * sqrtf(nr)) : INFINITY;
+    }
+    const bool is_m =
+        masked ? (masked[row] != 0) : (mask_tokens ? mask_tokens[row] == mask_id : false);
+    const float c = is_m ? conf[row] : 0.0f;
+    scores[row] = alpha * c + (1.0f - alpha) * v;
+  }
+}
+
+// ---------------------------------------------------------------- confidence
+
+struct SoftStat {
+  float m, s;
+  int a;
+};
+__device__ __forceinline__ SoftStat soft_merge(SoftStat x, SoftStat y) {
+  SoftStat r;
+  r.m = fmaxf(x.m, y.m);
+  if (r.m == -INFINITY) {
+    r.s = 0.f;
+  } else {
+    r.s = (x.m == -INFINITY ? 0.f : x.s * expf(x.m - r.m)) +
+          (y.m == -INFINITY ? 0.f : y.s * expf(y.m - r.m));
+  }
+  r.a = (x.m > y.m) ? x.a : ((y.m > x.m) ? y.a : min(x.a, y.a));
+  return r;
+}
+
+// statistics of one logits row, block-wide (256 threads)
+template <typename T>
+__device__ SoftStat row_softstat(const T* z, int V, SoftStat* red) {
+  SoftStat st{-INFINITY, 0.f, 0x7fffffff};
+  for (int i = threadIdx.x * 8; i < V; i += blockDim.x * 8) {
+    float f[8];
+    load_vec8<T>(z + i, f);
+    float cm = f[0];
+    int ca = i;
+#pragma unroll
+    for (int j = 1; j < 8; ++j)
+      if (f[j] > cm) {
+        cm = f[j];
+        ca = i + j;
+      }
+    const float nm = fmaxf(st.m, cm);
+    float s = (st.m == -INFINITY) ? 0.f : st.s * expf(st.m - nm);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += expf(f[j] - nm);
+    st.a = (cm > st.m) ? ca : st.a;
+    st.m = nm;
+    st.s = s;
+  }
+  // warp merge
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    SoftStat y;
+    y.m = __shfl_xor_sync(0xffffffffu, st.m, o);
+    y.s = __shfl_xor_sync(0xffffffffu, st.s, o);
+    y.a = __shfl_xor_sync(0xffffffffu, st.a, o);
+    st = soft_merge(st, y);
+  }
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = st;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    SoftStat t = red[0];
+    for (int i = 1; i < nw; ++i) t = soft_merge(t, red[i]);
+    red[32] = t;
+  }
+  __syncthreads();
+  const SoftStat r = red[32];
+  __syncthreads();
+  return r;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) confidence_kernel(const T* __restrict__ logits,
+                                                         const int32_t* __restrict__ logit_pos,
+                                                         int Mm, int V, int N,
+                                                         float* __restrict__ conf,
+                                                         int32_t* __restrict__ pred) {
+  __shared__ SoftStat red[33];
+  const int r = blockIdx.x;  // b * Mm + j
+  const int b = r / Mm;
+  const SoftStat st = row_softstat<T>(logits + (size_t)r * V, V, red);
+  if (threadIdx.x == 0) {
+    const int p = logit_pos[r];
+    if (p >= 0 && p < N) {
+      conf[(size_t)b * N + p] = 1.0f / st.s;
+      if (pred) pred[(size_t)b * N + p] = st.a;
+    }
+  }
+}
+
+// logits [cap, V] fp32 of the LM rows (DLLM_F32 models)
+__global__ void __launch_bounds__(256) confidence_rows_f32_kernel(
+    const float* __restrict__ logits, int V, const int* __restrict__ lm_rows,
+    const int* __restrict__ n_lm, const int* __restrict__ row_pos,
+    const int* __restrict__ row_seq, int N, float* __restrict__ conf,
+    int32_t* __restrict__ pred) {
+  __shared__ SoftStat red[33];
+  const int j = blockIdx.x;
+  if (j >= *n_lm) return;
+  const SoftStat st = row_softstat<float>(logits + (size_t)j * V, V, red);
+  if (threadIdx.x == 0) {
+    const int r = lm_rows[j];
+    const size_t o = (size_t)row_seq[r] * N + row_pos[r];
+    conf[o] = 1.0f / st.s;
+    pred[o] = st.a;
+  }
+}
+
+// merge of the per-tile statistics written by the LM-head GEMM epilogue
+__global__ void __launch_bounds__(128) lm_merge_kernel(const float* __restrict__ part, int tiles,
+                                                       const int* __restrict__ lm_rows,
+                                                       const int* __restrict__ n_lm, int cap,
+                                                       const int* __restrict__ row_pos,
+                                                       const int* __restrict__ row_seq, int N,
+                                                       float* __restrict__ conf,
+                                                       int32_t* __restrict__ pred) {
+  const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= *n_lm || j >= cap) return;
+  const float* p = part + (size_t)j * tiles * 3;
+  SoftStat st{-INFINITY, 0.f, 0x7fffffff};
+  for (int t = lane; t < tiles; t += 32) {
+    SoftStat y{p[3 * t], p[3 * t + 1], __float_as_int(p[3 * t + 2])};
+    st = soft_merge(st, y);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    SoftStat y;
+    y.m = __shfl_xor_sync(0xffffffffu, st.m, o);
+    y.s = __shfl_xor_sync(0xffffffffu, st.s, o);
+    y.a = __shfl_xor_sync(0xffffffffu, st.a, o);
+    st = soft_merge(st, y);
+  }
+  if (lane == 0) {
+    const int r = lm_rows[j];
+    const size_t o = (size_t)row_seq[r] * N + row_pos[r];
+    conf[o] = 1.0f / st.s;
+    pred[o] = st.a;
+  }
+}
+
+// ---------------------------------------------------------------- select
+
+constexpr int SEL_THREADS = 1024;
+constexpr int SEL_MAX_PER_THREAD = 16;  // N <= 16384
+
+__global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __restrict__ scores,
+                                                             int N, int mode, int k, float tau,
+                                                             int32_t* __restrict__ idx,
+                                                             int32_t* __restrict__ count,
+                                                             int k_cap, int* status) {
+  __shared__ int hist[256];
+  __shared__ int red[33];
+  __shared__ int s_digit, s_above;
+  const int b = blockIdx.x;
+  const float* sc = scores + (size_t)b * N;
+  const int E = (N + SEL_THREADS - 1) / SEL_THREADS;
+  const int i0 = threadIdx.x * E;  // contiguous chunk keeps position order for the scans
+  uint32_t key[SEL_MAX_PER_THREAD];
+  int n_cand = 0;
+#pragma unroll
+  for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
+    key[e] = 0u;
+    if (e < E && i0 + e < N) {
+      const float x = sc[i0 + e];
+      if (mode == DLLM_SELECT_TOPK) {
+        key[e] = order_key(x);
+        ++n_cand;
+      } else if (x > tau) {  // NaN compares false
+        key[e] = order_key(x);
+        ++n_cand;
+      }
+    }
+  }
+  int total = block_sum_int(n_cand, red);
+  int keff;
+  if (mode == DLLM_SELECT_TOPK) {
+    keff = min(min(k, N), k_cap);
+  } else {
+    keff = min(total, k_cap);
+    if (total > k_cap && threadIdx.x == 0) raise_status(status, DEV_CAPACITY);
+  }
+  if (keff <= 0) {
+    if (threadIdx.x == 0) count[b] = 0;
+    return;
+  }
+  // radix select of the keff-th largest key, 8 bits per pass from the top
+  uint32_t prefix = 0u, pmask = 0u;
+  int remaining = keff;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
+      if (e < E && i0 + e < N) {
+        const bool cand = (mode == DLLM_SELECT_TOPK) || key[e] != 0u;
+        if (cand && (key[e] & pmask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int above = 0, dg = 0;
+      for (int bin = 255; bin >= 0; --bin) {
+        if (above + hist[bin] >= remaining) {
+          dg = bin;
+          break;
+        }
+        above += hist[bin];
+      }
+      s_digit = dg;
+      s_above = above;
+    }
+    __syncthreads();
+    remaining -= s_above;
+    prefix |= (uint32_t)s_digit << shift;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;  // keff-th largest key; take `remaining` ties, lowest positions first
+  int n_tie = 0;
+#pragma unroll
+  for (int e = 0; e < SEL_MAX_PER_THREAD; ++e)
+    if (e < E && i0 + e < N) {
+      const bool cand = (mode == DLLM_SELECT_TOPK) || key[e] != 0u;
+      n_tie += (cand && key[e] == T) ? 1 : 0;
+    }
+  const int tie_incl = block_inclusive_scan(n_tie, red);
+  int tie_rank = tie_incl - n_tie;
+  bool sel[SEL_MAX_PER_THREAD];
+  int n_sel = 0;
+#pragma unroll
+  for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
+    sel[e] = false;
+    if (e < E && i0 + e < N) {
+      const bool cand = (mode == DLLM_SELECT_TOPK) || key[e] != 0u;
+      if (cand && key[e] > T) {
+        sel[e] = true;
+      } else if (cand && key[e] == T) {
+        sel[e] = tie_rank < remaining;
+        ++tie_rank;
+      }
+      n_sel += sel[e] ? 1 : 0;
+    }
+  }
+  const int sel_incl = block_inclusive_scan(n_sel, red);
+  int o = sel_incl - n_sel;
+  int32_t* out = idx + (size_t)b * k_cap;
+#pragma unroll
+  for (int e = 0; e < SEL_MAX_PER_THREAD; ++e)
+    if (sel[e]) out[o++] = i0 + e;
+  if (threadIdx.x == blockDim.x - 1) count[b] = sel_incl;
+}
+
+// ---------------------------------------------------------------- unmask
+
+__global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ conf,
+                                                      const int32_t* __restrict__ pred,
+                                                      int32_t* __restrict__ tokens, int N,
+                                                      int mask_id, int gen_start, int block_len,
+                                                      int n_unmask, int32_t* __restrict__ pos_out,
+                                                      const int32_t* __restrict__ forced) {
+  __shared__ int red[33];
+  __shared__ uint32_t skey[1024];
+  __shared__ unsigned char smask[1024];
+  const int b = blockIdx.x;
+  int32_t* tk = tokens + (size_t)b * N;
+  const float* cf = conf + (size_t)b * N;
+  const int32_t* pr = pred + (size_t)b * N;
+  int32_t* po = pos_out ? pos_out + (size_t)b * n_unmask : nullptr;
+  if (forced) {
+    for (int j = threadIdx.x; j < n_unmask; j += blockDim.x) {
+      const int p = forced[(size_t)b * n_unmask + j];
+      if (p >= 0 && p < N) tk[p] = pr[p];
+      if (po) po[j] = (p >= 0 && p < N) ? p : -1;
+    }
+    return;
+  }
+  int first = N;
+  for (int p = gen_start + threadIdx.x; p < N; p += blockDim.x)
+    if (tk[p] == mask_id) first = min(first, p);
+  first = block_min_int(first, red);
+  if (first >= N || n_unmask <= 0) {
+    if (po)
+      for (int j = threadIdx.x; j < n_unmask; j += blockDim.x) po[j] = -1;
+    return;
+  }
+  const int blk = gen_start + ((first - gen_start) / block_len) * block_len;
+  const int L = min(block_len, N - blk);
+  const int t = threadIdx.x;
+  bool is_m = false;
+  uint32_t mykey = 0u;
+  if (t < L) {
+    is_m = tk[blk + t] == mask_id;
+    mykey = order_key(cf[blk + t]);
+    skey[t] = mykey;
+    smask[t] = is_m ? 1 : 0;
+  }
+  __syncthreads();
+  bool sel = false;
+  if (t < L && is_m) {
+    int rank = 0;
+    for (int j = 0; j < L; ++j) {
+      if (!smask[j]) continue;
+      const uint32_t kj = skey[j];
+      rank += (kj > mykey || (kj == mykey && j < t)) ? 1 : 0;
+    }
+    sel = rank < n_unmask;
+  }
+  const int incl = block_inclusive_scan(sel ? 1 : 0, red);
+  __shared__ int s_total;
+  if (threadIdx.x == blockDim.x - 1) s_total = incl;
+  __syncthreads();
+  if (sel) {
+    const int p = blk + t;
+    tk[p] = pr[p];
+    if (po) po[incl - 1] = p;
+  }
+  if (po)
+    for (int j = s_total + threadIdx.x; j < n_unmask; j += blockDim.x) po[j] = -1;
+}
+
+// ---------------------------------------------------------------- row bookkeeping
+
+__global__ void __launch_bounds__(1024) row_map_kernel(const int32_t* __restrict__ idx,
+                                                       const int32_t* __restrict__ count, int B,
+                                                       int k_cap, int N, int* __restrict__ row_off,
+                                                       int* __restrict__ row_pos,
+                                                       int* __restrict__ row_seq, int* status) {
+  __shared__ int red[33];
+  __shared__ int s_carry;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+    const int b = b0 + threadIdx.x;
+    int c = 0;
+    if (b < B) {
+      c = count[b];
+      if (c < 0 || c > k_cap) {
+        raise_status(status, DEV_CAPACITY);
+        c = c < 0 ? 0 : k_cap;
+      }
+    }
+    const int incl = block_inclusive_scan(c, red);
+    const int carry = s_carry;
+    if (b < B) row_off[b] = carry + incl - c;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) s_carry = carry + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) row_off[B] = s_carry;
+  __syncthreads();
+  for (int b = 0; b < B; ++b) {
+    int c = count[b];
+    c = c < 0 ? 0 : (c > k_cap ? k_cap : c);
+    const int off = row_off[b];
+    for (int j = threadIdx.x; j < c; j += blockDim.x) {
+      int p = idx[(size_t)b * k_cap + j];
+      const bool bad = p < 0 || p >= N || (j > 0 && idx[(size_t)b * k_cap + j - 1] >= p);
+      if (bad) {
+        raise_status(status, DEV_BAD_INDEX);
+        p = p < 0 ? 0 : (p >= N ? N - 1 : p);
+      }
+      row_pos[off + j] = p;
+      row_seq[off + j] = b;
+    }
+  }
+}
+
+__global__ void row_map_dense_kernel(int B, int N, int* row_off, int* row_pos, int* row_seq) {
+  const size_t total = (size_t)B * N;
+  for (size_t r = blockIdx.x * (size_t)blockDim.x + threadIdx.x; r < total;
+       r += (size_t)gridDim.x * blockDim.x) {
+    row_pos[r] = (int)(r % N);
+    row_seq[r] = (int)(r / N);
+  }
+  if (blockIdx.x == 0)
+    for (int b = threadIdx.x; b <= B; b += blockDim.x) row_off[b] = b * N;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) gather_rows_kernel(
+    const T* __restrict__ src_full, const T* __restrict__ embed,
+    const int32_t* __restrict__ tokens, const int* __restrict__ row_pos,
+    const int* __restrict__ row_seq, const int* __restrict__ M_dev, int M_cap, int N, int d,
+    T* __restrict__ x, T* __restrict__ h_ref, int vocab, int* status) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  const size_t src_row = (size_t)row_seq[r] * N + row_pos[r];
+  const T* src;
+  if (tokens) {
+    int t = tokens[src_row];
+    if (t < 0 || t >= vocab) {
+      if (lane == 0) raise_status(status, DEV_BAD_INDEX);
+      t = t < 0 ? 0 : vocab - 1;
+    }
+    src = embed + (size_t)t * d;
+  } else {
+    src = src_full + src_row * d;
+  }
+  constexpr int VEC = 16 / sizeof(T);
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* x4 = reinterpret_cast<uint4*>(x + (size_t)r * d);
+  uint4* h4 = h_ref ? reinterpret_cast<uint4*>(h_ref + src_row * d) : nullptr;
+  for (int i = lane; i < d / VEC; i += 32) {
+    const uint4 v = __ldg(s4 + i);
+    x4[i] = v;
+    if (h4) h4[i] = v;
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void rmsnorm_row(const T* __restrict__ x, const T* __restrict__ g,
+                                            T* __restrict__ o, int d, float eps) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+  for (int i = lane * 8; i < d; i += 256) {
+    float f[8];
+    load_vec8<T>(x + i, f);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+  }
+  ss = warp_sum(ss);
+  const float s = rsqrtf(ss / (float)d + eps);
+  for (int i = lane * 8; i < d; i += 256) {
+    float f[8], w[8];
+    load_vec8<T>(x + i, f);
+    load_vec8<T>(g + i, w);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) f[j] = f[j] * s * w[j];
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint4*>(o + i) = pack8(f);
+    } else {
+      float4* o4 = reinterpret_cast<float4*>(o + i);
+      o4[0] = make_float4(f[0], f[1], f[2], f[3]);
+      o4[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x,
+                                                      const T* __restrict__ g, T* __restrict__ o,
+                                                      const int* __restrict__ M_dev, int M_cap,
+                                                      int d, float eps) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  rmsnorm_row<T>(x + (size_t)r * d, g, o + (size_t)r * d, d, eps);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const T* __restrict__ x,
+                                                           const T* __restrict__ g,
+                                                           T* __restrict__ o,
+                                                           const int* __restrict__ rows,
+                                                           const int* __restrict__ n_rows,
+                                                           int cap, int d, float eps) {
+  const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (j >= min(*n_rows, cap)) return;
+  rmsnorm_row<T>(x + (size_t)rows[j] * d, g, o + (size_t)j * d, d, eps);
+}
+
+__global__ void rope_table_kernel(float2* table, int N, int hd, double theta) {
+  const int half = hd / 2;
+  const size_t total = (size_t)N * half;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int p = (int)(i / half), j = (int)(i % half);
+    const double inv = pow(theta, -2.0 * j / hd);
+    double sn, cs;
+    sincos((double)p * inv, &sn, &cs);
+    table[i] = make_float2((float)cs, (float)sn);
+  }
+}
+
+__global__ void __launch_bounds__(1024) masked_rows_kernel(const int32_t* __restrict__ tokens,
+                                                           int mask_id,
+                                                           const int* __restrict__ row_pos,
+                                                           const int* __restrict__ row_seq,
+                                                           const int* __restrict__ M_dev,
+                                                           int M_cap, int N, int* __restrict__ out,
+                                                           int* __restrict__ n_out) {
+  __shared__ int red[33];
+  __shared__ int s_carry;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int r0 = 0; r0 < M; r0 += blockDim.x) {
+    const int r = r0 + threadIdx.x;
+    const int f = (r < M && tokens[(size_t)row_seq[r] * N + row_pos[r]] == mask_id) ? 1 : 0;
+    const int incl = block_inclusive_scan(f, red);
+    const int carry = s_carry;
+    if (f) out[carry + incl - 1] = r;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) s_carry = carry + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *n_out = s_carry;
+}
+
+__global__ void copy_idx_kernel(const int32_t* src_idx, const int32_t* src_count,
+                                int32_t* dst_idx, int32_t* dst_count, int B, int k_cap) {
+  const size_t total = (size_t)B * k_cap;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x)
+    dst_idx[i] = src_idx[i];
+  if (blockIdx.x == 0)
+    for (int b = threadIdx.x; b < B; b += blockDim.x) dst_count[b] = src_count[b];
+}
+
+// ---------------------------------------------------------------- fp32 layer pieces
+
+// C[M,N] = A[M,K] B[N,K]^T (+ R[M,N]); 64x64 tile, 256 threads, 4x4 per thread
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A,
+                                                       const float* __restrict__ Bm,
+                                                       float* __restrict__ C,
+                                                       const float* __restrict__ R,
+                                                       const int* __restrict__ M_dev, int M_cap,
+                                                       int N, int K) {
+  __shared__ float As[16][65];
+  __shared__ float Bs[16][65];
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  if (m0 >= M) return;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int i = threadIdx.x; i < 64 * 16; i += 256) {
+      const int r = i / 16, kk = i % 16;
+      As[kk][r] = (m0 + r < M && k0 + kk < K) ? A[(size_t)(m0 + r) * K + k0 + kk] : 0.f;
+      Bs[kk][r] = (n0 + r < N && k0 + kk < K) ? Bm[(size_t)(n0 + r) * K + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        a[i] = As[kk][ty * 4 + i];
+        b[i] = Bs[kk][tx * 4 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty * 4 + i;
+    if (m >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n >= N) continue;
+      float v = acc[i][j];
+      if (R) v += R[(size_t)m * N + n];
+      C[(size_t)m * N + n] = v;
+    }
+  }
+}
+
+__global__ void qkv_post_f32_kernel(const float* __restrict__ qr, const float* __restrict__ kr,
+                                    const float* __restrict__ vr, float* __restrict__ q,
+                                    float* __restrict__ kc, float* __restrict__ vc,
+                                    const int* __restrict__ row_pos,
+                                    const int* __restrict__ row_seq, const int* __restrict__ M_dev,
+                                    int M_cap, int Nseq, int Hq, int Hkv, int hd,
+                                    const float2* __restrict__ rope) {
+  const int r = blockIdx.x;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  const int pos = row_pos[r], seq = row_seq[r];
+  const int half = hd / 2;
+  const size_t cache_row = ((size_t)seq * Nseq + pos) * Hkv * hd;
+  for (int i = threadIdx.x; i < (Hq + 2 * Hkv) * half; i += blockDim.x) {
+    const int h = i / half, j = i % half;
+    const float* src;
+    float* dst;
+    bool rot = rope != nullptr;
+    if (h < Hq) {
+      src = qr + (size_t)r * Hq * hd + h * hd;
+      dst = q + (size_t)r * Hq * hd + h * hd;
+    } else if (h < Hq + Hkv) {
+      src = kr + (size_t)r * Hkv * hd + (h - Hq) * hd;
+      dst = kc + cache_row + (h - Hq) * hd;
+    } else {
+      src = vr + (size_t)r * Hkv * hd + (h - Hq - Hkv) * hd;
+      dst = vc + cache_row + (h - Hq - Hkv) * hd;
+      rot = false;
+    }
+    const float x1 = src[j], x2 = src[j + half];
+    if (rot) {
+      const float2 t = rope[(size_t)pos * half + j];
+      dst[j] = x1 * t.x - x2 * t.y;
+      dst[j + half] = x2 * t.x + x1 * t.y;
+    } else {
+      dst[j] = x1;
+      dst[j + half] = x2;
+    }
+  }
+}
+
+__global__ void swiglu_f32_kernel(const float* __restrict__ g, const float* __restrict__ u,
+                                  float* __restrict__ a, const int* __restrict__ M_dev, int M_cap,
+                                  int F) {
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  const size_t total = (size_t)M * F;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float x = g[i];
+    a[i] = x / (1.0f + expf(-x)) * u[i];
+  }
+}
+
+// one block per (row, head): scores of all keys in shared memory, softmax, P V
+__global__ void __launch_bounds__(128) attention_f32_kernel(
+    const float* __restrict__ q, const float* __restrict__ kc, const float* __restrict__ vc,
+    float* __restrict__ o, const int* __restrict__ row_seq, const int* __restrict__ M_dev,
+    int M_cap, int Nseq, int Hq, int Hkv, int hd) {
+  extern __shared__ float s_p[];
+  __shared__ float red[33];
+  const int r = blockIdx.x, h = blockIdx.y;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  const int seq = row_seq[r], g = (h * Hkv) / Hq;
+  const float* qv = q + ((size_t)r * Hq + h) * hd;
+  const float scale = rsqrtf((float)hd);
+  float mx = -INFINITY;
+  for (int j = threadIdx.x; j < Nseq; j += blockDim.x) {
+    const float* kv = kc + (((size_t)seq * Nseq + j) * Hkv + g) * hd;
+    float s = 0.f;
+    for (int e = 0; e < hd; ++e) s = fmaf(qv[e], kv[e], s);
+    s *= scale;
+    s_p[j] = s;
+    mx = fmaxf(mx, s);
+  }
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int i = 1; i < (int)(blockDim.x >> 5); ++i) t = fmaxf(t, red[i]);
+    red[32] = t;
+  }
+  __syncthreads();
+  mx = red[32];
+  __syncthreads();
+  float sum = 0.f;
+  for (int j = threadIdx.x; j < Nseq; j += blockDim.x) {
+    const float e = expf(s_p[j] - mx);
+    s_p[j] = e;
+    sum += e;
+  }
+  sum = warp_sum(sum);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    red[32] = t;
+  }
+  __syncthreads();
+  const float inv = 1.0f / red[32];
+  for (int e = threadIdx.x; e < hd; e += blockDim.x) {
+    float acc = 0.f;
+    for (int j = 0; j < Nseq; ++j)
+      acc = fmaf(s_p[j], vc[(((size_t)seq * Nseq + j) * Hkv + g) * hd + e], acc);
+    o[((size_t)r * Hq + h) * hd + e] = acc * inv;
+  }
+}
+
+inline int grid_for(size_t n, int threads, int cap = 148 * 16) {
+  size_t g = (n + threads - 1) / threads;
+  if (g < 1) g = 1;
+  if (g > (size_t)cap) g = cap;
+  return (int)g;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- launchers
+
+template <typename T>
+void launch_score(const T* h_cur, const T* embed, const int32_t* tokens, const T* h_ref, int B,
+                  int N, int d, const float* conf, const uint8_t* masked,
+                  const int32_t* mask_tokens, int mask_id, float alpha, int kind, float* scores,
+                  int vocab, int* status, cudaStream_t s) {
+  const int rows = B * N;
+  if (rows <= 0) return;
+  ProfScope prof("score", s);
+  score_kernel<T><<<(rows + 7) / 8, 256, 0, s>>>(h_cur, embed, tokens, h_ref, rows, N, d, conf,
+                                                 masked, mask_tokens, mask_id, alpha, kind,
+                                                 scores, vocab, status);
+}
+template void launch_score<float>(const float*, const float*, const int32_t*, const float*, int,
+                                  int, int, const float*, const uint8_t*, const int32_t*, int,
+                                  float, int, float*, int, int*, cudaStream_t);
+template void launch_score<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                          const int32_t*, const __nv_bfloat16*, int, int, int,
+                                          const float*, const uint8_t*, const int32_t*, int, float,
+                                          int, float*, int, int*, cudaStream_t);
+
+template <typename T>
+void launch_confidence(const T* logits, const int32_t* logit_pos, int B, int Mm, int V, int N,
+                       float* conf, int32_t* pred, cudaStream_t s) {
+  if (B * Mm <= 0) return;
+  ProfScope prof("confidence", s);
+  confidence_kernel<T><<<B * Mm, 256, 0, s>>>(logits, logit_pos, Mm, V, N, conf, pred);
+}
+template void launch_confidence<float>(const float*, const int32_t*, int, int, int, int, float*,
+                                       int32_t*, cudaStream_t);
+template void launch_confidence<__nv_bfloat16>(const __nv_bfloat16*, const int32_t*, int, int, int,
+                                               int, float*, int32_t*, cudaStream_t);
+
+void launch_select(const float* scores, int B, int N, int mode, int k, float tau, int32_t* idx,
+                   int32_t* count, int k_cap, int* status, cudaStream_t s) {
+  if (B <= 0) return;
+  ProfScope prof("select", s);
+  select_kernel<<<B, SEL_THREADS, 0, s>>>(scores, N, mode, k, tau, idx, count, k_cap, status);
+}
+
+void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
+                   int mask_id, int gen_start, int block_len, int n_unmask, int32_t* pos_out,
+                   const int32_t* forced, cudaStream_t s) {
+  if (B <= 0) return;
+  ProfScope prof("unmask", s);
+  unmask_kernel<<<B, 1024, 0, s>>>(conf, pred, tokens, N, mask_id, gen_start, block_len, n_unmask,
+                                   pos_out, forced);
+}
+
+void launch_row_map(const int32_t* idx, const int32_t* count, int B, int k_cap, int N,
+                    int* row_off, int* row_pos, int* row_seq, int* status, cudaStream_t s) {
+  ProfScope prof("row_map", s);
+  row_map_kernel<<<1, 1024, 0, s>>>(idx, count, B, k_cap, N, row_off, row_pos, row_seq, status);
+}
+
+void launch_row_map_dense(int B, int N, int* row_off, int* row_pos, int* row_seq,
+                          cudaStream_t s) {
+  ProfScope prof("row_map", s);
+  row_map_dense_kernel<<<grid_for((size_t)B * N, 256), 256, 0, s>>>(B, N, row_off, row_pos,
+                                                                    row_seq);
+}
+
+void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
+                     int32_t* dst_count, int B, int k_cap, cudaStream_t s) {
+  ProfScope prof("copy_idx", s);
+  copy_idx_kernel<<<grid_for((size_t)B * k_cap, 256), 256, 0, s>>>(src_idx, src_count, dst_idx,
+                                                                   dst_count, B, k_cap);
+}
+
+template <typename T>
+void launch_gather_rows(const T* src_full, const T* embed, const int32_t* tokens,
+                        const int* row_pos, const int* row_seq, const int* M_dev, int M_cap,
+                        int N, int d, T* x, T* h_ref, int vocab, int* status, cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("gather", s);
+  gather_rows_kernel<T><<<(M_cap + 7) / 8, 256, 0, s>>>(src_full, embed, tokens, row_pos,
+                                                        row_seq, M_dev, M_cap, N, d, x, h_ref,
+                                                        vocab, status);
+}
+template void launch_gather_rows<float>(const float*, const float*, const int32_t*, const int*,
+                                        const int*, const int*, int, int, int, float*, float*,
+                                        int, int*, cudaStream_t);
+template void launch_gather_rows<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                const int32_t*, const int*, const int*,
+                                                const int*, int, int, int, __nv_bfloat16*,
+                                                __nv_bfloat16*, int, int*, cudaStream_t);
+
+template <typename T>
+void launch_rmsnorm(const T* x, const T* g, T* out, const int* M_dev, int M_cap, int d, float eps,
+                    cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("rmsnorm", s);
+  rmsnorm_kernel<T><<<(M_cap + 7) / 8, 256, 0, s>>>(x, g, out, M_dev, M_cap, d, eps);
+}
+template void launch_rmsnorm<float>(const float*, const float*, float*, const int*, int, int,
+                                    float, cudaStream_t);
+template void launch_rmsnorm<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                            __nv_bfloat16*, const int*, int, int, float,
+                                            cudaStream_t);
+
+template <typename T>
+void launch_rmsnorm_rows(const T* x, const T* g, T* out, const int* rows, const int* n_rows,
+                         int cap, int d, float eps, cudaStream_t s) {
+  if (cap <= 0) return;
+  ProfScope prof("rmsnorm", s);
+  rmsnorm_rows_kernel<T><<<(cap + 7) / 8, 256, 0, s>>>(x, g, out, rows, n_rows, cap, d, eps);
+}
+template void launch_rmsnorm_rows<float>(const float*, const float*, float*, const int*,
+                                         const int*, int, int, float, cudaStream_t);
+template void launch_rmsnorm_rows<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                                 __nv_bfloat16*, const int*, const int*, int, int,
+                                                 float, cudaStream_t);
+
+void launch_rope_table(float2* table, int N, int hd, float theta, cudaStream_t s) {
+  ProfScope prof("rope_table", s);
+  rope_table_kernel<<<grid_for((size_t)N * hd / 2, 256), 256, 0, s>>>(table, N, hd,
+                                                                      (double)theta);
+}
+
+void launch_masked_rows(const int32_t* tokens, int mask_id, const int* row_pos,
+                        const int* row_seq, const int* M_dev, int M_cap, int N, int* lm_rows,
+                        int* n_lm, cudaStream_t s) {
+  ProfScope prof("masked_rows", s);
+  masked_rows_kernel<<<1, 1024, 0, s>>>(tokens, mask_id, row_pos, row_seq, M_dev, M_cap, N,
+                                        lm_rows, n_lm);
+}
+
+void launch_lm_merge(const float* lm_part, int tiles, const int* lm_rows, const int* n_lm,
+                     int cap, const int* row_pos, const int* row_seq, int N, float* conf,
+                     int32_t* pred, cudaStream_t s) {
+  if (cap <= 0) return;
+  ProfScope prof("lm_merge", s);
+  lm_merge_kernel<<<(cap + 3) / 4, 128, 0, s>>>(lm_part, tiles, lm_rows, n_lm, cap, row_pos,
+                                                row_seq, N, conf, pred);
+}
+
+void launch_gemm_f32(const float* A, const float* B, float* C, const float* R, const int* M_dev,
+                     int M_cap, int N, int K, cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("gemm_f32", s);
+  dim3 grid((N + 63) / 64, (M_cap + 63) / 64);
+  gemm_f32_kernel<<<grid, 256, 0, s>>>(A, B, C, R, M_dev, M_cap, N, K);
+}
+
+void launch_qkv_post_f32(const float* q_raw, const float* k_raw, const float* v_raw,
+                         float* q_out, float* kc, float* vc, const int* row_pos,
+                         const int* row_seq, const int* M_dev, int M_cap, int Nseq, int Hq,
+                         int Hkv, int hd, const float2* rope, cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("qkv_post_f32", s);
+  qkv_post_f32_kernel<<<M_cap, 256, 0, s>>>(q_raw, k_raw, v_raw, q_out, kc, vc, row_pos, row_seq,
+                                            M_dev, M_cap, Nseq, Hq, Hkv, hd, rope);
+}
+
+void launch_swiglu_f32(const float* g, const float* u, float* a, const int* M_dev, int M_cap,
+                       int F, cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("swiglu_f32", s);
+  swiglu_f32_kernel<<<grid_for((size_t)M_cap * F, 256), 256, 0, s>>>(g, u, a, M_dev, M_cap, F);
+}
+
+void launch_attention_f32(const float* q, const float* kc, const float* vc, float* o,
+                          const int* row_seq, const int* M_dev, int M_cap, int Nseq, int Hq,
+                          int Hkv, int hd, cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("attention_f32", s);
+  const size_t smem = (size_t)Nseq * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(attention_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         64 * 1024);
+    attr = true;
+  }
+  dim3 grid(M_cap, Hq);
+  attention_f32_kernel<<<grid, 128, smem, s>>>(q, kc, vc, o, row_seq, M_dev, M_cap, Nseq, Hq, Hkv,
+                                               hd);
+}
+
+void launch_confidence_rows_f32(const float* logits, int V, const int* lm_rows, const int* n_lm,
+                                int cap, const int* row_pos, const int* row_seq, int N,
+                                float* conf, int32_t* pred, cudaStream_t s) {
+  if (cap <= 0) return;
+  ProfScope prof("confidence", s);
+  confidence_rows_f32_kernel<<<cap, 256, 0, s>>>(logits, V, lm_rows, n_lm, row_pos, row_seq, N,
+                                                 conf, pred);
+}
+
+}  // namespace dllm

@@ -1,0 +1,76 @@
+"""The C-ABI library loads, exports every entry point the header declares,
+and rejects bad arguments on the host before touching the GPU (CPU tests)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dllm.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dllm_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_token_recompute_b200 import build
+    path = build.build()
+    return C.CDLL(path)
+
+
+def test_header_declares_the_step_entry_points():
+    names = _declared()
+    for n in ("dllm_score", "dllm_select", "dllm_partial_layer", "dllm_step", "dllm_unmask"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_host_only_calls(lib):
+    lib.dllm_status_string.restype = C.c_char_p
+    assert lib.dllm_status_string(0) == b"ok"
+    assert b"workspace" in lib.dllm_status_string(3)
+    assert lib.dllm_status_string(99) == b"unknown status"
+    assert lib.dllm_version() >= 100
+
+
+def test_bad_arguments_are_rejected_before_launch(lib):
+    import sparse_token_recompute_b200 as S
+    # negative sizes / bad enums / missing pointers: status codes, no CUDA work
+    assert S._select(None, -1, 10, 0, 1, 0.0, None, None, 1, None, 0, None) == 1
+    assert S._select(None, 1, 10, 7, 1, 0.0, None, None, 1, None, 0, None) == 1
+    assert S._select(None, 1, 10, 0, 5, 0.0, None, None, 2, None, 0, None) == 5  # k > k_cap
+    assert S._select(None, 1, 20000, 0, 5, 0.0, None, None, 8, None, 0, None) == 2
+    assert S._unmask(None, None, None, 1, 10, 0, 0, 0, 1, None, None) == 1   # block_len 0
+    assert S._unmask(None, None, None, 1, 10, 0, 0, 2048, 1, None, None) == 2
+    assert S._score(None, None, 1, 4, 16, 5, None, None, 0, 0, None, None, None, 0.5, 0,
+                    None, None) == 1  # bad dtype
+    assert S._gemm(None, None, None, 4, 10, 64, 0, 0, None, 0, None) == 1
+    cfg = S.make_cfg(1, 100, 4, 4, 64, 688, 1024, 5e5, 1e-5, 1023, "bf16")
+    lw = S.LayerW()
+    assert S._layer(C.byref(cfg), C.byref(lw), None, 1, None, None, None, 4, 1, 8, None, None,
+                    None, 0, None) == 2  # d not a multiple of 128 on the bf16 path
+    cfg = S.make_cfg(1, 256, 4, 3, 64, 688, 1024, 5e5, 1e-5, 1023, "f32")
+    assert S._layer_ws(C.byref(cfg), 1, 8, 4) == 0  # heads not divisible by kv heads
+    cfg = S.make_cfg(1, 256, 4, 4, 64, 688, 1024, 5e5, 1e-5, 1023, "f32")
+    assert S._layer(C.byref(cfg), C.byref(lw), None, 1, None, None, None, 4, 1, 8, None, None,
+                    None, 0, None) == 1  # null weights
+
+
+def test_workspace_sizes_are_host_computable(lib):
+    import sparse_token_recompute_b200 as S
+    cfg = S.make_cfg(1, 256, 4, 4, 64, 688, 1024, 5e5, 1e-5, 1023, "f32")
+    pol = S.make_policy(k=32, n_unmask=8, gen_start=64, block_len=64)
+    a = S.dllm_step_workspace_size(cfg, 1, 128, pol)
+    b = S.dllm_step_workspace_size(cfg, 2, 128, pol)
+    assert 0 < a < b
+    assert S.dllm_partial_layer_workspace_size(cfg, 1, 128, 32) > 0
+    assert S.dllm_select_workspace_size(4, 100) >= 4
