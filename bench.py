@@ -183,10 +183,17 @@ def bs1_measure(S, W, steps, warmup):
             S.dllm_step(model, cache, tokens, pol, False, ws)
         torch.cuda.synchronize()
         K = min(steps, 20)
+        S.profile_reset()
+        S.profile_enable(True)
         ms = time_steps(S, model, cache, tokens, pol, ws, K, stream) / K
+        S.profile_enable(False)
+        prof = S.profile_read()
         out[f"r{int(ratio * 100)}"] = {"k": shape.k, "ms_per_step": round(ms, 4),
                                        "steps_per_s": round(1000.0 / ms, 2),
-                                       "tokens_per_s": round(shape.n_unmask * 1000.0 / ms, 1)}
+                                       "tokens_per_s": round(shape.n_unmask * 1000.0 / ms, 1),
+                                       "kernels_ms_per_step": {
+                                           n: [v[0] // K, round(v[1] / K, 4)]
+                                           for n, v in sorted(prof.items())}}
         del cache, ws
     return out
 

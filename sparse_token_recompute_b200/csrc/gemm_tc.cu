@@ -589,23 +589,43 @@ GemmPlan gemm_plan(const GemmSpec& g) {
   };
   int bn = g.force_bn;
   int splits = g.force_splits;
+  auto tiles_for = [&](int c) {
+    const int cols = g.epi == EPI_SWIGLU ? N / 2 : N;
+    const int w = g.epi == EPI_SWIGLU ? c / 2 : c;
+    return pl.m_tiles_cap * ((cols + w - 1) / w);
+  };
   if (!bn) {
+    // Rows per weight byte decide the regime: below ~256 rows the GEMM streams its
+    // weights from HBM (time ~ bytes moved / bandwidth, inflated when too few units
+    // keep the SMs busy); above, it is tensor-bound (time ~ waves x tile main loop).
     const int cands[3] = {256, 128, 64};
+    const double wbytes = 2.0 * N * g.K;
+    const double rows = std::min(g.M_cap, BM * pl.m_tiles_cap);
+    const bool weight_bound = g.M_cap < 256;
     double best = 1e30;
     for (int c : cands) {
       if (!bn_ok(c)) continue;
       if (g.epi == EPI_LMHEAD && c < 128) continue;  // stats buffers are sized for >= 128
-      const int tiles = pl.m_tiles_cap * ((N + c - 1) / c);
-      for (int sp = 1; sp <= 16; ++sp) {
-        if (g.epi == EPI_LMHEAD && sp > 1) break;
+      const int tiles = tiles_for(c);
+      for (int sp = 1; sp <= 8; ++sp) {
+        if (sp > 1 && (g.epi == EPI_LMHEAD || !weight_bound)) break;
         if (sp > 1 && kb_total / sp < 4) break;
         const int units = tiles * sp;
         const int waves = (units + sms - 1) / sms;
-        const int kb = (kb_total + sp - 1) / sp;
-        // time ~ waves * (mainloop per unit + fixed cost); wide tiles amortise the A reads
-        const double per_unit = (double)kb * (BM * 64.0 + c * 64.0) / 64.0 + 600.0;
-        double t = waves * per_unit;
-        if (sp > 1) t += 2.0 * (double)sp * std::min(g.M_cap, BM * pl.m_tiles_cap) * c / sms * 0.05;
+        double t;
+        if (weight_bound) {
+          const double partial = sp > 1 ? 2.0 * sp * rows * N * 4.0 : 0.0;
+          const double inflate = (double)waves * sms / units;
+          t = (wbytes + partial) * inflate + 2.0 * rows * g.K * tiles;  // + A reads from L2
+        } else {
+          const int kb = (kb_total + sp - 1) / sp;
+          // one 64-deep k-block of an M=128 x N=c tile: 2c tensor cycles, plus a
+          // fixed per-unit cost (prologue, epilogue drain); narrow tiles move more
+          // operand bytes per FMA through shared memory, charged in proportion
+          const double smem_ratio = ((128.0 + c) / (128.0 * c)) / ((128.0 + 256) / (128.0 * 256));
+          const double per_kb = 2.0 * c * std::max(1.0, smem_ratio);
+          t = waves * (kb * per_kb + 1500.0);
+        }
         if (t < best * 0.999) {
           best = t;
           bn = c;

@@ -1,0 +1,109 @@
+"""Single-kernel cases for profiling the library's kernels under ncu.
+
+Each case sets up inputs larger than L2 (so DRAM counters mean something)
+but a few GB at most, runs the kernel `--warmup` times untimed and then
+`--iters` times, and prints the CUDA-event time per launch.
+
+  python -m sparse_token_recompute_b200.profile_cases gemm --M 9856 --N 12288 --K 4096
+  python -m sparse_token_recompute_b200.profile_cases score --B 32 --L 1024 --d 4096
+  python -m sparse_token_recompute_b200.profile_cases layer --B 32 --N 1536 --k 308
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+import dllm_synth as SY
+import sparse_token_recompute_b200 as S
+
+
+def _time(fn, warmup, iters):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / max(iters, 1)
+
+
+def case_gemm(a):
+    A = SY.normal((a.M, a.K), 1.0, 1, "cuda", "bf16")
+    Bm = SY.normal((a.N, a.K), 0.02, 2, "cuda", "bf16")
+    Cm = torch.empty(a.M, a.N, dtype=torch.bfloat16, device="cuda")
+    ws = S.Workspace(S.dllm_gemm_workspace_size(a.M, a.N, a.K, a.splits))
+    ms = _time(lambda: S.dllm_gemm_bf16(A, Bm, Cm, splits=a.splits, ws=ws), a.warmup, a.iters)
+    fl = 2.0 * a.M * a.N * a.K
+    return {"case": "gemm", "M": a.M, "N": a.N, "K": a.K, "ms": ms, "tflops": fl / ms / 1e9,
+            "bytes_min": 2 * (a.M * a.K + a.N * a.K + a.M * a.N)}
+
+
+def case_score(a):
+    si = SY.score_inputs(a.B, a.L, a.d, a.V, a.Mm, device="cuda")
+    scores = torch.empty(a.B, a.L, dtype=torch.float32, device="cuda")
+    idx = torch.empty(a.B, a.k, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(a.B, dtype=torch.int32, device="cuda")
+    conf = si.conf.clone()
+
+    def run():
+        S.dllm_score(si.h_cur, si.h_ref, conf, si.masked, scores, 0.5, 0, logits=si.logits,
+                     logit_pos=si.logit_pos, pred=si.pred)
+        S.dllm_select(scores, idx, cnt, S.DLLM_SELECT_TOPK, a.k)
+
+    ms = _time(run, a.warmup, a.iters)
+    nbytes = 2 * a.B * a.L * a.d * 2 + a.B * a.Mm * a.V * 2
+    return {"case": "score+select", "ms": ms, "GBps": nbytes / ms / 1e6, "bytes": nbytes}
+
+
+def case_layer(a):
+    shape = SY.with_(SY.DENSE8B_B32_N1536, n_layers=1)
+    W = SY.model_weights(shape, seed=0, device="cuda")
+    cfg = S.cfg_from_shape(shape)
+    lw = S.layer_struct(W["layers"][0])
+    kv = (a.B, a.N, shape.n_kv_heads, shape.head_dim)
+    kc = SY.normal(kv, 1.0, 3, "cuda", "bf16")
+    vc = SY.normal(kv, 1.0, 4, "cuda", "bf16")
+    h = SY.normal((a.B, a.N, shape.d), 1.0, 5, "cuda", "bf16")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(6)
+    idx = torch.sort(torch.rand(a.B, a.N, generator=g, device="cuda").argsort(1)[:, :a.k], 1)[0]
+    idx = idx.to(torch.int32).contiguous()
+    cnt = torch.full((a.B,), a.k, dtype=torch.int32, device="cuda")
+    x = torch.empty(a.B * a.k, shape.d, dtype=torch.bfloat16, device="cuda")
+    ws = S.Workspace(S.dllm_partial_layer_workspace_size(cfg, a.B, a.N, a.k))
+    ms = _time(lambda: S.dllm_partial_layer(cfg, lw, h, x, idx, cnt, kc, vc, ws, True),
+               a.warmup, a.iters)
+    return {"case": "partial_layer", "ms": ms}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["gemm", "score", "layer"])
+    ap.add_argument("--M", type=int, default=9856)
+    ap.add_argument("--N", type=int, default=12288)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--splits", type=int, default=0)
+    ap.add_argument("--B", type=int, default=32)
+    ap.add_argument("--L", type=int, default=1024)
+    ap.add_argument("--d", type=int, default=4096)
+    ap.add_argument("--V", type=int, default=32768)
+    ap.add_argument("--Mm", type=int, default=256)
+    ap.add_argument("--k", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=2)
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args()
+    if a.case == "layer" and a.k == 256:
+        a.k = 308
+    if a.case == "layer":
+        a.N = 1536 if a.N == 12288 else a.N
+    out = {"gemm": case_gemm, "score": case_score, "layer": case_layer}[a.case](a)
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()
