@@ -185,12 +185,27 @@ def bs1_measure(S, W, steps, warmup):
         K = min(steps, 20)
         S.profile_reset()
         S.profile_enable(True)
-        ms = time_steps(S, model, cache, tokens, pol, ws, K, stream) / K
+        ms_prof = time_steps(S, model, cache, tokens, pol, ws, K, stream) / K
         S.profile_enable(False)
         prof = S.profile_read()
+        ms_eager = time_steps(S, model, cache, tokens, pol, ws, K, stream) / K
+        # the same step replayed from a CUDA graph (no per-launch host cost)
+        graph = S.StepGraph(model, cache, tokens, pol, ws)
+        graph.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)        # replay() launches on the current stream
+        for _ in range(K):
+            graph.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / K
+        del graph
         out[f"r{int(ratio * 100)}"] = {"k": shape.k, "ms_per_step": round(ms, 4),
                                        "steps_per_s": round(1000.0 / ms, 2),
                                        "tokens_per_s": round(shape.n_unmask * 1000.0 / ms, 1),
+                                       "ms_per_step_eager": round(ms_eager, 4),
+                                       "ms_per_step_eager_profiled": round(ms_prof, 4),
                                        "kernels_ms_per_step": {
                                            n: [v[0] // K, round(v[1] / K, 4)]
                                            for n, v in sorted(prof.items())}}

@@ -251,6 +251,22 @@ dllm_status dllm_step(const dllm_model_cfg* cfg, const dllm_model_w* w, const dl
                       dllm_stream_t stream);
 
 /*
+ * dllm_attention_bf16 - the partial attention of one layer on its own
+ * [DyLLM 1, 2.B]: the selected query rows attend to all N cached keys of
+ * their sequence, no mask, scale 1/sqrt(head_dim), query head h reading KV
+ * head floor(h * n_kv_heads / n_heads).
+ * q: compact rows [B*k_cap, n_heads*head_dim] bf16, packed by sequence as in
+ * dllm_partial_layer (count[b] rows for sequence b); k_cache, v_cache
+ * [B, N, n_kv_heads, head_dim] bf16; o: compact [B*k_cap, n_heads*head_dim].
+ * head_dim 64 or 128.  ws: dllm_attention_workspace_size(B) bytes.
+ */
+size_t dllm_attention_workspace_size(int B);
+dllm_status dllm_attention_bf16(const void* q, const void* k_cache, const void* v_cache, void* o,
+                                const int32_t* count, int B, int k_cap, int N, int n_heads,
+                                int n_kv_heads, int head_dim, void* ws, size_t ws_bytes,
+                                dllm_stream_t stream);
+
+/*
  * dllm_get_device_status - synchronises `stream`, copies the device status
  * word of a workspace used by dllm_select / dllm_partial_layer / dllm_step
  * into *status_out (HOST memory), and clears it.  Returns DLLM_ERR_DEVICE

@@ -88,6 +88,9 @@ _step = _sig("dllm_step", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER
                                _i, _i, C.POINTER(Policy), _i, vp, vp, vp, vp, vp, vp, vp, vp,
                                _sz, vp])
 _devstat = _sig("dllm_get_device_status", _i, [vp, vp, C.POINTER(C.c_int32)])
+_attn_ws = _sig("dllm_attention_workspace_size", _sz, [_i])
+_attn = _sig("dllm_attention_bf16", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i, _i, vp, _sz,
+                                         vp])
 _gemm_ws = _sig("dllm_gemm_workspace_size", _sz, [_i, _i, _i, _i])
 _gemm = _sig("dllm_gemm_bf16", _i, [vp, vp, vp, _i, _i, _i, _i, _i, vp, _sz, vp])
 _prof_enable = _sig("dllm_profile_enable", None, [_i])
@@ -217,6 +220,22 @@ def dllm_gemm_bf16(A, Bm, Cm, accumulate=False, splits=0, ws: Workspace = None, 
     return ws
 
 
+def dllm_attention_workspace_size(B: int) -> int:
+    return int(_attn_ws(B))
+
+
+def dllm_attention_bf16(q, k_cache, v_cache, o, count, k_cap: int, ws: Workspace = None,
+                        stream=None):
+    B, N, Hkv, hd = k_cache.shape
+    Hq = q.shape[1] // hd
+    if ws is None:
+        ws = Workspace(dllm_attention_workspace_size(B), q.device)
+    st = _attn(ptr(q), ptr(k_cache), ptr(v_cache), ptr(o), ptr(count), B, int(k_cap), N, Hq, Hkv,
+               hd, ws.ptr, ws.nbytes, _stream(stream))
+    _check(st, "dllm_attention_bf16")
+    return ws
+
+
 def profile_enable(on: bool = True):
     _prof_enable(int(bool(on)))
 
@@ -331,7 +350,35 @@ def dllm_step_host(model: Model, cache: Cache, tokens_host, pol: Policy, dense: 
     pos_host.copy_(dev_pos, non_blocking=True)
 
 
-__all__ = [n for n in dir() if n.startswith(("dllm_", "DLLM_"))] + [
+class StepGraph:
+    """One ``dllm_step`` captured into a CUDA graph and replayed.
+
+    Every launch of a step depends only on device data (the index lists and
+    row counts are produced on the device), so a step with fixed buffers can
+    be recorded once and replayed for each later step, removing the per-launch
+    host cost.  Capture once after an eager call of the same step (which sets
+    the kernels' shared-memory attributes); buffers must stay at the same
+    addresses for the life of the graph.
+    """
+
+    def __init__(self, model: Model, cache: Cache, tokens, pol: Policy, ws: Workspace,
+                 dense: bool = False, pos_out=None):
+        import torch
+        profile_enable(False)  # per-launch timing events cannot be read back from a graph
+        self.stream = torch.cuda.Stream()
+        self.graph = torch.cuda.CUDAGraph()
+        self.stream.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(self.graph, stream=self.stream):
+            dllm_step(model, cache, tokens, pol, dense, ws, pos_out=pos_out,
+                      stream=self.stream)
+        torch.cuda.current_stream().wait_stream(self.stream)
+
+    def replay(self):
+        self.graph.replay()
+
+
+__all__ = [n for n in dir() if n.startswith(("dllm_", "DLLM_"))] + ["StepGraph",
+
     "Model", "Cache", "Workspace", "ModelCfg", "LayerW", "Policy", "make_cfg", "cfg_from_shape",
     "make_policy", "profile_enable", "profile_reset", "profile_read", "status_string", "version",
     "DllmError", "LIB_PATH"]

@@ -1,6 +1,7 @@
 """Builds the sm_100a shared library ``libdllm.so`` in-tree with nvcc.
 
-Usage: ``python -m sparse_token_recompute_b200.build [--force]``.  Each CUDA
+Usage: ``python sparse_token_recompute_b200/build.py [--force]`` (run by path:
+importing the package loads the library this script builds).  Each CUDA
 source is compiled to an object in ``_build/`` (in parallel), then linked
 into ``sparse_token_recompute_b200/libdllm.so`` with a static CUDA runtime.
 """

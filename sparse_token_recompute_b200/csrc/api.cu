@@ -4,6 +4,7 @@
 // caller's workspace with 256-byte alignment.
 #include <math.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <algorithm>
@@ -288,6 +289,17 @@ void layout_layer(Bump& bp, const dllm_model_cfg* c, int B, int N, int cap, Laye
   w.counter_bytes = cnt;
 }
 
+// DLLM_ATTENTION=mma selects the warp-level MMA attention kernel instead of
+// the tcgen05 one (used to compare the two on the same inputs).
+bool attention_legacy() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("DLLM_ATTENTION");
+    v = (e && strcmp(e, "mma") == 0) ? 1 : 0;
+  }
+  return v == 1;
+}
+
 // One transformer layer over the compact rows in x (in place).
 dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void* x, int M_cap,
                           const int* M_dev, const LayerWs& w, int B, int N, int k_cap,
@@ -328,9 +340,17 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     g.hd = hd;
     g.rope = rope;
     if (gemm_launch(g, s) != cudaSuccess) return DLLM_ERR_CUDA;
-    launch_attention_bf16(static_cast<const bf*>(w.q), static_cast<const bf*>(k_cache),
-                          static_cast<const bf*>(v_cache), static_cast<bf*>(w.o), w.row_off, B,
-                          k_cap, N, c->n_heads, c->n_kv_heads, hd, s);
+    if (attention_legacy()) {
+      launch_attention_bf16(static_cast<const bf*>(w.q), static_cast<const bf*>(k_cache),
+                            static_cast<const bf*>(v_cache), static_cast<bf*>(w.o), w.row_off, B,
+                            k_cap, N, c->n_heads, c->n_kv_heads, hd, s);
+    } else if (launch_attention_tc(static_cast<const bf*>(w.q), M_cap,
+                                   static_cast<const bf*>(k_cache),
+                                   static_cast<const bf*>(v_cache), static_cast<bf*>(w.o),
+                                   w.row_off, B, k_cap, N, c->n_heads, c->n_kv_heads, hd,
+                                   w.status, s) != cudaSuccess) {
+      return DLLM_ERR_CUDA;
+    }
     GemmSpec go = g;
     go.epi = EPI_RESID;
     go.A = static_cast<const bf*>(w.o);
@@ -544,6 +564,41 @@ extern "C" dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, in
   if (g.counters && cudaMemsetAsync(g.counters, 0, p.counter_bytes, s) != cudaSuccess)
     return DLLM_ERR_CUDA;
   return cuda_status(gemm_launch(g, s));
+}
+
+// ---------------------------------------------------------------- attention alone
+
+extern "C" size_t dllm_attention_workspace_size(int B) {
+  Bump bp(nullptr);
+  bp.take<char>(kHeader);
+  bp.take<int>((size_t)std::max(B, 0) + 1);
+  return bp.off;
+}
+
+extern "C" dllm_status dllm_attention_bf16(const void* q, const void* k_cache,
+                                           const void* v_cache, void* o, const int32_t* count,
+                                           int B, int k_cap, int N, int n_heads, int n_kv_heads,
+                                           int head_dim, void* ws, size_t ws_bytes,
+                                           dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B < 0 || k_cap < 1 || N < 0 || n_heads <= 0 || n_kv_heads <= 0) return DLLM_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || N == 0) return DLLM_OK;
+  if (!q || !k_cache || !v_cache || !o || !count) return DLLM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16))
+    return DLLM_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dllm_attention_workspace_size(B))
+    return DLLM_ERR_WORKSPACE;
+  Bump bp(ws);
+  int* status = bp.take<int>(kHeader / sizeof(int));
+  int* row_off = bp.take<int>((size_t)B + 1);
+  launch_row_map(nullptr, count, B, k_cap, N, row_off, nullptr, nullptr, status, s);
+  const cudaError_t e = launch_attention_tc(
+      static_cast<const __nv_bfloat16*>(q), B * k_cap, static_cast<const __nv_bfloat16*>(k_cache),
+      static_cast<const __nv_bfloat16*>(v_cache), static_cast<__nv_bfloat16*>(o), row_off, B,
+      k_cap, N, n_heads, n_kv_heads, head_dim, status, s);
+  return e == cudaSuccess ? check_launch() : DLLM_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------- partial layer

@@ -63,6 +63,7 @@ struct Params {
   const float2* rope;
   float* lm_part;
   int V;
+  int a_tx;  // bytes one A box delivers (fewer than a full 128-row tile when M_cap < 128)
   float* partials;
   int* counters;
   int* status;
@@ -333,7 +334,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), A_BYTES + B_BYTES);
+          mbar_arrive_expect_tx(full_bar(stage), (uint32_t)p.a_tx + B_BYTES);
           const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
           tma_load_2d(a_dst, &tmA, full_bar(stage), kb * BK, m * BM);
@@ -509,33 +510,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaDriverEntryPointQueryResult q;
-    void* f = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-  });
-  return fn;
-}
-
 // [rows, cols] bf16 row-major, box (64 cols, box_rows rows), 128-byte swizzle
 bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows) {
-  auto fn = encode_fn();
-  if (!fn || !ptr || rows <= 0 || cols <= 0) return false;
-  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (cols % 8)) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), gdim, gstride,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  if (rows <= 0 || cols <= 0) return false;
+  return tmap_bf16_2d(m, ptr, (uint64_t)rows, (uint64_t)cols, (uint32_t)box_rows);
 }
 
 template <int BN, int EPI>
@@ -608,15 +586,24 @@ GemmPlan gemm_plan(const GemmSpec& g) {
       if (g.epi == EPI_LMHEAD && c < 128) continue;  // stats buffers are sized for >= 128
       const int tiles = tiles_for(c);
       for (int sp = 1; sp <= 8; ++sp) {
-        if (sp > 1 && (g.epi == EPI_LMHEAD || !weight_bound)) break;
+        if (g.force_splits && sp != g.force_splits) continue;
+        if (!g.force_splits && sp > 1 && (g.epi == EPI_LMHEAD || !weight_bound)) break;
         if (sp > 1 && kb_total / sp < 4) break;
         const int units = tiles * sp;
         const int waves = (units + sms - 1) / sms;
         double t;
         if (weight_bound) {
-          const double partial = sp > 1 ? 2.0 * sp * rows * N * 4.0 : 0.0;
-          const double inflate = (double)waves * sms / units;
-          t = (wbytes + partial) * inflate + 2.0 * rows * g.K * tiles;  // + A reads from L2
+          // Weight streaming, wave by wave: a CTA pulls about kUnitBW from HBM and
+          // the whole GPU at most kCapBW; a split adds a serialized fixup (partial
+          // tiles through L2, measured ~10 us), so narrow tiles beat splitting K.
+          constexpr double kUnitBW = 85e9, kCapBW = 5.8e12, kFixed = 5e-6, kSplit = 10e-6;
+          const double unit_bytes = wbytes / units;
+          double tw = 0.0;
+          for (int left = units; left > 0; left -= sms) {
+            const int n = std::min(left, sms);
+            tw += n * unit_bytes / std::min(kCapBW, n * kUnitBW);
+          }
+          t = tw + kFixed + (sp > 1 ? kSplit : 0.0) + (double)rows * g.K * 2.0 * tiles / 40e12;
         } else {
           const int kb = (kb_total + sp - 1) / sp;
           // one 64-deep k-block of an M=128 x N=c tile: 2c tensor cycles, plus a
@@ -687,7 +674,11 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   if (pl.splits > 1 && (!g.partials || !g.counters)) return cudaErrorInvalidValue;
 
   CUtensorMap ta, tb0, tb1, tb2;
-  if (!make_map(&ta, g.A, g.M_cap, g.K, BM)) return cudaErrorInvalidValue;
+  // with fewer than 128 rows the A box covers only them (rounded to 16): the MMA still
+  // reads 128 smem rows, but rows >= M_cap only feed output rows that are never stored
+  const int a_rows = g.M_cap < BM ? ((g.M_cap + 15) / 16) * 16 : BM;
+  p.a_tx = a_rows * BK * 2;
+  if (!make_map(&ta, g.A, g.M_cap, g.K, a_rows)) return cudaErrorInvalidValue;
   const int bbox = (g.epi == EPI_SWIGLU) ? pl.bn / 2 : pl.bn;
   if (!make_map(&tb0, g.B[0], g.seg_cols[0], g.K, bbox)) return cudaErrorInvalidValue;
   tb1 = tb0;

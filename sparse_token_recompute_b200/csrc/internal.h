@@ -1,6 +1,7 @@
 // Internal launchers shared by the C-ABI layer (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -19,6 +20,12 @@ struct ProfScope {
   ProfScope(const char* name, cudaStream_t st) : s(st) { prof_begin(name, st); }
   ~ProfScope() { prof_end(s); }
 };
+
+// ----- TMA descriptors -----
+// [rows, cols] bf16 row-major, box (64 columns, box_rows rows), 128-byte swizzle;
+// cached by (address, shape, box)
+bool tmap_bf16_2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols,
+                  uint32_t box_rows);
 
 // ----- tcgen05 GEMM -----
 enum EpiKind { EPI_STORE = 0, EPI_RESID = 1, EPI_SWIGLU = 2, EPI_QKV = 3, EPI_LMHEAD = 4 };
@@ -112,6 +119,12 @@ void launch_confidence_rows_f32(const float* logits, int V, const int* lm_rows, 
                                 float* conf, int32_t* pred, cudaStream_t s);
 
 // ----- bf16 attention -----
+// tcgen05 flash attention (Q compact [M_cap, Hq*hd], caches [B, N, Hkv, hd])
+cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
+                                const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
+                                int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
+                                cudaStream_t s);
+// warp-level MMA flash attention (mma.sync), kept for comparison
 void launch_attention_bf16(const __nv_bfloat16* q, const __nv_bfloat16* kc,
                            const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
                            int B, int k_cap, int Nseq, int Hq, int Hkv, int hd,

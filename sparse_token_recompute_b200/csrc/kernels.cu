@@ -130,19 +130,32 @@ __global__ void __launch_bounds__(256) score_kernel(const T* __restrict__ h_cur,
   const T* hr = h_ref + (size_t)row * d;
   float nc = 0.f, nr = 0.f, dd = 0.f, l1 = 0.f;
   int eq = 1;
-  for (int i = lane * 8; i < d; i += 32 * 8) {
-    float a[8], b[8];
-    load_vec8<T>(hc + i, a);
-    load_vec8<T>(hr + i, b);
+  // U vector pairs per lane in flight before any arithmetic
+  constexpr int U = 4;
+  for (int base = lane * 8; base < d; base += 32 * 8 * U) {
+    float a[U][8], b[U][8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float df = a[j] - b[j];
-      nc = fmaf(a[j], a[j], nc);
-      nr = fmaf(b[j], b[j], nr);
-      dd = fmaf(df, df, dd);
-      l1 += fabsf(df);
-      eq &= (__float_as_uint(a[j]) == __float_as_uint(b[j]));
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * 256;
+      if (i < d) {
+        load_vec8<T>(hc + i, a[u]);
+        load_vec8<T>(hr + i, b[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[u][j] = b[u][j] = 0.f;
+      }
     }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float df = a[u][j] - b[u][j];
+        nc = fmaf(a[u][j], a[u][j], nc);
+        nr = fmaf(b[u][j], b[u][j], nr);
+        dd = fmaf(df, df, dd);
+        l1 += fabsf(df);
+        eq &= (__float_as_uint(a[u][j]) == __float_as_uint(b[u][j]));
+      }
   }
   nc = warp_sum(nc);
   nr = warp_sum(nr);
@@ -195,22 +208,42 @@ __device__ __forceinline__ SoftStat soft_merge(SoftStat x, SoftStat y) {
 // statistics of one logits row, block-wide (256 threads)
 template <typename T>
 __device__ SoftStat row_softstat(const T* z, int V, SoftStat* red) {
+  // Chunks of U vectors of 8 per thread: U loads in flight, one rescale per chunk,
+  // exp(x) evaluated as exp2(x * log2 e).
+  constexpr int U = 4;
+  constexpr float LOG2E = 1.4426950408889634f;
   SoftStat st{-INFINITY, 0.f, 0x7fffffff};
-  for (int i = threadIdx.x * 8; i < V; i += blockDim.x * 8) {
-    float f[8];
-    load_vec8<T>(z + i, f);
-    float cm = f[0];
-    int ca = i;
+  const int stride = blockDim.x * 8;
+  for (int base = threadIdx.x * 8; base < V; base += stride * U) {
+    float f[U][8];
 #pragma unroll
-    for (int j = 1; j < 8; ++j)
-      if (f[j] > cm) {
-        cm = f[j];
-        ca = i + j;
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * stride;
+      if (i < V) {
+        load_vec8<T>(z + i, f[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[u][j] = -INFINITY;
       }
-    const float nm = fmaxf(st.m, cm);
-    float s = (st.m == -INFINITY) ? 0.f : st.s * expf(st.m - nm);
+    }
+    float cm = -INFINITY;
+    int ca = 0x7fffffff;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) s += expf(f[j] - nm);
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (f[u][j] > cm) {  // strict: the first (lowest) index of a tie is kept
+          cm = f[u][j];
+          ca = base + u * stride + j;
+        }
+    if (cm == -INFINITY) continue;
+    const float nm = fmaxf(st.m, cm);
+    const float nmL = nm * LOG2E;
+    float s = (st.m == -INFINITY) ? 0.f : st.s * exp2f(fmaf(st.m, LOG2E, -nmL));
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s += exp2f(fmaf(f[u][j], LOG2E, -nmL));
     st.a = (cm > st.m) ? ca : st.a;
     st.m = nm;
     st.s = s;
@@ -518,6 +551,7 @@ __global__ void __launch_bounds__(1024) row_map_kernel(const int32_t* __restrict
   }
   if (threadIdx.x == 0) row_off[B] = s_carry;
   __syncthreads();
+  if (!idx) return;  // offsets only
   for (int b = 0; b < B; ++b) {
     int c = count[b];
     c = c < 0 ? 0 : (c > k_cap ? k_cap : c);

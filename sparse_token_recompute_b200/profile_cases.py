@@ -7,6 +7,8 @@ but a few GB at most, runs the kernel `--warmup` times untimed and then
   python -m sparse_token_recompute_b200.profile_cases gemm --M 9856 --N 12288 --K 4096
   python -m sparse_token_recompute_b200.profile_cases score --B 32 --L 1024 --d 4096
   python -m sparse_token_recompute_b200.profile_cases layer --B 32 --N 1536 --k 308
+  python -m sparse_token_recompute_b200.profile_cases attention --B 32 --N 1536 --k 308
+  python -m sparse_token_recompute_b200.profile_cases step --B 1 --ratio 0.10
 """
 from __future__ import annotations
 
@@ -60,6 +62,38 @@ def case_score(a):
     return {"case": "score+select", "ms": ms, "GBps": nbytes / ms / 1e6, "bytes": nbytes}
 
 
+def case_attention(a):
+    """Selected-query attention of one 8B layer: B sequences x k rows, N keys, 32 heads."""
+    H, hd = a.heads, 128
+    q = SY.normal((a.B * a.k, H * hd), 1.0, 1, "cuda", "bf16")
+    kc = SY.normal((a.B, a.N, a.kv_heads, hd), 1.0, 2, "cuda", "bf16")
+    vc = SY.normal((a.B, a.N, a.kv_heads, hd), 1.0, 3, "cuda", "bf16")
+    o = torch.empty_like(q)
+    cnt = torch.full((a.B,), a.k, dtype=torch.int32, device="cuda")
+    ws = S.Workspace(S.dllm_attention_workspace_size(a.B))
+    ms = _time(lambda: S.dllm_attention_bf16(q, kc, vc, o, cnt, a.k, ws=ws), a.warmup, a.iters)
+    fl = 4.0 * a.B * a.k * a.N * H * hd
+    return {"case": "attention", "ms": ms, "tflops": fl / ms / 1e9,
+            "kv_bytes": 2 * a.B * a.N * a.kv_heads * hd * 2}
+
+
+def case_step(a):
+    """Whole partial denoising steps of the 8B model at batch B, N tokens, ratio r:
+    one dense step, `--warmup` partial steps, then `--iters` timed partial steps."""
+    base = SY.DENSE8B_B1_N768 if a.B == 1 else SY.DENSE8B_B32_N1536
+    shape = SY.with_(base, ratio=a.ratio)
+    W = SY.model_weights(shape, seed=0, device="cuda")
+    model = S.Model(S.cfg_from_shape(shape), W)
+    tokens = SY.prompt_tokens(shape, seed=1, device="cuda")
+    cache = S.Cache(model.cfg, shape.batch, shape.seq_len)
+    pol = S.make_policy(0, shape.alpha, 0, 0, shape.k, 0.0, shape.n_unmask, shape.prompt_len,
+                        shape.block_len)
+    ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+    S.dllm_step(model, cache, tokens, pol, True, ws)
+    ms = _time(lambda: S.dllm_step(model, cache, tokens, pol, False, ws), a.warmup, a.iters)
+    return {"case": "step", "B": shape.batch, "N": shape.seq_len, "k": shape.k, "ms": ms}
+
+
 def case_layer(a):
     shape = SY.with_(SY.DENSE8B_B32_N1536, n_layers=1)
     W = SY.model_weights(shape, seed=0, device="cuda")
@@ -83,7 +117,10 @@ def case_layer(a):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "score", "layer"])
+    ap.add_argument("case", choices=["gemm", "score", "layer", "attention", "step"])
+    ap.add_argument("--ratio", type=float, default=0.10)
+    ap.add_argument("--heads", type=int, default=32)
+    ap.add_argument("--kv-heads", dest="kv_heads", type=int, default=32)
     ap.add_argument("--M", type=int, default=9856)
     ap.add_argument("--N", type=int, default=12288)
     ap.add_argument("--K", type=int, default=4096)
@@ -97,11 +134,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
-    if a.case == "layer" and a.k == 256:
+    if a.case in ("layer", "attention") and a.k == 256:
         a.k = 308
-    if a.case == "layer":
+    if a.case in ("layer", "attention"):
         a.N = 1536 if a.N == 12288 else a.N
-    out = {"gemm": case_gemm, "score": case_score, "layer": case_layer}[a.case](a)
+    out = {"gemm": case_gemm, "score": case_score, "layer": case_layer,
+           "attention": case_attention, "step": case_step}[a.case](a)
     print(json.dumps(out))
 
 

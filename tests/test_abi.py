@@ -18,7 +18,11 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def lib():
-    from sparse_token_recompute_b200 import build
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_dllm_build", os.path.join(ROOT, "sparse_token_recompute_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
     path = build.build()
     return C.CDLL(path)
 

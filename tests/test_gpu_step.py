@@ -156,6 +156,7 @@ def test_step_zero_ratio_leaves_gpu_caches_untouched(lib):
     snap = [t.clone() for t in r.cache.k + r.cache.v] + [r.cache.h_ref.clone(),
                                                           r.cache.conf.clone()]
     r.pol.k = 0
+    r.ws = lib.Workspace(lib.dllm_step_workspace_size(r.model.cfg, r.B, r.N, r.pol))
     idx, cnt, pos, sc = r.gpu_step(False)
     assert np.all(cnt == 0)
     after = r.cache.k + r.cache.v + [r.cache.h_ref, r.cache.conf]
