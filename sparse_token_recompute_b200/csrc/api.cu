@@ -205,59 +205,10 @@ struct LayerWs {
   float* vraw;
   float* graw;
   float* uraw;
-  float* partials;
-  int* counters;
-  size_t counter_bytes;
 };
 
-void plan_gemm_scratch(const dllm_model_cfg* c, int cap, size_t* part, size_t* cnt) {
-  *part = 0;
-  *cnt = 0;
-  if (c->dtype != DLLM_BF16 || cap <= 0) return;
-  const int q = c->n_heads * c->head_dim, kv = c->n_kv_heads * c->head_dim;
-  GemmSpec g{};
-  g.M_cap = cap;
-  g.K = c->d;
-  g.hd = c->head_dim;
-  // QKV
-  g.epi = EPI_QKV;
-  g.n_seg = 3;
-  g.seg_cols[0] = q;
-  g.seg_cols[1] = kv;
-  g.seg_cols[2] = kv;
-  GemmPlan p = gemm_plan(g);
-  *part = std::max(*part, p.partial_bytes);
-  *cnt = std::max(*cnt, p.counter_bytes);
-  // O
-  g.epi = EPI_RESID;
-  g.n_seg = 1;
-  g.seg_cols[0] = c->d;
-  g.K = q;
-  p = gemm_plan(g);
-  *part = std::max(*part, p.partial_bytes);
-  *cnt = std::max(*cnt, p.counter_bytes);
-  // gate/up
-  g.epi = EPI_SWIGLU;
-  g.n_seg = 2;
-  g.seg_cols[0] = c->ffn;
-  g.seg_cols[1] = c->ffn;
-  g.K = c->d;
-  p = gemm_plan(g);
-  *part = std::max(*part, p.partial_bytes);
-  *cnt = std::max(*cnt, p.counter_bytes);
-  // down
-  g.epi = EPI_RESID;
-  g.n_seg = 1;
-  g.seg_cols[0] = c->d;
-  g.K = c->ffn;
-  p = gemm_plan(g);
-  *part = std::max(*part, p.partial_bytes);
-  *cnt = std::max(*cnt, p.counter_bytes);
-}
-
-// `cap` rows of activations; split-K scratch for GEMM plans at both `cap` and `cap2` rows
-void layout_layer(Bump& bp, const dllm_model_cfg* c, int B, int N, int cap, LayerWs& w,
-                  int cap2 = 0) {
+// scratch of a layer pass over up to `cap` compact rows
+void layout_layer(Bump& bp, const dllm_model_cfg* c, int B, int N, int cap, LayerWs& w) {
   const size_t es = esize(c->dtype);
   const int q = c->n_heads * c->head_dim, kv = c->n_kv_heads * c->head_dim;
   w.row_off = bp.take<int>(B + 1);
@@ -276,17 +227,6 @@ void layout_layer(Bump& bp, const dllm_model_cfg* c, int B, int N, int cap, Laye
     w.graw = bp.take<float>((size_t)cap * c->ffn);
     w.uraw = bp.take<float>((size_t)cap * c->ffn);
   }
-  size_t part = 0, cnt = 0;
-  plan_gemm_scratch(c, cap, &part, &cnt);
-  if (cap2 > 0) {
-    size_t p2 = 0, c2 = 0;
-    plan_gemm_scratch(c, cap2, &p2, &c2);
-    part = std::max(part, p2);
-    cnt = std::max(cnt, c2);
-  }
-  w.partials = part ? bp.take<float>(part / sizeof(float)) : nullptr;
-  w.counters = cnt ? bp.take<int>(cnt / sizeof(int)) : nullptr;
-  w.counter_bytes = cnt;
 }
 
 // DLLM_ATTENTION=mma selects the warp-level MMA attention kernel instead of
@@ -319,8 +259,6 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     g.M_cap = M_cap;
     g.M_dev = M_dev;
     g.K = d;
-    g.partials = w.partials;
-    g.counters = w.counters;
     g.status = w.status;
     g.epi = EPI_QKV;
     g.B[0] = static_cast<const bf*>(lw->wq);
@@ -529,8 +467,6 @@ extern "C" size_t dllm_gemm_workspace_size(int M, int N, int K, int splits) {
   GemmPlan p = gemm_plan(g);
   Bump bp(nullptr);
   bp.take<char>(kHeader);
-  bp.take<char>(p.partial_bytes);
-  bp.take<char>(p.counter_bytes);
   return bp.off;
 }
 
@@ -559,10 +495,6 @@ extern "C" dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, in
   GemmPlan p = gemm_plan(g);
   Bump bp(ws);
   g.status = bp.take<int>(kHeader / sizeof(int));
-  g.partials = p.partial_bytes ? bp.take<float>(p.partial_bytes / sizeof(float)) : nullptr;
-  g.counters = p.counter_bytes ? bp.take<int>(p.counter_bytes / sizeof(int)) : nullptr;
-  if (g.counters && cudaMemsetAsync(g.counters, 0, p.counter_bytes, s) != cudaSuccess)
-    return DLLM_ERR_CUDA;
   return cuda_status(gemm_launch(g, s));
 }
 
@@ -635,8 +567,6 @@ extern "C" dllm_status dllm_partial_layer(const dllm_model_cfg* c, const dllm_la
   LayerWs w{};
   w.status = bp.take<int>(kHeader / sizeof(int));
   layout_layer(bp, c, B, N, cap, w);
-  if (w.counters && cudaMemsetAsync(w.counters, 0, w.counter_bytes, s) != cudaSuccess)
-    return DLLM_ERR_CUDA;
   launch_row_map(idx, count, B, k_cap, N, w.row_off, w.row_pos, w.row_seq, w.status, s);
   const bool use_rope = c->rope_theta > 0.f;
   if (use_rope) launch_rope_table(w.rope, N, c->head_dim, c->rope_theta, s);
@@ -685,7 +615,7 @@ void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, Ste
   const size_t es = esize(c->dtype);
   const int cap = B * N;  // covers the dense step
   w.status = bp.take<int>(kHeader / sizeof(int));
-  layout_layer(bp, c, B, N, cap, w.L, B * k_cap);
+  layout_layer(bp, c, B, N, cap, w.L);
   w.L.status = w.status;
   w.x = bp.take<char>((size_t)cap * c->d * es);
   w.h_full = bp.take<char>((size_t)cap * c->d * es);
@@ -756,8 +686,6 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
   StepWs w{};
   layout_step(bp, c, B, N, k_cap, w);
   LayerWs& L = w.L;
-  if (L.counters && cudaMemsetAsync(L.counters, 0, L.counter_bytes, s) != cudaSuccess)
-    return DLLM_ERR_CUDA;
   const bool use_rope = c->rope_theta > 0.f;
   if (use_rope) launch_rope_table(L.rope, N, c->head_dim, c->rope_theta, s);
   const bool bf = c->dtype == DLLM_BF16;

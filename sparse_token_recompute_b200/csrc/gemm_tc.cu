@@ -14,9 +14,10 @@
 //   * warps 2-5: epilogue, one TMEM lane quadrant each (thread = one row),
 //     fused per use: plain store, residual add, SwiGLU, RoPE + K/V cache
 //     scatter, or the LM-head online softmax statistics;
-//   * split-K units write fp32 partial tiles; the last unit of a tile (by an
-//     atomic ticket) adds the partials in split order, so the result does
-//     not depend on which CTA finishes last.
+//   * weight-streaming shapes may split K across the CTAs of a thread-block
+//     cluster: each CTA stages its fp32 partial tile in shared memory and the
+//     cluster reduces it over distributed shared memory in split order, so
+//     the result does not depend on timing.
 // No TMA multicast is used anywhere.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -64,8 +65,6 @@ struct Params {
   float* lm_part;
   int V;
   int a_tx;  // bytes one A box delivers (fewer than a full 128-row tile when M_cap < 128)
-  float* partials;
-  int* counters;
   int* status;
 };
 
@@ -96,6 +95,32 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+// ---------------------------------------------------------------- cluster / DSMEM
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// the address of the same shared-memory offset in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+// every thread of every CTA in the cluster
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
 
 // ---------------------------------------------------------------- epilogues
 // `ld(c, v)` fills v[0..31] with fp32 columns [c, c+32) of this thread's row
@@ -264,8 +289,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // bars: full[STAGES], empty[STAGES], tfull[2], tempty[2], drain[1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  volatile int* s_last = abort_flag + 1;
-  volatile int* epi_abort = abort_flag + 2;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -298,7 +321,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
-    *epi_abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -429,14 +451,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // warp-uniform outcome: TMEM loads below are warp-collective
       const bool ok = __all_sync(0xffffffffu,
                                  mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
-      if (p.splits > 1) {
-        // and block-uniform among the epilogue warps, which meet at named barriers
-        if (!ok) *epi_abort = 1;
-        named_bar_sync(1, EPI_THREADS);
-        if (*epi_abort) break;
-      } else if (!ok) {
-        break;
-      }
+      if (!ok) break;
       tc_fence_after();
       const int row = m * BM + r_in_tile;
       const bool row_ok = row < M;
@@ -444,55 +459,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (p.splits == 1) {
         epilogue_tile<BN, EPI>(p, row, row_ok, m, n,
                                [&](int c, float* v) { tmem_ld_32x32b_x32(t_row + c, v); });
-        tc_fence_before();
-        mbar_arrive(tempty_bar(acc));
       } else {
-        const int tile = m * p.tiles_n + n;
-        float* part = p.partials + (((size_t)tile * p.splits + s) * BM + r_in_tile) * BN;
+        // split K inside a cluster: stage this CTA's fp32 partial rows in its own
+        // shared memory (the stage ring is idle once the accumulator is complete)
+        float* rrow = reinterpret_cast<float*>(smem) + (size_t)r_in_tile * (BN + 4);
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
           float v[32];
           tmem_ld_32x32b_x32(t_row + c, v);
-          if (row_ok) {
-            float4* dst = reinterpret_cast<float4*>(part + c);
+          float4* dst = reinterpret_cast<float4*>(rrow + c);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              __stcg(dst + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(tempty_bar(acc));
-        __threadfence();
-        named_bar_sync(1, EPI_THREADS);
-        if (threadIdx.x == 64) {
-          const int old = atomicAdd(&p.counters[tile], 1);
-          *s_last = (old == p.splits - 1) ? 1 : 0;
-        }
-        named_bar_sync(1, EPI_THREADS);
-        if (*s_last) {
-          __threadfence();
-          const float* base = p.partials + ((size_t)tile * p.splits * BM + r_in_tile) * BN;
-          epilogue_tile<BN, EPI>(p, row, row_ok, m, n, [&](int c, float* v) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-            if (row_ok) {
-              for (int sp = 0; sp < p.splits; ++sp) {
-                const float4* src =
-                    reinterpret_cast<const float4*>(base + (size_t)sp * BM * BN + c);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const float4 t = __ldcg(src + i);
-                  v[4 * i] += t.x;
-                  v[4 * i + 1] += t.y;
-                  v[4 * i + 2] += t.z;
-                  v[4 * i + 3] += t.w;
-                }
-              }
-            }
-          });
-          if (threadIdx.x == 64) p.counters[tile] = 0;
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -502,6 +484,65 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (p.splits > 1) {
+    // The S CTAs of a cluster computed the S K-slices of one tile.  After the
+    // first cluster barrier every partial is staged; CTA `rank` sums rows
+    // [rank*SR, rank*SR + SR) of all S partials over distributed shared memory
+    // (in split order, so the result does not depend on timing) and runs the
+    // fused epilogue on them.  The second barrier keeps every CTA (and its
+    // staged partial) alive until all reads are done.
+    cluster_sync_all();
+    if (warp >= 2 && (int)blockIdx.x < n_units) {
+      int m, n, s;
+      decode_unit(blockIdx.x, m_tiles, p.tiles_n, p.splits, m, n, s);
+      const int S = p.splits;
+      const int rank = (int)cluster_ctarank();
+      const int SR = (BM + S - 1) / S;
+      const int r0 = rank * SR;
+      const int valid = min(BM, M - m * BM);
+      const int nrow = max(0, min(min(BM, r0 + SR), valid) - r0);
+      const int t = threadIdx.x - 64;
+      float* R = reinterpret_cast<float*>(smem);
+      constexpr int Q4 = BN / 4;
+      for (int e = t; e < nrow * Q4; e += EPI_THREADS) {
+        const int rr = r0 + e / Q4, c4 = e - (e / Q4) * Q4;
+        float* mine = R + (size_t)rr * (BN + 4) + c4 * 4;
+        const uint32_t la = smem_u32(mine);
+        float4 part[8];
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp)
+          if (sp < S) part[sp] = ld_dsmem_f4(mapa_rank(la, (uint32_t)sp));
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp)
+          if (sp < S) {
+            a.x += part[sp].x;
+            a.y += part[sp].y;
+            a.z += part[sp].z;
+            a.w += part[sp].w;
+          }
+        *reinterpret_cast<float4*>(mine) = a;  // only this CTA reads its own slice rows
+      }
+      named_bar_sync(1, EPI_THREADS);
+      if (t < nrow) {
+        const int rl = r0 + t;
+        const int row = m * BM + rl;
+        const float* yrow = R + (size_t)rl * (BN + 4);
+        epilogue_tile<BN, EPI>(p, row, row < M, m, n, [&](int c, float* v) {
+          const float4* src = reinterpret_cast<const float4*>(yrow + c);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 x = src[i];
+            v[4 * i] = x.x;
+            v[4 * i + 1] = x.y;
+            v[4 * i + 2] = x.z;
+            v[4 * i + 3] = x.w;
+          }
+        });
+      }
+    }
+    cluster_sync_all();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
@@ -527,8 +568,24 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  gemm_tc_kernel<BN, EPI><<<grid, NUM_THREADS, smem, s>>>(a, b0, b1, b2, p);
-  return cudaGetLastError();
+  if (p.splits == 1) {
+    gemm_tc_kernel<BN, EPI><<<grid, NUM_THREADS, smem, s>>>(a, b0, b1, b2, p);
+    return cudaGetLastError();
+  }
+  // split K: one unit per CTA, the `splits` CTAs of a tile in one cluster
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)p.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI>, a, b0, b1, b2, p);
 }
 
 template <int EPI>
@@ -572,52 +629,44 @@ GemmPlan gemm_plan(const GemmSpec& g) {
     const int w = g.epi == EPI_SWIGLU ? c / 2 : c;
     return pl.m_tiles_cap * ((cols + w - 1) / w);
   };
-  if (!bn) {
-    // Rows per weight byte decide the regime: below ~256 rows the GEMM streams its
-    // weights from HBM (time ~ bytes moved / bandwidth, inflated when too few units
-    // keep the SMs busy); above, it is tensor-bound (time ~ waves x tile main loop).
+  const bool weight_bound = g.M_cap < 256;
+  if (!bn && weight_bound) {
+    // Weight streaming (fewer than 256 rows): each CTA keeps a ring of 32 KB
+    // weight boxes in flight, and about 64 streaming CTAs saturate HBM (ncu and
+    // split sweeps on the 77-row projections of the 8B shape: O-proj 23 -> 15 us
+    // at 4 splits, down 60 -> 25 us; QKV and gate/up fastest unsplit with 48 and
+    // 96 tiles).  So: the widest tile the epilogue allows, then split K across a
+    // cluster until ~64 CTAs stream.
+    for (int c : {256, 128, 64}) {
+      if (bn_ok(c)) {
+        bn = c;
+        break;
+      }
+    }
+    if (!bn) bn = 64;
+    const int tiles = tiles_for(bn);
+    int sp = 1;
+    if (g.epi != EPI_LMHEAD) sp = std::max(1, std::min(8, (64 + tiles / 2) / std::max(tiles, 1)));
+    while (sp > 1 && kb_total / sp < 4) --sp;
+    if (!splits) splits = sp;
+  } else if (!bn) {
+    // Tensor-bound: time ~ waves x main loop of a tile; no split.
     const int cands[3] = {256, 128, 64};
-    const double wbytes = 2.0 * N * g.K;
-    const double rows = std::min(g.M_cap, BM * pl.m_tiles_cap);
-    const bool weight_bound = g.M_cap < 256;
     double best = 1e30;
     for (int c : cands) {
       if (!bn_ok(c)) continue;
       if (g.epi == EPI_LMHEAD && c < 128) continue;  // stats buffers are sized for >= 128
-      const int tiles = tiles_for(c);
-      for (int sp = 1; sp <= 8; ++sp) {
-        if (g.force_splits && sp != g.force_splits) continue;
-        if (!g.force_splits && sp > 1 && (g.epi == EPI_LMHEAD || !weight_bound)) break;
-        if (sp > 1 && kb_total / sp < 4) break;
-        const int units = tiles * sp;
-        const int waves = (units + sms - 1) / sms;
-        double t;
-        if (weight_bound) {
-          // Weight streaming, wave by wave: a CTA pulls about kUnitBW from HBM and
-          // the whole GPU at most kCapBW; a split adds a serialized fixup (partial
-          // tiles through L2, measured ~10 us), so narrow tiles beat splitting K.
-          constexpr double kUnitBW = 85e9, kCapBW = 5.8e12, kFixed = 5e-6, kSplit = 10e-6;
-          const double unit_bytes = wbytes / units;
-          double tw = 0.0;
-          for (int left = units; left > 0; left -= sms) {
-            const int n = std::min(left, sms);
-            tw += n * unit_bytes / std::min(kCapBW, n * kUnitBW);
-          }
-          t = tw + kFixed + (sp > 1 ? kSplit : 0.0) + (double)rows * g.K * 2.0 * tiles / 40e12;
-        } else {
-          const int kb = (kb_total + sp - 1) / sp;
-          // one 64-deep k-block of an M=128 x N=c tile: 2c tensor cycles, plus a
-          // fixed per-unit cost (prologue, epilogue drain); narrow tiles move more
-          // operand bytes per FMA through shared memory, charged in proportion
-          const double smem_ratio = ((128.0 + c) / (128.0 * c)) / ((128.0 + 256) / (128.0 * 256));
-          const double per_kb = 2.0 * c * std::max(1.0, smem_ratio);
-          t = waves * (kb * per_kb + 1500.0);
-        }
-        if (t < best * 0.999) {
-          best = t;
-          bn = c;
-          splits = sp;
-        }
+      const int units = tiles_for(c);
+      const int waves = (units + sms - 1) / sms;
+      // one 64-deep k-block of an M=128 x N=c tile: 2c tensor cycles, plus a
+      // fixed per-unit cost (prologue, epilogue drain); narrow tiles move more
+      // operand bytes per FMA through shared memory, charged in proportion
+      const double smem_ratio = ((128.0 + c) / (128.0 * c)) / ((128.0 + 256) / (128.0 * 256));
+      const double per_kb = 2.0 * c * std::max(1.0, smem_ratio);
+      const double t = waves * (kb_total * per_kb + 1500.0);
+      if (t < best * 0.999) {
+        best = t;
+        bn = c;
       }
     }
     if (!bn) bn = 64;
@@ -633,10 +682,8 @@ GemmPlan gemm_plan(const GemmSpec& g) {
   pl.splits = splits;
   pl.tiles_n = (g.epi == EPI_SWIGLU) ? (N / 2 + bn / 2 - 1) / (bn / 2) : (N + bn - 1) / bn;
   pl.units_cap = pl.m_tiles_cap * pl.tiles_n * pl.splits;
-  pl.grid = std::max(1, std::min(pl.units_cap, sms));
-  pl.partial_bytes =
-      splits > 1 ? (size_t)pl.m_tiles_cap * pl.tiles_n * splits * BM * bn * sizeof(float) : 0;
-  pl.counter_bytes = splits > 1 ? (size_t)pl.m_tiles_cap * pl.tiles_n * sizeof(int) : 0;
+  // split K runs one unit per CTA (clusters of `splits`); otherwise persistent CTAs
+  pl.grid = splits > 1 ? pl.units_cap : std::max(1, std::min(pl.units_cap, sms));
   return pl;
 }
 
@@ -668,10 +715,7 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   p.rope = g.rope;
   p.lm_part = g.lm_part;
   p.V = N;
-  p.partials = g.partials;
-  p.counters = g.counters;
   p.status = g.status;
-  if (pl.splits > 1 && (!g.partials || !g.counters)) return cudaErrorInvalidValue;
 
   CUtensorMap ta, tb0, tb1, tb2;
   // with fewer than 128 rows the A box covers only them (rounded to 16): the MMA still

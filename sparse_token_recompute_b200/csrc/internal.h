@@ -56,9 +56,6 @@ struct GemmSpec {
   // LMHEAD partial softmax stats [M_cap, n_tiles] x (max, sum, argmax)
   float* lm_part;
   int lm_tiles;  // out: number of column tiles (set by plan)
-  // split-K scratch
-  float* partials;
-  int* counters;
   int* status;
   int force_bn;      // 0: choose
   int force_splits;  // 0: choose
@@ -66,7 +63,6 @@ struct GemmSpec {
 
 struct GemmPlan {
   int bn, splits, tiles_n, m_tiles_cap, units_cap, grid;
-  size_t partial_bytes, counter_bytes;
 };
 
 int gemm_total_cols(const GemmSpec& g);

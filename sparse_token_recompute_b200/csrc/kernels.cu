@@ -618,6 +618,43 @@ __device__ __forceinline__ void rmsnorm_row(const T* __restrict__ x, const T* __
                                             T* __restrict__ o, int d, float eps) {
   const int lane = threadIdx.x & 31;
   float ss = 0.f;
+  if (d <= 256 * 16) {
+    // whole row in registers (up to 16 vectors of 8 per lane): every load is
+    // issued before the first use, then the row is normalised from registers
+    float f[16][8];
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      const int i = lane * 8 + v * 256;
+      if (i < d) load_vec8<T>(x + i, f[v]);
+    }
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      if (lane * 8 + v * 256 < d) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) ss = fmaf(f[v][j], f[v][j], ss);
+      }
+    }
+    ss = warp_sum(ss);
+    const float s = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      const int i = lane * 8 + v * 256;
+      if (i < d) {
+        float w[8];
+        load_vec8<T>(g + i, w);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[v][j] = f[v][j] * s * w[j];
+        if constexpr (sizeof(T) == 2) {
+          *reinterpret_cast<uint4*>(o + i) = pack8(f[v]);
+        } else {
+          float4* o4 = reinterpret_cast<float4*>(o + i);
+          o4[0] = make_float4(f[v][0], f[v][1], f[v][2], f[v][3]);
+          o4[1] = make_float4(f[v][4], f[v][5], f[v][6], f[v][7]);
+        }
+      }
+    }
+    return;
+  }
   for (int i = lane * 8; i < d; i += 256) {
     float f[8];
     load_vec8<T>(x + i, f);
