@@ -267,6 +267,31 @@ dllm_status dllm_attention_bf16(const void* q, const void* k_cache, const void* 
                                 dllm_stream_t stream);
 
 /*
+ * dllm_attention_bf16_noalloc - dllm_attention_bf16 without a workspace, for
+ * callers that cannot allocate device memory: code running while a CUDA
+ * graph is captured (cudaMalloc cannot be captured and may synchronise the
+ * device), servers whose memory is split into fixed pools before serving,
+ * plugins that only receive the tensors they compute on.  The pages have no
+ * counterpart; this is an integration convenience.
+ * Same arguments and result as dllm_attention_bf16 minus ws/ws_bytes.  Its
+ * scratch (a status word and B + 1 row offsets) is a fixed array in the
+ * library's device memory, sized for at most DLLM_NOALLOC_MAX_SEQS sequences
+ * (larger B returns DLLM_ERR_CAPACITY before anything is launched); every GPU
+ * that loads the library holds it until the process exits.  The first call on
+ * a device looks up the array's device address: make it before any stream
+ * capture.  All calls share the array: calls that may overlap on the GPU
+ * (other streams, other host threads on the same device) race and must be
+ * ordered by the caller.  Device-side faults are recorded in the shared
+ * status word, which this entry point clears at the start of each call and
+ * does not report.
+ */
+#define DLLM_NOALLOC_MAX_SEQS 4096
+dllm_status dllm_attention_bf16_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                        void* o, const int32_t* count, int B, int k_cap, int N,
+                                        int n_heads, int n_kv_heads, int head_dim,
+                                        dllm_stream_t stream);
+
+/*
  * dllm_get_device_status - synchronises `stream`, copies the device status
  * word of a workspace used by dllm_select / dllm_partial_layer / dllm_step
  * into *status_out (HOST memory), and clears it.  Returns DLLM_ERR_DEVICE

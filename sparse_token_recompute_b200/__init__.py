@@ -88,6 +88,8 @@ _step = _sig("dllm_step", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER
                                _i, _i, C.POINTER(Policy), _i, vp, vp, vp, vp, vp, vp, vp, vp,
                                _sz, vp])
 _devstat = _sig("dllm_get_device_status", _i, [vp, vp, C.POINTER(C.c_int32)])
+_attn_noalloc = _sig("dllm_attention_bf16_noalloc", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i,
+                                                         _i, vp])
 _attn_ws = _sig("dllm_attention_workspace_size", _sz, [_i])
 _attn = _sig("dllm_attention_bf16", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i, _i, vp, _sz,
                                          vp])
@@ -234,6 +236,20 @@ def dllm_attention_bf16(q, k_cache, v_cache, o, count, k_cap: int, ws: Workspace
                hd, ws.ptr, ws.nbytes, _stream(stream))
     _check(st, "dllm_attention_bf16")
     return ws
+
+
+DLLM_NOALLOC_MAX_SEQS = 4096
+
+
+def dllm_attention_bf16_noalloc(q, k_cache, v_cache, o, count, k_cap: int, stream=None):
+    """Partial attention without a workspace, for callers that cannot allocate
+    device memory (e.g. inside CUDA-graph capture, after the first call on the
+    device); its scratch is a fixed array inside the library shared by all calls."""
+    B, N, Hkv, hd = k_cache.shape
+    Hq = q.shape[1] // hd
+    st = _attn_noalloc(ptr(q), ptr(k_cache), ptr(v_cache), ptr(o), ptr(count), B, int(k_cap), N,
+                       Hq, Hkv, hd, _stream(stream))
+    _check(st, "dllm_attention_bf16_noalloc")
 
 
 def profile_enable(on: bool = True):
