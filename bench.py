@@ -120,13 +120,25 @@ def dist_env():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest value of x over all ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tokens_per_s(world: int, tokens_per_step_per_rank: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: every rank reveals its own tokens each step (weak scaling)."""
+    return world * tokens_per_step_per_rank * 1000.0 / ms_per_step_max
+
+
+def rank_inputs(shape, rank: int, device="cuda"):
+    """Each rank generates its own sequences (seed 1 + rank) with replicated weights (seed 0)."""
+    return SY.prompt_tokens(shape, seed=1 + rank, device=device)
 
 
 def barrier(world):
@@ -143,7 +155,7 @@ def setup(S, shape, rank, layers=0):
         shape = SY.with_(shape, n_layers=layers)
     W = SY.model_weights(shape, seed=0, device="cuda")
     model = S.Model(S.cfg_from_shape(shape), W)
-    tokens = SY.prompt_tokens(shape, seed=1 + rank, device="cuda")
+    tokens = rank_inputs(shape, rank)
     cache = S.Cache(model.cfg, shape.batch, shape.seq_len)
     pol = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k, n_unmask=shape.n_unmask,
                         gen_start=shape.prompt_len, block_len=shape.block_len)
@@ -288,7 +300,7 @@ def run_ours(args):
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
     tok_per_step = shape.batch * shape.n_unmask
-    value = world * tok_per_step * 1000.0 / ms_step
+    value = job_tokens_per_s(world, tok_per_step, ms_step)
 
     # end to end through the public API with host token buffers
     tok_h = torch.empty_like(tokens, device="cpu").pin_memory()
@@ -342,7 +354,7 @@ def run_ours(args):
             "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long step)",
             "flops_per_step": flops_step, "launches": gemm_launches,
             "avg_launch_ms": round(gemm_ms / max(gemm_launches, 1), 4), "traffic": None},
-        "e2e": {"value": round(world * tok_per_step * 1000.0 / ms_e2e, 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_tokens_per_s(world, tok_per_step, ms_e2e), 2), "unit": "tokens/s",
                 "ms_per_step": round(ms_e2e, 4),
                 "h2d_bytes_per_step": tokens.numel() * 4,
                 "d2h_bytes_per_step": tokens.numel() * 4 + pos_d.numel() * 4},
