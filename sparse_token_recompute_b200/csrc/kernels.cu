@@ -205,11 +205,20 @@ __device__ __forceinline__ SoftStat soft_merge(SoftStat x, SoftStat y) {
   return r;
 }
 
-// statistics of one logits row, block-wide (256 threads)
+// 2^x with the hardware approximation (relative error about 2^-22), flushing
+// subnormal results to zero; the confidence sums need no more than that
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// statistics (max, sum of exp(z - max), first argmax) of one logits row, block-wide
 template <typename T>
 __device__ SoftStat row_softstat(const T* z, int V, SoftStat* red) {
-  // Chunks of U vectors of 8 per thread: U loads in flight, one rescale per chunk,
-  // exp(x) evaluated as exp2(x * log2 e).
+  // Chunks of U vectors of 8 per thread: U loads in flight; per chunk a max tree,
+  // the argmax searched only when the chunk raises the running maximum, one
+  // rescale, and exp(x) as 2^(x log2 e).
   constexpr int U = 4;
   constexpr float LOG2E = 1.4426950408889634f;
   SoftStat st{-INFINITY, 0.f, 0x7fffffff};
@@ -226,27 +235,32 @@ __device__ SoftStat row_softstat(const T* z, int V, SoftStat* red) {
         for (int j = 0; j < 8; ++j) f[u][j] = -INFINITY;
       }
     }
-    float cm = -INFINITY;
-    int ca = 0x7fffffff;
+    float mq[U];
 #pragma unroll
     for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (f[u][j] > cm) {  // strict: the first (lowest) index of a tie is kept
-          cm = f[u][j];
-          ca = base + u * stride + j;
-        }
+      mq[u] = fmaxf(fmaxf(fmaxf(f[u][0], f[u][1]), fmaxf(f[u][2], f[u][3])),
+                    fmaxf(fmaxf(f[u][4], f[u][5]), fmaxf(f[u][6], f[u][7])));
+    const float cm = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
     if (cm == -INFINITY) continue;
-    const float nm = fmaxf(st.m, cm);
-    const float nmL = nm * LOG2E;
-    float s = (st.m == -INFINITY) ? 0.f : st.s * exp2f(fmaf(st.m, LOG2E, -nmL));
+    if (cm > st.m) {
+      // first (lowest) index holding the new maximum
+      int ca = 0x7fffffff;
+#pragma unroll
+      for (int u = U - 1; u >= 0; --u)
+#pragma unroll
+        for (int j = 7; j >= 0; --j)
+          if (f[u][j] == cm) ca = base + u * stride + j;
+      st.s = (st.m == -INFINITY) ? 0.f : st.s * ex2_approx((st.m - cm) * LOG2E);
+      st.m = cm;
+      st.a = ca;
+    }
+    const float mL = st.m * LOG2E;
+    float sv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s += exp2f(fmaf(f[u][j], LOG2E, -nmL));
-    st.a = (cm > st.m) ? ca : st.a;
-    st.m = nm;
-    st.s = s;
+      for (int j = 0; j < 8; ++j) sv[j & 3] += ex2_approx(fmaf(f[u][j], LOG2E, -mL));
+    st.s += (sv[0] + sv[1]) + (sv[2] + sv[3]);
   }
   // warp merge
 #pragma unroll
@@ -400,17 +414,38 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
       }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0, dg = 0;
-      for (int bin = 255; bin >= 0; --bin) {
-        if (above + hist[bin] >= remaining) {
-          dg = bin;
-          break;
-        }
-        above += hist[bin];
+    if (threadIdx.x < 32) {
+      // warp-parallel search from the top bin: lane l owns bins 255-8l .. 248-8l;
+      // an exclusive suffix sum over lanes gives the count above each lane's bins
+      const int lane = threadIdx.x;
+      int cnt[8], own = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        cnt[q] = hist[255 - 8 * lane - q];
+        own += cnt[q];
       }
-      s_digit = dg;
-      s_above = above;
+      int incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      int above = incl - own;  // count in higher bins than this lane's
+      // the lane whose bins cross `remaining` finds the digit
+      if (above < remaining && above + own >= remaining) {
+        int dg = -1;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {  // static indices: cnt[] stays in registers
+          if (dg < 0) {
+            if (above + cnt[q] >= remaining)
+              dg = 255 - 8 * lane - q;
+            else
+              above += cnt[q];
+          }
+        }
+        s_digit = dg;
+        s_above = above;
+      }
     }
     __syncthreads();
     remaining -= s_above;

@@ -58,8 +58,14 @@ def case_score(a):
         S.dllm_select(scores, idx, cnt, S.DLLM_SELECT_TOPK, a.k)
 
     ms = _time(run, a.warmup, a.iters)
+    S.profile_reset()
+    S.profile_enable(True)
+    _time(run, 0, a.iters)
+    S.profile_enable(False)
+    per = {k: round(v[1] / v[0] * 1000, 1) for k, v in S.profile_read().items()}
     nbytes = 2 * a.B * a.L * a.d * 2 + a.B * a.Mm * a.V * 2
-    return {"case": "score+select", "ms": ms, "GBps": nbytes / ms / 1e6, "bytes": nbytes}
+    return {"case": "score+select", "ms": ms, "GBps": nbytes / ms / 1e6, "bytes": nbytes,
+            "us_per_kernel": per}
 
 
 def case_attention(a):
