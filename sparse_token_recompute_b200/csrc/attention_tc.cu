@@ -3,23 +3,29 @@
 // The selected query rows of each sequence attend to all N cached keys of
 // that sequence, bidirectionally: O = softmax(Q K^T / sqrt(hd)) V.
 //
-// One CTA = one (sequence, query head, tile of 128 compact query rows).
-// Warp roles (192 threads):
-//   warp 0  TMA producer: the Q tile once, then K and V tiles of 128 keys
-//           into a two-stage ring (128-byte-swizzled 64-column boxes);
-//   warp 1  TMEM owner and tcgen05.mma issuer: S_j = Q K_j^T into one of two
-//           TMEM S buffers, then O += P_{j-1} V_{j-1} into the TMEM O buffer;
-//   warps 2-5  softmax, one query row per thread (its TMEM lane): read S_j,
-//           exponentiate against a per-row reference maximum, write P_j
-//           (bf16) into shared memory in the swizzled K-major layout the MMA
-//           reads, and finally normalise O and store it.
-// The reference maximum is only raised (and O rescaled in TMEM) when a tile
-// exceeds it by more than 2^8 in the exp2 domain, so P stays <= 256 and the
-// result is the same softmax; the running sum uses the same reference.
+// One CTA = one (sequence, query head) and up to two tiles of 128 compact
+// query rows (A and B) that share every K/V tile.  Warp roles (320 threads):
+//   warp 0     TMA producer: both Q tiles once, then K and V tiles of 128 keys
+//              through one ring of shared-memory slots (128-byte-swizzled
+//              64-column boxes);
+//   warp 1     TMEM owner and tcgen05.mma issuer;
+//   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one query row
+//              per thread (its TMEM lane).
+// TMEM holds S_A, S_B (fp32, 128 columns each) and O_A, O_B.  Each softmax
+// group reads S_X, exponentiates against a per-row reference maximum and
+// writes P_X back over the first 64 columns of S_X as packed bf16 pairs; the
+// P V product reads its A operand straight from TMEM.  The issuer alternates
+// the groups -- ... PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1) ... -- so one
+// group's softmax overlaps the other group's MMAs.  tcgen05 operations from
+// one thread complete in issue order, so QK_X(j+1) cannot overwrite P_X(j)
+// before PV_X(j) has read it, and once S_X(j) is reported complete PV_X(j-1)
+// is complete too (O_X may then be rescaled in place).
+// The reference maximum is only raised (and O rescaled) when a tile exceeds
+// it by more than 2^8 in the exp2 domain, so P stays <= 256 and the result is
+// the same softmax; the running sum uses the same reference.
 // Every mbarrier wait is bounded; a timeout sets DLLM_DEV_TIMEOUT, drains the
 // block's outstanding copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -28,24 +34,29 @@ namespace dllm {
 
 namespace {
 
-constexpr int BQ = 128;       // query rows per CTA
-constexpr int BKV = 128;      // keys per tile
-constexpr int NTHREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+hd)
+constexpr int BT = 128;       // query rows per tile (= TMEM lanes)
+constexpr int NTILE = 2;      // query tiles per CTA
+constexpr int BKV = 128;      // keys per K/V tile
+constexpr int NTHREADS = 64 + NTILE * 128;
+constexpr uint32_t TMEM_COLS = 512;  // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kSmemMax = 227 * 1024;  // dynamic shared memory a block may opt in to
 
 template <int HD>
 struct Smem {
-  static constexpr int BLK = 64;                       // columns per swizzled box
-  static constexpr int Q_BYTES = BQ * HD * 2;          // HD/64 boxes of 128 rows x 128 B
+  static constexpr int Q_TILE = BT * HD * 2;     // HD/64 boxes of 128 rows x 128 B
   static constexpr int KV_BYTES = BKV * HD * 2;
-  static constexpr int P_BYTES = BQ * BKV * 2;         // 2 boxes of 128 rows x 64 keys
+  // K and V tiles share one ring of slots in consumption order K0 V0 K1 V1 ...,
+  // as many as fit next to the two Q tiles (at most 8)
+  static constexpr int SLOTS_FIT = (kSmemMax - 1280 - NTILE * Q_TILE) / KV_BYTES;
+  static constexpr int SLOTS = SLOTS_FIT < 8 ? SLOTS_FIT : 8;
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + Q_BYTES;
-  static constexpr int V_OFF = K_OFF + 2 * KV_BYTES;
-  static constexpr int P_OFF = V_OFF + 2 * KV_BYTES;
-  static constexpr int BAR_OFF = P_OFF + 2 * P_BYTES;
-  static constexpr int TOTAL = BAR_OFF + 256 + 1024;   // + barriers + alignment slack
+  static constexpr int RING_OFF = Q_OFF + NTILE * Q_TILE;
+  static constexpr int BAR_OFF = RING_OFF + SLOTS * KV_BYTES;
+  // + barriers + alignment slack; at least 116 KB so that one CTA (which holds
+  // all 512 TMEM columns) is resident per SM
+  static constexpr int TOTAL = (BAR_OFF + 256 + 1024) > 116 * 1024 ? (BAR_OFF + 256 + 1024)
+                                                                   : 116 * 1024;
 };
 
 struct AttnParams {
@@ -56,10 +67,7 @@ struct AttnParams {
   int* status;
 };
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) { tmem_ld_32x32b_x32(taddr, v); }
-
-// 32 columns without the trailing wait: several loads can be in flight before
-// one tcgen05.wait::ld
+// 32 columns without the trailing wait: several loads in flight before one wait
 __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
   asm volatile(
@@ -76,30 +84,40 @@ __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float* v) {
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
-
-__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const float* v) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
       "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-      "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-      "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-      "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-      "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-      "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-      "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-      "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-      "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-      "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-      "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+
+// 2^x with the hardware approximation (relative error about 2^-22); subnormal
+// results flush to zero, which only drops probabilities below 2^-126
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// max of three values in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&t);
 }
 
 __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
@@ -120,6 +138,18 @@ __device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t 
   return d;
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16, fp32 accumulate: A (M=128 lanes x K=16)
+// occupies 8 consecutive 32-bit columns, two bf16 per column (lower index low)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 template <int HD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -129,8 +159,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int b = blockIdx.z, h = blockIdx.y;
   const int off = p.row_off[b];
   const int cnt = p.row_off[b + 1] - off;
-  const int q0 = blockIdx.x * BQ;
+  const int q0 = blockIdx.x * (NTILE * BT);
   if (q0 >= cnt) return;
+  const int nt = (cnt - q0 > BT) ? 2 : 1;  // query tiles holding rows in this CTA
+  // softmax warps of tile x that hold at least one selected row
+  auto live_warps = [&](int x) {
+    const int rows = min(BT, cnt - q0 - x * BT);
+    return rows > 0 ? (rows + 31) / 32 : 1;
+  };
   const int g = (h * p.Hkv) / p.Hq;
   const int T = (p.Nseq + BKV - 1) / BKV;
 
@@ -138,37 +174,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR_OFF);
-  // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], s_free[2], p_full[2],
-  // pv_done[2], drain
-  const uint32_t q_full = smem_u32(&bars[0]);
-  auto k_full = [&](int i) { return smem_u32(&bars[1 + i]); };
-  auto v_full = [&](int i) { return smem_u32(&bars[3 + i]); };
-  auto k_empty = [&](int i) { return smem_u32(&bars[5 + i]); };
-  auto v_empty = [&](int i) { return smem_u32(&bars[7 + i]); };
-  auto s_full = [&](int i) { return smem_u32(&bars[9 + i]); };
-  auto s_free = [&](int i) { return smem_u32(&bars[11 + i]); };
-  auto p_full = [&](int i) { return smem_u32(&bars[13 + i]); };
-  auto pv_done = [&](int i) { return smem_u32(&bars[15 + i]); };
-  const uint32_t drain_bar = smem_u32(&bars[17]);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[18]);
+  // s_full[X], p_full[X], pv_done[X], q_full, drain, full[slot], empty[slot]
+  constexpr int NS = L::SLOTS;
+  static_assert(NS >= 2 && 7 + 2 * NS + 1 <= 32, "barrier area holds 32 words");
+  auto s_full = [&](int x) { return smem_u32(&bars[0 + x]); };
+  auto p_full = [&](int x) { return smem_u32(&bars[2 + x]); };
+  auto pv_done = [&](int x) { return smem_u32(&bars[4 + x]); };
+  const uint32_t q_full = smem_u32(&bars[6]);
+  const uint32_t drain_bar = smem_u32(&bars[7]);
+  auto full = [&](int i) { return smem_u32(&bars[8 + i]); };
+  auto empty = [&](int i) { return smem_u32(&bars[8 + NS + i]); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[8 + 2 * NS]);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sQ = smem_u32(sm + L::Q_OFF);
-  const uint32_t sK = smem_u32(sm + L::K_OFF);
-  const uint32_t sV = smem_u32(sm + L::V_OFF);
-  const uint32_t sP = smem_u32(sm + L::P_OFF);
+  const uint32_t sRing = smem_u32(sm + L::RING_OFF);
+  // ring item n: K tile n/2 (n even) or V tile n/2 (n odd); slot n % NS, use n / NS
+  auto slot_of = [&](int n) { return n % NS; };
+  auto use_par = [&](int n) { return (uint32_t)((n / NS) & 1); };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(full(i), 1);
+      mbar_init(empty(i), 1);
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(k_full(i), 1);
-      mbar_init(v_full(i), 1);
-      mbar_init(k_empty(i), 1);
-      mbar_init(v_empty(i), 1);
       mbar_init(s_full(i), 1);
-      mbar_init(s_free(i), 128);
-      mbar_init(p_full(i), 128);
+      mbar_init(p_full(i), 32 * live_warps(i));
       mbar_init(pv_done(i), 1);
     }
     mbar_init(drain_bar, 1);
@@ -188,209 +222,196 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;            // two S buffers of 128 columns
-  const uint32_t tO = tmem + 2 * BKV;  // O buffer of HD columns
+  auto tS = [&](int x) { return tmem + (uint32_t)(x * 128); };
+  auto tO = [&](int x) { return tmem + 256u + (uint32_t)(x * 128); };
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
       const int krow0 = b * p.Nseq;
-      uint32_t issued = 0, issue_par = 0;  // bit i: K stage i (0,1), V stage i (2,3)
+      uint32_t issued = 0, issue_par = 0;  // per slot: a load in flight, its parity
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, L::Q_BYTES);
-      for (int c = 0; c < NB; ++c)
-        tma_load_2d(sQ + c * BQ * 128, &tmQ, q_full, h * HD + c * 64, off + q0);
-      for (int j = 0; j < T && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t par = ((j >> 1) & 1) ^ 1u;
-        if (!mbar_wait(k_empty(st), par, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(k_full(st), L::KV_BYTES);
+      mbar_arrive_expect_tx(q_full, nt * L::Q_TILE);
+      for (int x = 0; x < nt; ++x)
         for (int c = 0; c < NB; ++c)
-          tma_load_2d(sK + st * L::KV_BYTES + c * BKV * 128, &tmK, k_full(st), g * HD + c * 64,
-                      krow0 + j * BKV);
-        issued |= 1u << st;
-        issue_par = (issue_par & ~(1u << st)) | (((uint32_t)(j >> 1) & 1u) << st);
-        if (!mbar_wait(v_empty(st), par, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(v_full(st), L::KV_BYTES);
+          tma_load_2d(sQ + x * L::Q_TILE + c * BT * 128, &tmQ, q_full, h * HD + c * 64,
+                      off + q0 + x * BT);
+      for (int n = 0; n < 2 * T; ++n) {
+        const int j = n >> 1, sl = slot_of(n);
+        const uint32_t u = use_par(n);
+        if (!mbar_wait(empty(sl), u ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        mbar_arrive_expect_tx(full(sl), L::KV_BYTES);
+        const CUtensorMap* tm = (n & 1) ? &tmV : &tmK;
         for (int c = 0; c < NB; ++c)
-          tma_load_2d(sV + st * L::KV_BYTES + c * BKV * 128, &tmV, v_full(st), g * HD + c * 64,
+          tma_load_2d(sRing + sl * L::KV_BYTES + c * BKV * 128, tm, full(sl), g * HD + c * 64,
                       krow0 + j * BKV);
-        issued |= 1u << (2 + st);
-        issue_par = (issue_par & ~(1u << (2 + st))) | (((uint32_t)(j >> 1) & 1u) << (2 + st));
+        issued |= 1u << sl;
+        issue_par = (issue_par & ~(1u << sl)) | (u << sl);
       }
       if (!ok) {
         wait_drain(q_full, 0);
-        for (int st = 0; st < 2; ++st) {
-          if (issued & (1u << st)) wait_drain(k_full(st), (issue_par >> st) & 1u);
-          if (issued & (1u << (2 + st))) wait_drain(v_full(st), (issue_par >> (2 + st)) & 1u);
-        }
+        for (int sl = 0; sl < NS; ++sl)
+          if (issued & (1u << sl)) wait_drain(full(sl), (issue_par >> sl) & 1u);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_qk = umma_idesc_bf16(BQ, BKV);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16(BQ, HD) | (1u << 16);  // B (V) MN-major
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(BT, BKV);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(BT, HD) | (1u << 16);  // B (V) MN-major
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       bool any = false;
-      auto do_pv = [&](int j) -> bool {
-        const int st = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(p_full(st), par, abort_flag, p.status)) return false;
-        if (!mbar_wait(v_full(st), par, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t pb = sP + st * L::P_BYTES;
-        const uint32_t vb = sV + st * L::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t da = umma_desc_k_sw128(pb + (kk >> 2) * (BQ * 128) + (kk & 3) * 32);
-          const uint64_t db = umma_desc_mn_sw128(vb + kk * 2048, BKV * 128);
-          tc_mma_bf16(tO, da, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        any = true;
-        tc_commit(pv_done(st));
-        tc_commit(v_empty(st));
-        return true;
-      };
-      for (int j = 0; j < T && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(k_full(st), par, abort_flag, p.status)) { ok = false; break; }
-        if (j >= 2 && !mbar_wait(s_free(st), par ^ 1u, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kb = sK + st * L::KV_BYTES;
+      auto qk = [&](int x, int j) {
+        const uint32_t kb = sRing + slot_of(2 * j) * L::KV_BYTES;
+        const uint32_t qb = sQ + x * L::Q_TILE;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t da = umma_desc_k_sw128(sQ + (kk >> 2) * (BQ * 128) + (kk & 3) * 32);
+          const uint64_t da = umma_desc_k_sw128(qb + (kk >> 2) * (BT * 128) + (kk & 3) * 32);
           const uint64_t db = umma_desc_k_sw128(kb + (kk >> 2) * (BKV * 128) + (kk & 3) * 32);
-          tc_mma_bf16(tS + st * BKV, da, db, idesc_qk, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tS(x), da, db, idesc_qk, kk > 0 ? 1u : 0u);
         }
+        tc_commit(s_full(x));
         any = true;
-        tc_commit(s_full(st));
-        tc_commit(k_empty(st));
-        if (j >= 1 && !do_pv(j - 1)) { ok = false; break; }
+      };
+      auto pv = [&](int x, int j) -> bool {
+        if (!mbar_wait(p_full(x), j & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t vb = sRing + slot_of(2 * j + 1) * L::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint64_t db = umma_desc_mn_sw128(vb + kk * 2048, BKV * 128);
+          tc_mma_ts(tO(x), tS(x) + (uint32_t)(kk * 8), db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (j == T - 1) tc_commit(pv_done(x));  // single phase: O_X is final
+        return true;
+      };
+      auto wait_k = [&](int j) {
+        if (!mbar_wait(full(slot_of(2 * j)), use_par(2 * j), abort_flag, p.status)) return false;
+        tc_fence_after();
+        return true;
+      };
+      if (ok && (ok = wait_k(0))) {
+        for (int x = 0; x < nt; ++x) qk(x, 0);
+        tc_commit(empty(slot_of(0)));
       }
-      if (ok) ok = do_pv(T - 1);
+      for (int j = 0; j < T && ok; ++j) {
+        if (!mbar_wait(full(slot_of(2 * j + 1)), use_par(2 * j + 1), abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        const bool more = j + 1 < T;
+        if (!pv(0, j)) { ok = false; break; }
+        if (more) {
+          if (!wait_k(j + 1)) { ok = false; break; }
+          qk(0, j + 1);
+        }
+        if (nt == 2) {
+          if (!pv(1, j)) { ok = false; break; }
+          if (more) qk(1, j + 1);
+        }
+        tc_commit(empty(slot_of(2 * j + 1)));
+        if (more) tc_commit(empty(slot_of(2 * j + 2)));
+      }
       if (!ok && any) {
         tc_commit(drain_bar);
         wait_drain(drain_bar, 0);
       }
     }
   } else {
-    // ------------------------------------------------------------------ softmax warps
+    // ------------------------------------------------------------------ softmax groups
+    const int x = (warp - 2) >> 2;        // tile: 0 = A (warps 2-5), 1 = B (warps 6-9)
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // query row in the tile (= TMEM lane)
+    const int r = quad * 32 + lane;       // query row in the tile (= TMEM lane)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    float m_ref = -INFINITY, lsum = 0.f;
-    bool ok = true;
-    for (int j = 0; j < T; ++j) {
-      const int st = j & 1;
-      const uint32_t par = (j >> 1) & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(s_full(st), par, abort_flag, p.status));
-      if (!ok) break;
-      tc_fence_after();
-      float s[BKV];
-#pragma unroll
-      for (int c = 0; c < BKV; c += 32) tmem_ld32_nowait(tS + st * BKV + lane_off + c, s + c);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(s_free(st));
-      const int kbase = j * BKV;
-      // 8 independent max chains instead of one 128-long dependency
-      float mxv[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) mxv[t] = -INFINITY;
-      if (kbase + BKV <= p.Nseq) {
-#pragma unroll
-        for (int i = 0; i < BKV; ++i) {
-          s[i] *= p.scale_log2;
-          mxv[i & 7] = fmaxf(mxv[i & 7], s[i]);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < BKV; ++i) {
-          s[i] = (kbase + i < p.Nseq) ? s[i] * p.scale_log2 : -INFINITY;
-          mxv[i & 7] = fmaxf(mxv[i & 7], s[i]);
-        }
-      }
-      const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
-                             fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
-      // raise the reference maximum only when this tile exceeds it by > 2^8
-      const bool need = (j == 0) || (mx > m_ref + kRescaleLog2);
-      const bool rescale_o = __any_sync(0xffffffffu, need && j > 0);
-      float alpha = 1.f;
-      if (need) {
-        alpha = (j == 0) ? 0.f : exp2f(m_ref - mx);
-        m_ref = mx;
-      }
-      lsum *= (j == 0) ? 0.f : alpha;
-      // P buffer st was last read by PV_{j-2}
-      if (j >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(st), par ^ 1u, abort_flag, p.status));
-        if (!ok) break;
-      }
-      if (rescale_o) {
-        const int pj = j - 1;
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(pv_done(pj & 1), (pj >> 1) & 1, abort_flag, p.status));
+    // a warp whose 32 rows are all past the sequence's selected rows takes no part
+    if (x < nt && quad < live_warps(x)) {
+      const float sc = p.scale_log2;
+      float m_ref = -INFINITY, lsum = 0.f;  // reference maximum in the exp2 domain
+      bool ok = true;
+      for (int j = 0; j < T; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), j & 1, abort_flag, p.status));
         if (!ok) break;
         tc_fence_after();
+        float s[BKV];
+#pragma unroll
+        for (int c = 0; c < BKV; c += 32) tmem_ld32_nowait(tS(x) + lane_off + c, s + c);
+        tmem_wait_ld();
+        const int kbase = j * BKV;
+        if (kbase + BKV > p.Nseq) {
+#pragma unroll
+          for (int i = 0; i < BKV; ++i) s[i] = (kbase + i < p.Nseq) ? s[i] : -INFINITY;
+        }
+        // the maximum of the raw scores (the scale is positive)
+        float mxv[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mxv[t] = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < BKV; i += 2) mxv[(i >> 1) & 3] = fmax3(mxv[(i >> 1) & 3], s[i], s[i + 1]);
+        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])) * sc;
+        // raise the reference maximum only when this tile exceeds it by > 2^8
+        const bool need = (j == 0) || (mx > m_ref + kRescaleLog2);
+        const bool rescale_o = __any_sync(0xffffffffu, need && j > 0);
+        float alpha = 1.f;
+        if (need) {
+          alpha = (j == 0) ? 0.f : ex2_approx(m_ref - mx);
+          m_ref = mx;
+        }
+        lsum *= (j == 0) ? 0.f : alpha;
+        if (rescale_o) {
+          // S_X(j) complete implies PV_X(j-1) complete: O_X is stable until P_X(j) is ready
+#pragma unroll 1
+          for (int c = 0; c < HD; c += 32) {
+            float o[32];
+            tmem_ld32_nowait(tO(x) + lane_off + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO(x) + lane_off + c, reinterpret_cast<const uint32_t*>(o));
+          }
+          tmem_wait_st();
+        }
+        const float neg_m = -m_ref;
+        float rsv[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) rsv[t] = 0.f;
+        uint32_t pk[BKV / 2];
+#pragma unroll
+        for (int i = 0; i < BKV; i += 2) {
+          const float x0 = fmaf(s[i], sc, neg_m), x1 = fmaf(s[i + 1], sc, neg_m);
+          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          rsv[i & 7] += e0;
+          rsv[(i + 1) & 7] += e1;
+          pk[i >> 1] = pack_bf2(e0, e1);
+        }
+        lsum += ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
+        // P_X over the first 64 columns of S_X (S_X has been read into registers)
+        tmem_st32(tS(x) + lane_off, pk);
+        tmem_st32(tS(x) + lane_off + 32, pk + 32);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full(x));
+      }
+      if (ok) {
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(x), 0, abort_flag, p.status));
+      }
+      if (ok) {
+        tc_fence_after();
+        const int row = q0 + x * BT + r;
+        const float inv = 1.0f / lsum;
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           float o[32];
-          tmem_ld32(tO + lane_off + c, o);
+          tmem_ld32_nowait(tO(x) + lane_off + c, o);
+          tmem_wait_ld();
+          if (row < cnt) {
+            __nv_bfloat16* dst = p.O + (size_t)(off + row) * p.ldo + h * HD + c;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st_32x32b_x32(tO + lane_off + c, o);
-        }
-        tmem_wait_st();
-      }
-      float rsv[8];
+            for (int i = 0; i < 32; i += 8) {
+              float f[8];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) rsv[t] = 0.f;
-      const uint32_t prow = sP + st * L::P_BYTES + r * 128;
-#pragma unroll
-      for (int blk = 0; blk < 2; ++blk) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          float e[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            e[i] = exp2f(s[blk * 64 + ch * 8 + i] - m_ref);
-            rsv[i] += e[i];
-          }
-          const uint4 v = pack8(e);
-          const uint32_t addr = prow + blk * (BQ * 128) + ((ch ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-                       "r"(v.z), "r"(v.w)
-                       : "memory");
-        }
-      }
-      lsum += ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(p_full(st));
-    }
-    if (ok) {
-      const int jl = T - 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(pv_done(jl & 1), (jl >> 1) & 1, abort_flag, p.status));
-    }
-    if (ok) {
-      tc_fence_after();
-      const int row = q0 + r;
-      const float inv = 1.0f / lsum;
-#pragma unroll 1
-      for (int c = 0; c < HD; c += 32) {
-        float o[32];
-        tmem_ld32(tO + lane_off + c, o);
-        if (row < cnt) {
-          __nv_bfloat16* dst = p.O + (size_t)(off + row) * p.ldo + h * HD + c;
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            float f[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) f[t] = o[i + t] * inv;
-            *reinterpret_cast<uint4*>(dst + i) = pack8(f);
+              for (int t = 0; t < 8; ++t) f[t] = o[i + t] * inv;
+              *reinterpret_cast<uint4*>(dst + i) = pack8(f);
+            }
           }
         }
       }
@@ -403,10 +424,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
-}
-
-bool map2d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  return tmap_bf16_2d(m, ptr, rows, cols, box_rows);
 }
 
 template <int HD>
@@ -433,11 +450,13 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
   if (B <= 0 || k_cap <= 0 || M_cap <= 0) return cudaSuccess;
   if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
-  if (!map2d(&tq, q, (uint64_t)M_cap, (uint64_t)Hq * hd, BQ)) return cudaErrorInvalidValue;
-  if (!map2d(&tk, kc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV)) return cudaErrorInvalidValue;
-  if (!map2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV)) return cudaErrorInvalidValue;
+  if (!tmap_bf16_2d(&tq, q, (uint64_t)M_cap, (uint64_t)Hq * hd, BT)) return cudaErrorInvalidValue;
+  if (!tmap_bf16_2d(&tk, kc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
+    return cudaErrorInvalidValue;
+  if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
+    return cudaErrorInvalidValue;
   AttnParams p{row_off, o, Nseq, Hq, Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd), status};
-  dim3 grid((k_cap + BQ - 1) / BQ, Hq, B);
+  dim3 grid((k_cap + NTILE * BT - 1) / (NTILE * BT), Hq, B);
   ProfScope prof("attention", s);
   return hd == 128 ? launch_hd<128>(tq, tk, tv, p, grid, s) : launch_hd<64>(tq, tk, tv, p, grid, s);
 }

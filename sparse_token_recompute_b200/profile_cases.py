@@ -136,12 +136,13 @@ def main():
     ap.add_argument("--d", type=int, default=4096)
     ap.add_argument("--V", type=int, default=32768)
     ap.add_argument("--Mm", type=int, default=256)
-    ap.add_argument("--k", type=int, default=256)
+    ap.add_argument("--k", type=int, default=None,
+                    help="rows per sequence (default 256 for score, 308 for layer/attention)")
     ap.add_argument("--warmup", type=int, default=2)
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
-    if a.case in ("layer", "attention") and a.k == 256:
-        a.k = 308
+    if a.k is None:
+        a.k = 308 if a.case in ("layer", "attention") else 256
     if a.case in ("layer", "attention"):
         a.N = 1536 if a.N == 12288 else a.N
     out = {"gemm": case_gemm, "score": case_score, "layer": case_layer,
