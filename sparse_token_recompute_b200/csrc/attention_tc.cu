@@ -48,15 +48,16 @@ struct Smem {
   static constexpr int KV_BYTES = BKV * HD * 2;
   // K and V tiles share one ring of slots in consumption order K0 V0 K1 V1 ...,
   // as many as fit next to the two Q tiles (at most 8)
-  static constexpr int SLOTS_FIT = (kSmemMax - 1280 - NTILE * Q_TILE) / KV_BYTES;
+  static constexpr int SLOTS_FIT = (kSmemMax - 2304 - NTILE * Q_TILE) / KV_BYTES;
   static constexpr int SLOTS = SLOTS_FIT < 8 ? SLOTS_FIT : 8;
   static constexpr int Q_OFF = 0;
   static constexpr int RING_OFF = Q_OFF + NTILE * Q_TILE;
   static constexpr int BAR_OFF = RING_OFF + SLOTS * KV_BYTES;
+  static constexpr int STAT_OFF = BAR_OFF + 256;  // 2 x 128 floats for the key-split merge
   // + barriers + alignment slack; at least 116 KB so that one CTA (which holds
   // all 512 TMEM columns) is resident per SM
-  static constexpr int TOTAL = (BAR_OFF + 256 + 1024) > 116 * 1024 ? (BAR_OFF + 256 + 1024)
-                                                                   : 116 * 1024;
+  static constexpr int TOTAL = (STAT_OFF + 1024 + 1024) > 116 * 1024 ? (STAT_OFF + 1024 + 1024)
+                                                                     : 116 * 1024;
 };
 
 struct AttnParams {
@@ -115,6 +116,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// barrier `id` over `count` threads (a multiple of 32) of the block
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
   __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&t);
@@ -161,19 +167,29 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int cnt = p.row_off[b + 1] - off;
   const int q0 = blockIdx.x * (NTILE * BT);
   if (q0 >= cnt) return;
-  const int nt = (cnt - q0 > BT) ? 2 : 1;  // query tiles holding rows in this CTA
-  // softmax warps of tile x that hold at least one selected row
+  const int T = (p.Nseq + BKV - 1) / BKV;
+  const int nq = (cnt - q0 > BT) ? 2 : 1;  // query tiles holding rows in this CTA
+  // A lone query tile splits the keys instead: group A takes K/V tiles [0, TA),
+  // group B [TA, T), and the two partial softmax results are merged at the end.
+  const bool split = nq == 1 && T >= 2;
+  const int TA = split ? (T + 1) / 2 : T;
+  const int TB = split ? T - TA : T;
+  const int ngroups = (nq == 2 || split) ? 2 : 1;
+  auto ntiles = [&](int x) { return x == 0 ? TA : TB; };         // K/V tiles of group x
+  auto kv_first = [&](int x) { return (split && x == 1) ? TA : 0; };
+  auto qtile = [&](int x) { return split ? 0 : x; };             // query tile of group x
+  // softmax warps of group x that hold at least one selected row
   auto live_warps = [&](int x) {
-    const int rows = min(BT, cnt - q0 - x * BT);
+    const int rows = min(BT, cnt - q0 - qtile(x) * BT);
     return rows > 0 ? (rows + 31) / 32 : 1;
   };
   const int g = (h * p.Hkv) / p.Hq;
-  const int T = (p.Nseq + BKV - 1) / BKV;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR_OFF);
+  float* stat = reinterpret_cast<float*>(sm + L::STAT_OFF);  // group B's (m, l) per row
   // s_full[X], p_full[X], pv_done[X], q_full, drain, full[slot], empty[slot]
   constexpr int NS = L::SLOTS;
   static_assert(NS >= 2 && 7 + 2 * NS + 1 <= 32, "barrier area holds 32 words");
@@ -190,7 +206,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sQ = smem_u32(sm + L::Q_OFF);
   const uint32_t sRing = smem_u32(sm + L::RING_OFF);
-  // ring item n: K tile n/2 (n even) or V tile n/2 (n odd); slot n % NS, use n / NS
+  // The n-th K or V tile through the ring occupies slot n % NS for its (n / NS)-th use.
+  // Producer and issuer walk the same sequence of tiles:
+  //   two query tiles:  K0, V0, K1, V1, ...              (each read by both groups)
+  //   split keys:       K0, K_TA, then per j: V_j, K_{j+1}, V_{TA+j}, K_{TA+j+1}
   auto slot_of = [&](int n) { return n % NS; };
   auto use_par = [&](int n) { return (uint32_t)((n / NS) & 1); };
 
@@ -230,23 +249,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---------------------------------------------------------------- producer
       const int krow0 = b * p.Nseq;
       uint32_t issued = 0, issue_par = 0;  // per slot: a load in flight, its parity
-      bool ok = true;
-      mbar_arrive_expect_tx(q_full, nt * L::Q_TILE);
-      for (int x = 0; x < nt; ++x)
+      int n = 0;
+      auto load = [&](bool is_v, int tile) -> bool {
+        const int sl = slot_of(n);
+        const uint32_t u = use_par(n);
+        if (!mbar_wait(empty(sl), u ^ 1u, abort_flag, p.status)) return false;
+        mbar_arrive_expect_tx(full(sl), L::KV_BYTES);
+        const CUtensorMap* tm = is_v ? &tmV : &tmK;
+        for (int c = 0; c < NB; ++c)
+          tma_load_2d(sRing + sl * L::KV_BYTES + c * BKV * 128, tm, full(sl), g * HD + c * 64,
+                      krow0 + tile * BKV);
+        issued |= 1u << sl;
+        issue_par = (issue_par & ~(1u << sl)) | (u << sl);
+        ++n;
+        return true;
+      };
+      mbar_arrive_expect_tx(q_full, nq * L::Q_TILE);
+      for (int x = 0; x < nq; ++x)
         for (int c = 0; c < NB; ++c)
           tma_load_2d(sQ + x * L::Q_TILE + c * BT * 128, &tmQ, q_full, h * HD + c * 64,
                       off + q0 + x * BT);
-      for (int n = 0; n < 2 * T; ++n) {
-        const int j = n >> 1, sl = slot_of(n);
-        const uint32_t u = use_par(n);
-        if (!mbar_wait(empty(sl), u ^ 1u, abort_flag, p.status)) { ok = false; break; }
-        mbar_arrive_expect_tx(full(sl), L::KV_BYTES);
-        const CUtensorMap* tm = (n & 1) ? &tmV : &tmK;
-        for (int c = 0; c < NB; ++c)
-          tma_load_2d(sRing + sl * L::KV_BYTES + c * BKV * 128, tm, full(sl), g * HD + c * 64,
-                      krow0 + j * BKV);
-        issued |= 1u << sl;
-        issue_par = (issue_par & ~(1u << sl)) | (u << sl);
+      bool ok;
+      if (!split) {
+        ok = load(false, 0);
+        for (int j = 0; j < T && ok; ++j) {
+          ok = load(true, j);
+          if (ok && j + 1 < T) ok = load(false, j + 1);
+        }
+      } else {
+        ok = load(false, 0) && load(false, TA);
+        for (int j = 0; j < TA && ok; ++j) {
+          ok = load(true, j);
+          if (ok && j + 1 < TA) ok = load(false, j + 1);
+          if (ok && j < TB) ok = load(true, TA + j);
+          if (ok && j + 1 < TB) ok = load(false, TA + j + 1);
+        }
       }
       if (!ok) {
         wait_drain(q_full, 0);
@@ -261,9 +298,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idesc_pv = umma_idesc_bf16(BT, HD) | (1u << 16);  // B (V) MN-major
       bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
       bool any = false;
-      auto qk = [&](int x, int j) {
-        const uint32_t kb = sRing + slot_of(2 * j) * L::KV_BYTES;
-        const uint32_t qb = sQ + x * L::Q_TILE;
+      int m = 0;  // ring tiles consumed
+      auto take = [&]() -> int {  // slot of the next ring tile, once it has landed
+        const int sl = slot_of(m);
+        if (!mbar_wait(full(sl), use_par(m), abort_flag, p.status)) return -1;
+        tc_fence_after();
+        ++m;
+        return sl;
+      };
+      auto give = [&](int sl) { tc_commit(empty(sl)); };
+      auto qk = [&](int x, int sl) {
+        const uint32_t kb = sRing + sl * L::KV_BYTES;
+        const uint32_t qb = sQ + qtile(x) * L::Q_TILE;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint64_t da = umma_desc_k_sw128(qb + (kk >> 2) * (BT * 128) + (kk & 3) * 32);
@@ -273,44 +319,67 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_commit(s_full(x));
         any = true;
       };
-      auto pv = [&](int x, int j) -> bool {
+      auto pv = [&](int x, int j, int sl) -> bool {
         if (!mbar_wait(p_full(x), j & 1, abort_flag, p.status)) return false;
         tc_fence_after();
-        const uint32_t vb = sRing + slot_of(2 * j + 1) * L::KV_BYTES;
+        const uint32_t vb = sRing + sl * L::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk) {
           const uint64_t db = umma_desc_mn_sw128(vb + kk * 2048, BKV * 128);
           tc_mma_ts(tO(x), tS(x) + (uint32_t)(kk * 8), db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        if (j == T - 1) tc_commit(pv_done(x));  // single phase: O_X is final
+        if (j == ntiles(x) - 1) tc_commit(pv_done(x));  // single phase: O_X is final
         return true;
       };
-      auto wait_k = [&](int j) {
-        if (!mbar_wait(full(slot_of(2 * j)), use_par(2 * j), abort_flag, p.status)) return false;
-        tc_fence_after();
-        return true;
-      };
-      if (ok && (ok = wait_k(0))) {
-        for (int x = 0; x < nt; ++x) qk(x, 0);
-        tc_commit(empty(slot_of(0)));
-      }
-      for (int j = 0; j < T && ok; ++j) {
-        if (!mbar_wait(full(slot_of(2 * j + 1)), use_par(2 * j + 1), abort_flag, p.status)) {
-          ok = false;
-          break;
+      if (ok && !split) {
+        const int sk = take();
+        ok = sk >= 0;
+        if (ok) {
+          for (int x = 0; x < nq; ++x) qk(x, sk);
+          give(sk);
         }
-        const bool more = j + 1 < T;
-        if (!pv(0, j)) { ok = false; break; }
-        if (more) {
-          if (!wait_k(j + 1)) { ok = false; break; }
-          qk(0, j + 1);
+        for (int j = 0; j < T && ok; ++j) {
+          const int sv = take();
+          if (!(ok = sv >= 0 && pv(0, j, sv))) break;
+          int sk1 = -1;
+          if (j + 1 < T) {
+            if (!(ok = (sk1 = take()) >= 0)) break;
+            qk(0, sk1);
+          }
+          if (nq == 2) {
+            if (!(ok = pv(1, j, sv))) break;
+            if (sk1 >= 0) qk(1, sk1);
+          }
+          give(sv);
+          if (sk1 >= 0) give(sk1);
         }
-        if (nt == 2) {
-          if (!pv(1, j)) { ok = false; break; }
-          if (more) qk(1, j + 1);
+      } else if (ok) {
+        for (int x = 0; x < 2 && ok; ++x) {
+          const int sk = take();
+          if ((ok = sk >= 0)) {
+            qk(x, sk);
+            give(sk);
+          }
         }
-        tc_commit(empty(slot_of(2 * j + 1)));
-        if (more) tc_commit(empty(slot_of(2 * j + 2)));
+        for (int j = 0; j < TA && ok; ++j) {
+          int sl;
+          if (!(ok = (sl = take()) >= 0 && pv(0, j, sl))) break;
+          give(sl);
+          if (j + 1 < TA) {
+            if (!(ok = (sl = take()) >= 0)) break;
+            qk(0, sl);
+            give(sl);
+          }
+          if (j < TB) {
+            if (!(ok = (sl = take()) >= 0 && pv(1, j, sl))) break;
+            give(sl);
+          }
+          if (j + 1 < TB) {
+            if (!(ok = (sl = take()) >= 0)) break;
+            qk(1, sl);
+            give(sl);
+          }
+        }
       }
       if (!ok && any) {
         tc_commit(drain_bar);
@@ -319,16 +388,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax groups
-    const int x = (warp - 2) >> 2;        // tile: 0 = A (warps 2-5), 1 = B (warps 6-9)
+    const int x = (warp - 2) >> 2;        // group: 0 = A (warps 2-5), 1 = B (warps 6-9)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;       // query row in the tile (= TMEM lane)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     // a warp whose 32 rows are all past the sequence's selected rows takes no part
-    if (x < nt && quad < live_warps(x)) {
+    if (x < ngroups && quad < live_warps(x)) {
       const float sc = p.scale_log2;
       float m_ref = -INFINITY, lsum = 0.f;  // reference maximum in the exp2 domain
       bool ok = true;
-      for (int j = 0; j < T; ++j) {
+      const int nj = ntiles(x);
+      for (int j = 0; j < nj; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), j & 1, abort_flag, p.status));
         if (!ok) break;
         tc_fence_after();
@@ -336,7 +406,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int c = 0; c < BKV; c += 32) tmem_ld32_nowait(tS(x) + lane_off + c, s + c);
         tmem_wait_ld();
-        const int kbase = j * BKV;
+        const int kbase = (kv_first(x) + j) * BKV;
         if (kbase + BKV > p.Nseq) {
 #pragma unroll
           for (int i = 0; i < BKV; ++i) s[i] = (kbase + i < p.Nseq) ? s[i] : -INFINITY;
@@ -391,17 +461,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         mbar_arrive(p_full(x));
       }
-      if (ok) {
-        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(x), 0, abort_flag, p.status));
-      }
-      if (ok) {
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done(x), 0, abort_flag, p.status));
+      if (split) {
+        // group B hands its (m, l) to group A, which merges O_B into O_A
+        if (x == 1) {
+          stat[r] = m_ref;
+          stat[BT + r] = lsum;
+        }
+        tc_fence_before();
+        named_bar_sync(1, 2 * 32 * live_warps(0));
         tc_fence_after();
-        const int row = q0 + x * BT + r;
+      }
+      if (ok && (x == 0 || !split)) {
+        const int row = q0 + qtile(x) * BT + r;
+        float wa = 1.f, wb = 0.f;
+        if (split) {
+          const float mb = stat[r], lb = stat[BT + r];
+          const float mm = fmaxf(m_ref, mb);
+          wa = ex2_approx(m_ref - mm);
+          wb = ex2_approx(mb - mm);
+          lsum = lsum * wa + lb * wb;
+        }
         const float inv = 1.0f / lsum;
+        wa *= inv;
+        wb *= inv;
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
-          float o[32];
+          float o[32], ob[32];
           tmem_ld32_nowait(tO(x) + lane_off + c, o);
+          if (split) tmem_ld32_nowait(tO(1) + lane_off + c, ob);
           tmem_wait_ld();
           if (row < cnt) {
             __nv_bfloat16* dst = p.O + (size_t)(off + row) * p.ldo + h * HD + c;
@@ -409,7 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int i = 0; i < 32; i += 8) {
               float f[8];
 #pragma unroll
-              for (int t = 0; t < 8; ++t) f[t] = o[i + t] * inv;
+              for (int t = 0; t < 8; ++t) f[t] = split ? o[i + t] * wa + ob[i + t] * wb : o[i + t] * wa;
               *reinterpret_cast<uint4*>(dst + i) = pack8(f);
             }
           }

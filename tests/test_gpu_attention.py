@@ -16,6 +16,7 @@ pytestmark = pytest.mark.gpu
     (3, 1000, 4, 2, 64, [1, 256, 300]),    # GQA, hd 64, three query tiles
     (1, 2048, 28, 4, 128, [103]),          # 7B-class head layout
     (2, 64, 8, 8, 128, [0, 64]),           # a sequence with no rows, keys < one tile
+    (2, 300, 2, 1, 128, [100, 257]),       # lone tiles split the keys 2 + 1 tiles (ragged)
 ])
 def test_attention_matches_oracle(lib, B, N, Hq, Hkv, hd, counts):
     k_cap = max(max(counts), 1)
