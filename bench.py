@@ -37,6 +37,12 @@ import dllm_synth as SY  # noqa: E402
 METRIC = "tokens/s & denoise steps/s at 8B shape, bs 1/32; % of HBM / bf16 TC roofline"
 SHAPE = SY.DENSE8B_B32_N1536
 BS1 = SY.DENSE8B_B1_N768
+GQA = SY.GQA7B_B8_N2048
+# DRAM bytes (read + write) per launch of the layer-projection GEMM, averaged over
+# its four launches per layer (QKV, O, gate/up, down) at 32 x 308 rows of the 8B
+# layer, from the ncu capture summarised in
+# profiles/gemm_tc_8b_layer_b32_n1536_k308_dram.md; re-take it when gemm_tc changes.
+GEMM_TRAFFIC_PER_LAUNCH = 935.7e6
 
 
 def parse():
@@ -47,6 +53,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-bs1", action="store_true", help="skip the batch-1 measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gqa", action="store_true", help="skip the 7B GQA ratio sweep")
     ap.add_argument("--layers", type=int, default=0, help="(debug) override the layer count")
     return ap.parse_args()
 
@@ -182,7 +189,7 @@ def bs1_measure(S, W, steps, warmup):
     out = {}
     model = S.Model(S.cfg_from_shape(BS1), W)
     stream = torch.cuda.current_stream()
-    for ratio in (0.10, 0.25, 0.50):
+    for ratio in (0.10, 0.25, 0.50, 1.0):
         shape = SY.with_(BS1, ratio=ratio)
         tokens = SY.prompt_tokens(shape, seed=7, device="cuda")
         cache = S.Cache(model.cfg, 1, shape.seq_len)
@@ -221,6 +228,64 @@ def bs1_measure(S, W, steps, warmup):
                                        "kernels_ms_per_step": {
                                            n: [v[0] // K, round(v[1] / K, 4)]
                                            for n, v in sorted(prof.items())}}
+        del cache, ws
+    return out
+
+
+def gemm_bytes_per_launch(shape):
+    """Algorithmic bytes of the four projection GEMMs of one layer (A, weights, residual
+    in/out, outputs incl. the K/V rows scattered into the cache), averaged per launch."""
+    M = shape.batch * shape.k
+    d, q, kv, f = shape.d, shape.n_heads * shape.head_dim, shape.n_kv_heads * shape.head_dim, shape.ffn
+    e = 2
+    qkv = (M * d + (q + 2 * kv) * d + M * (q + 2 * kv)) * e
+    o = (M * q + d * q + 2 * M * d) * e
+    gu = (M * d + 2 * f * d + M * f) * e
+    down = (M * f + d * f + 2 * M * d) * e
+    return (qkv + o + gu + down) / 4.0
+
+
+def dense_step_ms(S, model, cache, tokens, pol, ws, stream, reps=2):
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        S.dllm_step(model, cache, tokens, pol, True, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def gqa_measure(S, steps, warmup):
+    """7B GQA shape (28 query / 4 K/V heads), 8 x 2048 tokens: one partial step at
+    5 ... 100 % recompute, and the dense step for comparison."""
+    import torch
+    stream = torch.cuda.current_stream()
+    W = SY.model_weights(GQA, seed=0, device="cuda")
+    model = S.Model(S.cfg_from_shape(GQA), W)
+    out = {"workload": f"7B-shaped GQA ({GQA.n_heads}q/{GQA.n_kv_heads}kv heads, d {GQA.d}, "
+                       f"ffn {GQA.ffn}, {GQA.n_layers} layers), {GQA.batch} x {GQA.seq_len} "
+                       f"tokens ({GQA.prompt_len} prompt + {GQA.gen_len} generated), "
+                       f"{GQA.n_unmask} revealed/seq/step"}
+    for ratio in (0.05, 0.10, 0.25, 0.50, 0.75, 1.0):
+        shape = SY.with_(GQA, ratio=ratio)
+        tokens = SY.prompt_tokens(shape, seed=9, device="cuda")
+        cache = S.Cache(model.cfg, shape.batch, shape.seq_len)
+        pol = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k,
+                            n_unmask=shape.n_unmask, gen_start=shape.prompt_len,
+                            block_len=shape.block_len)
+        ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+        S.dllm_step(model, cache, tokens, pol, True, ws)
+        for _ in range(warmup):
+            S.dllm_step(model, cache, tokens, pol, False, ws)
+        torch.cuda.synchronize()
+        K = min(steps, 10)
+        ms = time_steps(S, model, cache, tokens, pol, ws, K, stream) / K
+        out[f"r{int(round(ratio * 100))}"] = {
+            "k": shape.k, "ms_per_step": round(ms, 4), "steps_per_s": round(1000.0 / ms, 2),
+            "tokens_per_s": round(shape.batch * shape.n_unmask * 1000.0 / ms, 1)}
+        if ratio == 1.0:
+            out["dense_step_ms"] = round(dense_step_ms(S, model, cache, tokens, pol, ws, stream), 4)
         del cache, ws
     return out
 
@@ -318,6 +383,12 @@ def run_ours(args):
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
     barrier(world)
 
+    # a whole generation: dense step 0, then gen_len / n_unmask - 1 partial steps
+    ms_dense = max_over_ranks(dense_step_ms(S, model, cache, tokens, pol, ws, stream), world)
+    barrier(world)
+    n_gen = shape.gen_len // shape.n_unmask
+    gen_s = (ms_dense + (n_gen - 1) * ms_step) / 1000.0
+
     # roofline of the dominant kernel: the tensor-core GEMM of the layer projections
     M = shape.batch * shape.k
     q = shape.n_heads * shape.head_dim
@@ -353,7 +424,18 @@ def run_ours(args):
             "frac": round(achieved / tc_sus, 4) if achieved else None,
             "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long step)",
             "flops_per_step": flops_step, "launches": gemm_launches,
-            "avg_launch_ms": round(gemm_ms / max(gemm_launches, 1), 4), "traffic": None},
+            "avg_launch_ms": round(gemm_ms / max(gemm_launches, 1), 4),
+            "traffic": GEMM_TRAFFIC_PER_LAUNCH,
+            "algorithmic_bytes_per_launch": round(gemm_bytes_per_launch(shape)),
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, one capture "
+                              "of one 8B layer at 32 x 308 rows (same launches as here)"},
+        "generation": {
+            "steps": n_gen, "dense_step_ms": round(ms_dense, 4), "partial_step_ms": round(ms_step, 4),
+            "total_s": round(gen_s, 4),
+            "tokens_per_s": round(world * shape.batch * shape.gen_len / gen_s, 2),
+            "steps_per_s": round(n_gen / gen_s, 3),
+            "how": f"step 0 dense + {n_gen - 1} partial steps at the timed per-step cost; "
+                   f"tokens = sequences x {shape.gen_len} generated"},
         "e2e": {"value": round(job_tokens_per_s(world, tok_per_step, ms_e2e), 2), "unit": "tokens/s",
                 "ms_per_step": round(ms_e2e, 4),
                 "h2d_bytes_per_step": tokens.numel() * 4,
@@ -368,6 +450,10 @@ def run_ours(args):
         del cache, ws
         torch.cuda.empty_cache()
         result["bs1"] = bs1_measure(S, W, args.steps, args.warmup)
+    if not args.no_gqa and not args.layers and world == 1:
+        del W, model
+        torch.cuda.empty_cache()
+        result["gqa7b"] = gqa_measure(S, args.steps, args.warmup)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
