@@ -53,6 +53,20 @@ in the design notes):
   * Unmasking reveals, in the first generation block that still holds a
     masked position, the n masked positions of highest confidence
     (ties: lower position first) [SF-de §2].
+  * Over-threshold unmasking (the fast phase of [SF-de §2]): with a
+    threshold tau_u > 0, every masked position of the current block whose
+    confidence is strictly above tau_u is revealed; when fewer than n are
+    above it, the top-n rule applies instead.  Both cases reveal the
+    max(n, #above) most confident masked positions.  The stable region of
+    the fast phase is read as the current block (the pages give no rule
+    for the region's end point or the variance window).
+  * Response-only steps [DyLLM §2.C]: rows before select_from (the prompt)
+    are never selected in a partial step; their K/V stay as cached until a
+    dense step injects the prompt again.
+  * Periodic refresh [ES-nl Methodologie 3]: in a generation, a step is
+    dense (every row recomputed, every cache rewritten) at step 0, every
+    refresh_every steps, and, with refresh_on_block, at the first step at
+    which any sequence's current block differs from the previous step's.
 
 Parity pins: every public function here is pinned by tests under
 ``tests/test_oracle_*.py`` (closed forms, textbook/library special cases,
@@ -176,6 +190,10 @@ class Policy:
     n_unmask: int = 1
     gen_start: int = 0
     block_len: int = 32
+    select_from: int = 0          # positions below it are never selected (partial steps)
+    unmask_tau: float = 0.0       # > 0: over-threshold unmasking with top-n fallback
+    refresh_every: int = 0        # generation: dense step every R steps (0: never)
+    refresh_on_block: bool = False  # generation: dense step when a block changes
 
 
 @dataclass
@@ -382,14 +400,16 @@ def select_thresh(scores: np.ndarray, tau: float, k_cap: int):
     return np.array(sorted(over), dtype=np.int64), n_over
 
 
-def select(scores: np.ndarray, mode: int, k: int, tau: float, k_cap: int):
-    """Per-sequence selection over scores [B, N] -> list of ascending index arrays."""
+def select(scores: np.ndarray, mode: int, k: int, tau: float, k_cap: int, lo: int = 0):
+    """Per-sequence selection over scores [B, N] -> list of ascending index arrays.
+    Only positions >= lo are candidates (response-only steps, [DyLLM §2.C])."""
     out = []
     for b in range(scores.shape[0]):
+        sub = scores[b, lo:]
         if mode == SELECT_TOPK:
-            out.append(select_topk(scores[b], min(k, k_cap)))
+            out.append(lo + select_topk(sub, min(k, k_cap)))
         else:
-            out.append(select_thresh(scores[b], tau, k_cap)[0])
+            out.append(lo + select_thresh(sub, tau, k_cap)[0])
     return out
 
 
@@ -404,22 +424,34 @@ def current_block(tokens_b: np.ndarray, mask_id: int, gen_start: int, block_len:
     return start, min(start + block_len, N)
 
 
-def unmask_positions(conf_b, tokens_b, mask_id: int, gen_start: int, block_len: int, n: int):
-    """Positions revealed in one sequence this step, ascending [SF-de §2]."""
+def unmask_positions(conf_b, tokens_b, mask_id: int, gen_start: int, block_len: int, n: int,
+                     tau: float = 0.0):
+    """Positions revealed in one sequence this step, ascending [SF-de §2].
+    tau > 0: every masked position of the block with conf > tau, or the top n
+    when fewer than n are above it."""
     blk = current_block(tokens_b, mask_id, gen_start, block_len)
     if blk is None or n <= 0:
         return np.zeros(0, dtype=np.int64)
     cand = [p for p in range(blk[0], blk[1]) if tokens_b[p] == mask_id]
+    take = n
+    if tau > 0:
+        above = [p for p in cand if float(conf_b[p]) > tau]
+        take = max(n, len(above))
     cand.sort(key=lambda p: _rank_key(conf_b[p], p), reverse=True)
-    return np.array(sorted(cand[:n]), dtype=np.int64)
+    return np.array(sorted(cand[:take]), dtype=np.int64)
 
 
-def unmask(conf, pred, tokens, mask_id, gen_start, block_len, n):
-    """Applies the unmask rule to every sequence in place; returns pos [B, n] padded with -1."""
+def unmask_capacity(n: int, block_len: int, tau: float) -> int:
+    """Most positions one sequence can reveal in a step."""
+    return max(n, block_len) if tau > 0 else n
+
+
+def unmask(conf, pred, tokens, mask_id, gen_start, block_len, n, tau: float = 0.0):
+    """Applies the unmask rule to every sequence in place; returns pos [B, cap] padded with -1."""
     B = tokens.shape[0]
-    pos = -np.ones((B, max(n, 0)), dtype=np.int64)
+    pos = -np.ones((B, max(unmask_capacity(n, block_len, tau), 0)), dtype=np.int64)
     for b in range(B):
-        p = unmask_positions(conf[b], tokens[b], mask_id, gen_start, block_len, n)
+        p = unmask_positions(conf[b], tokens[b], mask_id, gen_start, block_len, n, tau)
         tokens[b, p] = pred[b, p]
         pos[b, :len(p)] = p
     return pos
@@ -509,7 +541,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
         v = variation(h, st.h_ref, pol.kind)
         scores = importance(v, st.conf, masked, pol.alpha)
         kc = k_cap if k_cap is not None else (pol.k if pol.mode == SELECT_TOPK else N)
-        idx = select(scores, pol.mode, pol.k, pol.tau, kc)
+        idx = select(scores, pol.mode, pol.k, pol.tau, kc, pol.select_from)
     b_of = np.concatenate([np.full(len(a), b, dtype=np.int64) for b, a in enumerate(idx)])
     p_of = np.concatenate(idx) if len(idx) else np.zeros(0, dtype=np.int64)
     x = h[b_of, p_of]
@@ -528,13 +560,40 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
         apply_unmask(st.pred, st.tokens, pos)
     else:
         pos = unmask(st.conf, st.pred, st.tokens, cfg.mask_id, pol.gen_start,
-                     pol.block_len, pol.n_unmask)
+                     pol.block_len, pol.n_unmask, pol.unmask_tau)
     rows = []
     off = 0
     for a in idx:
         rows.append(x[off:off + len(a)].copy())
         off += len(a)
     return StepOut(idx, scores, pos, rows)
+
+
+def block_starts(cfg: ModelCfg, pol: Policy, tokens: np.ndarray) -> List[int]:
+    """Start of each sequence's current block (-1 once it has no masked position)."""
+    out = []
+    for b in range(tokens.shape[0]):
+        blk = current_block(tokens[b], cfg.mask_id, pol.gen_start, pol.block_len)
+        out.append(-1 if blk is None else blk[0])
+    return out
+
+
+def generate(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, n_steps: int):
+    """n_steps denoising steps with the periodic refresh of [ES-nl Methodologie 3]:
+    a step is dense at t = 0, at every multiple of refresh_every, and (with
+    refresh_on_block) when any sequence's current block differs from the one
+    it had at the previous step.  Returns (dense flags, revealed positions)."""
+    dense_log, pos_log = [], []
+    prev = None
+    for t in range(n_steps):
+        blocks = block_starts(cfg, pol, st.tokens)
+        dense = (t == 0 or (pol.refresh_every > 0 and t % pol.refresh_every == 0)
+                 or (pol.refresh_on_block and prev is not None and blocks != prev))
+        prev = blocks
+        out = step(cfg, W, st, pol, dense)
+        dense_log.append(bool(dense))
+        pos_log.append(out.unmasked)
+    return dense_log, pos_log
 
 
 def dense_forward(cfg: ModelCfg, W: ModelW, tokens: np.ndarray) -> np.ndarray:

@@ -1,0 +1,200 @@
+"""Pins of the oracle's step variants beyond the basic top-k step.
+
+* Over-threshold unmasking (fast phase of "Accelerating Diffusion Large
+  Language Models with SlowFast Sampling", German summary §2): brute force
+  over small blocks with tied confidences, and its two limits.
+* Response-only selection (DyLLM, French summary §2.C): brute force.
+* Periodic refresh (ES-dLLM, Dutch summary "Methodologie" item 3): a refresh
+  at every step is the vanilla generation written out independently; no
+  refresh is the plain loop of steps; block refreshes fall where the block
+  index floor(t * n / block_len) changes when every step reveals n tokens.
+"""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle as O
+from dllm_synth import TINY, with_, model_weights, prompt_tokens
+from _util import oracle_cfg, oracle_weights, oracle_policy, f64
+
+RT = 1e-10
+
+
+def _setup(shape=TINY, seed=0, **kw):
+    s = with_(shape, **kw)
+    cfg = oracle_cfg(s)
+    W = oracle_weights(model_weights(s, seed=seed))
+    tok = f64(prompt_tokens(s, seed=1)).astype(np.int64)
+    return s, cfg, W, tok
+
+
+# ----------------------------------------------------------------- unmask
+
+
+def _brute_unmask(conf, tokens, mask_id, gen_start, block_len, n, tau):
+    """Every masked position of the block above tau, or else the n best;
+    "best" found by checking every subset against every outsider."""
+    N = len(tokens)
+    first = next((p for p in range(gen_start, N) if tokens[p] == mask_id), None)
+    if first is None or n <= 0:
+        return []
+    start = gen_start + (first - gen_start) // block_len * block_len
+    cand = [p for p in range(start, min(start + block_len, N)) if tokens[p] == mask_id]
+    above = [p for p in cand if conf[p] > tau] if tau > 0 else []
+    if tau > 0 and len(above) >= n:
+        return sorted(above)
+
+    def better(p, q):  # p ranks before q
+        return conf[p] > conf[q] or (conf[p] == conf[q] and p < q)
+
+    m = min(n, len(cand))
+    for S in itertools.combinations(cand, m):
+        rest = [q for q in cand if q not in S]
+        if all(better(p, q) for p in S for q in rest):
+            return sorted(S)
+    raise AssertionError("no dominant subset")
+
+
+def test_unmask_tau_brute_force():
+    rng = np.random.default_rng(3)
+    levels = np.array([0.05, 0.3, 0.3, 0.6, 0.9, 0.9, 0.97])
+    mask_id = 99
+    for _ in range(400):
+        N = int(rng.integers(4, 13))
+        gen_start = int(rng.integers(0, 3))
+        block_len = int(rng.integers(1, 6))
+        n = int(rng.integers(0, 4))
+        tau = float(rng.choice([0.0, 0.3, 0.6, 0.95]))
+        tokens = np.where(rng.random(N) < 0.6, mask_id, 1).astype(np.int64)
+        conf = rng.choice(levels, N)
+        got = O.unmask_positions(conf, tokens, mask_id, gen_start, block_len, n, tau)
+        exp = _brute_unmask(conf, tokens, mask_id, gen_start, block_len, n, tau)
+        assert list(got) == exp, (conf, tokens, gen_start, block_len, n, tau)
+
+
+def test_unmask_tau_limits():
+    rng = np.random.default_rng(4)
+    mask_id = 7
+    for _ in range(50):
+        N, bl, n = 24, 8, 2
+        tokens = np.where(rng.random(N) < 0.7, mask_id, 0).astype(np.int64)
+        conf = rng.random(N)
+        plain = O.unmask_positions(conf, tokens, mask_id, 0, bl, n)
+        # a threshold no confidence reaches is the plain top-n rule
+        assert list(O.unmask_positions(conf, tokens, mask_id, 0, bl, n, 2.0)) == list(plain)
+        # a threshold every confidence passes reveals the whole current block
+        blk = O.current_block(tokens, mask_id, 0, bl)
+        if blk is None:
+            continue
+        whole = [p for p in range(*blk) if tokens[p] == mask_id]
+        got = O.unmask_positions(conf, tokens, mask_id, 0, bl, n, 1e-30)
+        assert list(got) == sorted(whole)
+    assert O.unmask_capacity(4, 32, 0.0) == 4 and O.unmask_capacity(4, 32, 0.9) == 32
+
+
+# ----------------------------------------------------------------- selection
+
+
+def test_select_from_brute_force():
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        N = int(rng.integers(1, 12))
+        lo = int(rng.integers(0, N + 1))
+        k = int(rng.integers(0, N + 2))
+        sc = rng.choice(np.array([0.0, -0.0, 0.25, 0.25, 0.5, 1.0, np.nan]), (1, N))
+        got = O.select(sc, O.SELECT_TOPK, k, 0.0, k, lo)[0]
+        pos = list(range(lo, N))
+
+        def key(p):
+            v = sc[0, p]
+            return (0, 0.0, -p) if np.isnan(v) else (1, float(v) + 0.0, -p)
+        m = min(k, len(pos))
+        exp = None
+        for S in itertools.combinations(pos, m):
+            rest = [q for q in pos if q not in S]
+            if all(key(p) > key(q) for p in S for q in rest):
+                exp = sorted(S)
+                break
+        assert list(got) == exp
+        if lo == 0:
+            assert list(got) == list(O.select(sc, O.SELECT_TOPK, k, 0.0, k)[0])
+
+
+def test_response_only_step_keeps_prompt_caches():
+    s, cfg, W, tok = _setup(n_layers=2)
+    st = O.empty_state(cfg, tok)
+    pol = oracle_policy(s, select_from=s.prompt_len, k=24)
+    O.step(cfg, W, st, pol, dense=True)
+    before = st.copy()
+    out = O.step(cfg, W, st, pol, dense=False)
+    assert all(len(a) == 24 and a.min() >= s.prompt_len for a in out.idx)
+    P = s.prompt_len
+    for l in range(cfg.n_layers):
+        np.testing.assert_array_equal(st.k[l][:, :P], before.k[l][:, :P])
+        np.testing.assert_array_equal(st.v[l][:, :P], before.v[l][:, :P])
+    np.testing.assert_array_equal(st.h_ref[:, :P], before.h_ref[:, :P])
+
+
+# ----------------------------------------------------------------- refresh
+
+
+def _vanilla_generation(cfg, W, tok, pol, n_steps):
+    """Every step a full forward of the current tokens; confidence and argmax of
+    every masked position; the unmask rule."""
+    tok = tok.copy()
+    conf = np.zeros(tok.shape)
+    pred = np.zeros(tok.shape, dtype=np.int64)
+    for _ in range(n_steps):
+        final = O.dense_forward(cfg, W, tok)
+        for b in range(tok.shape[0]):
+            m = np.nonzero(tok[b] == cfg.mask_id)[0]
+            if len(m) == 0:
+                continue
+            n = O.store(O.rms_norm(final[b, m], W.final_norm, cfg.rms_eps), cfg.dtype)
+            z = n @ np.asarray(W.lm_head).T
+            zmax = z.max(axis=1, keepdims=True)
+            conf[b, m] = 1.0 / np.exp(z - zmax).sum(axis=1)
+            pred[b, m] = np.argmax(z, axis=1)
+        O.unmask(conf, pred, tok, cfg.mask_id, pol.gen_start, pol.block_len, pol.n_unmask)
+    return tok, conf
+
+
+def test_refresh_every_step_is_the_vanilla_generation():
+    s, cfg, W, tok = _setup(n_layers=2)
+    pol = oracle_policy(s, refresh_every=1)
+    st = O.empty_state(cfg, tok)
+    dense_log, _ = O.generate(cfg, W, st, pol, 4)
+    assert dense_log == [True] * 4
+    tok_v, conf_v = _vanilla_generation(cfg, W, tok, pol, 4)
+    np.testing.assert_array_equal(st.tokens, tok_v)
+    m = conf_v > 0
+    np.testing.assert_allclose(st.conf[m], conf_v[m], rtol=RT)
+
+
+def test_no_refresh_is_the_plain_step_loop():
+    s, cfg, W, tok = _setup()
+    pol = oracle_policy(s)
+    st = O.empty_state(cfg, tok)
+    dense_log, pos_log = O.generate(cfg, W, st, pol, 5)
+    assert dense_log == [True, False, False, False, False]
+    st2 = O.empty_state(cfg, tok)
+    for t in range(5):
+        out = O.step(cfg, W, st2, pol, dense=(t == 0))
+        np.testing.assert_array_equal(out.unmasked, pos_log[t])
+    np.testing.assert_array_equal(st.tokens, st2.tokens)
+    for a, b in zip(st.k + st.v, st2.k + st2.v):
+        np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("block_len,n,R", [(16, 8, 0), (24, 8, 5), (64, 8, 3)])
+def test_block_refresh_schedule(block_len, n, R):
+    s, cfg, W, tok = _setup(block_len=block_len, n_unmask=n)
+    pol = oracle_policy(s, refresh_on_block=True, refresh_every=R)
+    st = O.empty_state(cfg, tok)
+    T = 8
+    dense_log, pos_log = O.generate(cfg, W, st, pol, T)
+    exp = [t == 0 or (R > 0 and t % R == 0) or (t * n // block_len != (t - 1) * n // block_len)
+           for t in range(T)]
+    assert dense_log == exp
+    assert all((p >= 0).sum() == n for p in pos_log)
