@@ -136,6 +136,13 @@ typedef struct {
   int n_unmask;      /* positions revealed per sequence and step        */
   int gen_start;     /* first generated position                        */
   int block_len;     /* generation block length                         */
+  /* Step variants (0 disables each):                                     */
+  int select_from;   /* partial steps never select positions below it:   */
+                     /* response-only steps [DyLLM 2.C] use gen_start    */
+  float unmask_tau;  /* > 0: also reveal every masked position of the    */
+                     /* block with conf > unmask_tau [SF-de 2, fast phase]*/
+  int refresh_every; /* dllm_generate: dense step every R steps [ES-nl 3] */
+  int refresh_on_block; /* dllm_generate: dense step when a block changes */
 } dllm_policy;
 
 /* Supported shapes for DLLM_BF16 layer work: d, n_heads*head_dim,
@@ -184,6 +191,17 @@ dllm_status dllm_select(const float* scores, int B, int N, int mode, int k, floa
                         dllm_stream_t stream);
 
 /*
+ * dllm_select_range - dllm_select over the positions lo .. N-1 only: the
+ * selection of a response-only step [DyLLM 2.C], whose prompt rows keep
+ * their cached K/V until a dense step brings the prompt in again.  TOPK
+ * takes min(k, N - lo) positions; 0 <= lo <= N.  Same outputs and errors
+ * as dllm_select; lo = 0 is dllm_select.
+ */
+dllm_status dllm_select_range(const float* scores, int B, int N, int lo, int mode, int k,
+                              float tau, int32_t* idx, int32_t* count, int k_cap, void* ws,
+                              size_t ws_bytes, dllm_stream_t stream);
+
+/*
  * dllm_unmask - reveal the most confident masked positions [SF-de 2].
  *
  * For each sequence: the current block is [s, min(s + block_len, N)) with
@@ -197,6 +215,25 @@ dllm_status dllm_select(const float* scores, int B, int N, int mode, int k, floa
 dllm_status dllm_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
                         int mask_id, int gen_start, int block_len, int n_unmask,
                         int32_t* pos_out, dllm_stream_t stream);
+
+/*
+ * dllm_unmask_tau - dllm_unmask with the over-threshold rule of the fast
+ * phase [SF-de 2]: with tau > 0, every masked position of the current block
+ * whose conf > tau (strict, fp32) is revealed, and when fewer than n_unmask
+ * are above tau the n_unmask most confident ones are (the top-n fallback) -
+ * together, the max(n_unmask, #above) most confident masked positions of the
+ * block, at most pos_cap.  tau <= 0 is dllm_unmask.  pos_out [B, pos_cap]
+ * (pos_cap >= n_unmask; block_len suffices for any tau), ascending, -1 padded.
+ * Bit-exact.  The pages fix no threshold value; the "stable region" of the
+ * fast phase is read as the current block.
+ */
+dllm_status dllm_unmask_tau(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
+                            int mask_id, int gen_start, int block_len, int n_unmask, float tau,
+                            int32_t* pos_out, int pos_cap, dllm_stream_t stream);
+
+/* Entries per sequence of pos_out / forced_unmask_pos under a policy:
+ * n_unmask, or max(n_unmask, block_len) when unmask_tau > 0. */
+int dllm_unmask_capacity(const dllm_policy* policy);
 
 /*
  * dllm_partial_layer - one transformer layer on the selected rows only
@@ -234,11 +271,14 @@ dllm_status dllm_partial_layer(const dllm_model_cfg* cfg, const dllm_layer_w* w,
  *  5. dllm_partial_layer for layers score_layer .. n_layers-1;
  *  6. for selected rows whose token is [MASK]: final RMSNorm, LM head,
  *     cache.conf <- max softmax, cache.pred <- argmax (logits never stored);
- *  7. dllm_unmask with policy.n_unmask / gen_start / block_len.
+ *  7. dllm_unmask_tau with policy.n_unmask / unmask_tau / gen_start / block_len.
+ * policy.select_from > 0 (response-only steps [DyLLM 2.C]): steps 2-3 only
+ * consider positions >= select_from; the scores of the others are -inf.
  * forced_idx [B, k_cap] + forced_count [B] replace steps 2-3 when non-NULL;
- * forced_unmask_pos [B, n_unmask] (-1 padded) replaces step 7's choice.
+ * forced_unmask_pos [B, cap] (-1 padded) replaces step 7's choice, with
+ * cap = dllm_unmask_capacity(policy).
  * Outputs (each may be NULL): idx_out [B, k_cap], count_out [B],
- * pos_out [B, n_unmask], scores_out [B, N].
+ * pos_out [B, cap], scores_out [B, N].
  * The workspace size covers both dense and partial steps of this shape.
  */
 size_t dllm_step_workspace_size(const dllm_model_cfg* cfg, int B, int N,
@@ -249,6 +289,30 @@ dllm_status dllm_step(const dllm_model_cfg* cfg, const dllm_model_w* w, const dl
                       const int32_t* forced_unmask_pos, int32_t* idx_out, int32_t* count_out,
                       int32_t* pos_out, float* scores_out, void* ws, size_t ws_bytes,
                       dllm_stream_t stream);
+
+/*
+ * dllm_generate - n_steps denoising steps with the periodic cache refresh of
+ * [ES-nl Methodologie 3]: step t is dense (every row recomputed, every cache
+ * rewritten) when t = 0, when policy.refresh_every > 0 divides t, or - with
+ * policy.refresh_on_block - when any sequence's current block (the block of
+ * its first masked position) differs from the one it had at step t-1; every
+ * other step is a partial step of dllm_step.  With refresh_every = 1 this is
+ * the vanilla (dense every step) generation; with select_from = gen_start
+ * and refresh_every = R it is DyLLM's response-only decoding with the prompt
+ * injected every R steps [DyLLM 2.C].
+ * pos_log: device [n_steps, B, dllm_unmask_capacity(policy)] int32 or NULL,
+ * the positions revealed at each step.  dense_log: HOST [n_steps] uint8 or
+ * NULL, 1 where the step was dense.  Steps are launched on `stream` from the
+ * host without synchronising, except that refresh_on_block reads the B block
+ * starts back once per step (one small device-to-host copy, which waits for
+ * the previous step).  ws: dllm_generate_workspace_size() bytes.
+ */
+size_t dllm_generate_workspace_size(const dllm_model_cfg* cfg, int B, int N,
+                                    const dllm_policy* policy);
+dllm_status dllm_generate(const dllm_model_cfg* cfg, const dllm_model_w* w,
+                          const dllm_cache* cache, int32_t* tokens, int B, int N,
+                          const dllm_policy* policy, int n_steps, int32_t* pos_log,
+                          uint8_t* dense_log, void* ws, size_t ws_bytes, dllm_stream_t stream);
 
 /*
  * dllm_attention_bf16 - the partial attention of one layer on its own

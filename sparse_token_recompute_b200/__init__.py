@@ -61,7 +61,9 @@ class CacheS(C.Structure):
 class Policy(C.Structure):
     _fields_ = [("score_layer", C.c_int), ("alpha", C.c_float), ("kind", C.c_int),
                 ("mode", C.c_int), ("k", C.c_int), ("tau", C.c_float), ("n_unmask", C.c_int),
-                ("gen_start", C.c_int), ("block_len", C.c_int)]
+                ("gen_start", C.c_int), ("block_len", C.c_int), ("select_from", C.c_int),
+                ("unmask_tau", C.c_float), ("refresh_every", C.c_int),
+                ("refresh_on_block", C.c_int)]
 
 
 def _sig(name, res, args):
@@ -79,6 +81,10 @@ _score = _sig("dllm_score", _i, [vp, vp, _i, _i, _i, _i, vp, vp, _i, _i, vp, vp,
 _select_ws = _sig("dllm_select_workspace_size", _sz, [_i, _i])
 _select = _sig("dllm_select", _i, [vp, _i, _i, _i, _i, _f, vp, vp, _i, vp, _sz, vp])
 _unmask = _sig("dllm_unmask", _i, [vp, vp, vp, _i, _i, _i, _i, _i, _i, vp, vp])
+_unmask_tau = _sig("dllm_unmask_tau", _i, [vp, vp, vp, _i, _i, _i, _i, _i, _i, _f, vp, _i, vp])
+_unmask_cap = _sig("dllm_unmask_capacity", _i, [C.POINTER(Policy)])
+_select_range = _sig("dllm_select_range", _i, [vp, _i, _i, _i, _i, _i, _f, vp, vp, _i, vp, _sz,
+                                               vp])
 _layer_ws = _sig("dllm_partial_layer_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i, _i])
 _layer = _sig("dllm_partial_layer", _i, [C.POINTER(ModelCfg), C.POINTER(LayerW), vp, _i, vp,
                                          vp, vp, _i, _i, _i, vp, vp, vp, _sz, vp])
@@ -87,6 +93,11 @@ _step_ws = _sig("dllm_step_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i,
 _step = _sig("dllm_step", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS), vp,
                                _i, _i, C.POINTER(Policy), _i, vp, vp, vp, vp, vp, vp, vp, vp,
                                _sz, vp])
+_gen_ws = _sig("dllm_generate_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i,
+                                                     C.POINTER(Policy)])
+_gen = _sig("dllm_generate", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS), vp,
+                                  _i, _i, C.POINTER(Policy), _i, vp, C.POINTER(C.c_uint8), vp,
+                                  _sz, vp])
 _devstat = _sig("dllm_get_device_status", _i, [vp, vp, C.POINTER(C.c_int32)])
 _attn_noalloc = _sig("dllm_attention_bf16_noalloc", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i,
                                                          _i, vp])
@@ -195,6 +206,16 @@ def dllm_select(scores, idx, count, mode: int, k: int, tau: float = 0.0, ws: Wor
     _check(st, "dllm_select")
 
 
+def dllm_select_range(scores, idx, count, lo: int, mode: int, k: int, tau: float = 0.0,
+                      ws: Workspace = None, stream=None):
+    B, N = scores.shape
+    k_cap = idx.shape[1]
+    st = _select_range(ptr(scores), B, N, int(lo), int(mode), int(k), float(tau), ptr(idx),
+                       ptr(count), k_cap, ws.ptr if ws else None, ws.nbytes if ws else 0,
+                       _stream(stream))
+    _check(st, "dllm_select_range")
+
+
 def dllm_select_workspace_size(B: int, N: int) -> int:
     return int(_select_ws(B, N))
 
@@ -205,6 +226,20 @@ def dllm_unmask(conf, pred, tokens, mask_id: int, gen_start: int, block_len: int
     st = _unmask(ptr(conf), ptr(pred), ptr(tokens), B, N, int(mask_id), int(gen_start),
                  int(block_len), int(n_unmask), ptr(pos_out), _stream(stream))
     _check(st, "dllm_unmask")
+
+
+def dllm_unmask_tau(conf, pred, tokens, mask_id: int, gen_start: int, block_len: int,
+                    n_unmask: int, tau: float, pos_out=None, stream=None):
+    B, N = tokens.shape
+    pos_cap = pos_out.shape[1] if pos_out is not None else max(n_unmask, block_len)
+    st = _unmask_tau(ptr(conf), ptr(pred), ptr(tokens), B, N, int(mask_id), int(gen_start),
+                     int(block_len), int(n_unmask), float(tau), ptr(pos_out), int(pos_cap),
+                     _stream(stream))
+    _check(st, "dllm_unmask_tau")
+
+
+def dllm_unmask_capacity(pol: "Policy") -> int:
+    return int(_unmask_cap(C.byref(pol)))
 
 
 def dllm_gemm_workspace_size(M, N, K, splits=0) -> int:
@@ -322,9 +357,11 @@ class Cache:
 
 
 def make_policy(score_layer=0, alpha=0.5, kind=DLLM_SCORE_COS, mode=DLLM_SELECT_TOPK, k=1,
-                tau=0.0, n_unmask=1, gen_start=0, block_len=32) -> Policy:
+                tau=0.0, n_unmask=1, gen_start=0, block_len=32, select_from=0, unmask_tau=0.0,
+                refresh_every=0, refresh_on_block=False) -> Policy:
     return Policy(score_layer, float(alpha), kind, mode, k, float(tau), n_unmask, gen_start,
-                  block_len)
+                  block_len, int(select_from), float(unmask_tau), int(refresh_every),
+                  int(bool(refresh_on_block)))
 
 
 def dllm_partial_layer_workspace_size(cfg: ModelCfg, B: int, N: int, k_cap: int) -> int:
@@ -354,6 +391,23 @@ def dllm_step(model: Model, cache: Cache, tokens, pol: Policy, dense: bool, ws: 
                ptr(forced_unmask_pos), ptr(idx_out), ptr(count_out), ptr(pos_out),
                ptr(scores_out), ws.ptr, ws.nbytes, _stream(stream))
     _check(st, "dllm_step")
+
+
+def dllm_generate_workspace_size(cfg: ModelCfg, B: int, N: int, pol: Policy) -> int:
+    return int(_gen_ws(C.byref(cfg), B, N, C.byref(pol)))
+
+
+def dllm_generate(model: Model, cache: Cache, tokens, pol: Policy, n_steps: int, ws: Workspace,
+                  pos_log=None, stream=None):
+    """n_steps steps with the policy's refresh schedule; returns the per-step
+    dense flags (host list of bool).  pos_log: device [n_steps, B, capacity]."""
+    B, N = tokens.shape
+    flags = (C.c_uint8 * max(int(n_steps), 1))()
+    st = _gen(C.byref(model.cfg), C.byref(model.s), C.byref(cache.s), ptr(tokens), B, N,
+              C.byref(pol), int(n_steps), ptr(pos_log), flags, ws.ptr, ws.nbytes,
+              _stream(stream))
+    _check(st, "dllm_generate")
+    return [bool(flags[t]) for t in range(int(n_steps))]
 
 
 def dllm_step_host(model: Model, cache: Cache, tokens_host, pol: Policy, dense: bool,

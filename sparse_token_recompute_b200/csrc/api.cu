@@ -147,6 +147,8 @@ struct Bump {
 
 constexpr size_t kHeader = 256;  // device status word lives at offset 0
 
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
 inline dllm_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DLLM_OK : DLLM_ERR_CUDA; }
 
 inline dllm_status check_launch() {
@@ -399,45 +401,68 @@ extern "C" dllm_status dllm_score(const void* h_cur, const void* h_ref, int B, i
   if (dtype == DLLM_BF16)
     launch_score<__nv_bfloat16>(static_cast<const __nv_bfloat16*>(h_cur), nullptr, nullptr,
                                 static_cast<const __nv_bfloat16*>(h_ref), B, N, d, conf, masked,
-                                nullptr, -1, alpha, kind, scores, 0, nullptr, s);
+                                nullptr, -1, alpha, kind, scores, 0, 0, nullptr, s);
   else
     launch_score<float>(static_cast<const float*>(h_cur), nullptr, nullptr,
                         static_cast<const float*>(h_ref), B, N, d, conf, masked, nullptr, -1,
-                        alpha, kind, scores, 0, nullptr, s);
+                        alpha, kind, scores, 0, 0, nullptr, s);
   return check_launch();
 }
 
 extern "C" size_t dllm_select_workspace_size(int, int) { return kHeader; }
 
-extern "C" dllm_status dllm_select(const float* scores, int B, int N, int mode, int k, float tau,
-                                   int32_t* idx, int32_t* count, int k_cap, void* ws,
-                                   size_t ws_bytes, dllm_stream_t stream) {
+extern "C" dllm_status dllm_select_range(const float* scores, int B, int N, int lo, int mode,
+                                         int k, float tau, int32_t* idx, int32_t* count,
+                                         int k_cap, void* ws, size_t ws_bytes,
+                                         dllm_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (B < 0 || N < 0 || k < 0 || k_cap < 1) return DLLM_ERR_INVALID_ARG;
+  if (B < 0 || N < 0 || k < 0 || k_cap < 1 || lo < 0 || lo > N) return DLLM_ERR_INVALID_ARG;
   if (mode != DLLM_SELECT_TOPK && mode != DLLM_SELECT_THRESH) return DLLM_ERR_INVALID_ARG;
-  if (mode == DLLM_SELECT_TOPK && std::min(k, N) > k_cap) return DLLM_ERR_CAPACITY;
+  if (mode == DLLM_SELECT_TOPK && std::min(k, N - lo) > k_cap) return DLLM_ERR_CAPACITY;
   if (N > 16384) return DLLM_ERR_UNSUPPORTED_SHAPE;
   if (B == 0) return DLLM_OK;
   if (!scores || !idx || !count) return DLLM_ERR_INVALID_ARG;
   if (ws && ws_bytes < kHeader) return DLLM_ERR_WORKSPACE;
   if (ws && !aligned(ws, 256)) return DLLM_ERR_WORKSPACE;
-  launch_select(scores, B, N, mode, k, tau, idx, count, k_cap, static_cast<int*>(ws), s);
+  launch_select(scores, B, N, lo, mode, k, tau, idx, count, k_cap, static_cast<int*>(ws), s);
+  return check_launch();
+}
+
+extern "C" dllm_status dllm_select(const float* scores, int B, int N, int mode, int k, float tau,
+                                   int32_t* idx, int32_t* count, int k_cap, void* ws,
+                                   size_t ws_bytes, dllm_stream_t stream) {
+  return dllm_select_range(scores, B, N, 0, mode, k, tau, idx, count, k_cap, ws, ws_bytes,
+                           stream);
+}
+
+extern "C" int dllm_unmask_capacity(const dllm_policy* pol) {
+  if (!pol) return 0;
+  const int n = std::max(pol->n_unmask, 0);
+  return pol->unmask_tau > 0.f ? std::max(n, pol->block_len) : n;
+}
+
+extern "C" dllm_status dllm_unmask_tau(const float* conf, const int32_t* pred, int32_t* tokens,
+                                       int B, int N, int mask_id, int gen_start, int block_len,
+                                       int n_unmask, float tau, int32_t* pos_out, int pos_cap,
+                                       dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B < 0 || N < 0 || n_unmask < 0 || gen_start < 0 || block_len < 1 || pos_cap < n_unmask)
+    return DLLM_ERR_INVALID_ARG;
+  if (!(tau == tau) || tau == INFINITY) return DLLM_ERR_INVALID_ARG;  // NaN / +inf
+  if (block_len > 1024 || N > 16384) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || N == 0) return DLLM_OK;
+  if (!conf || !pred || !tokens) return DLLM_ERR_INVALID_ARG;
+  if (gen_start > N) return DLLM_ERR_INVALID_ARG;
+  launch_unmask(conf, pred, tokens, B, N, mask_id, gen_start, block_len, n_unmask, tau, pos_cap,
+                pos_out, nullptr, s);
   return check_launch();
 }
 
 extern "C" dllm_status dllm_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B,
                                    int N, int mask_id, int gen_start, int block_len, int n_unmask,
                                    int32_t* pos_out, dllm_stream_t stream) {
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (B < 0 || N < 0 || n_unmask < 0 || gen_start < 0 || block_len < 1)
-    return DLLM_ERR_INVALID_ARG;
-  if (block_len > 1024 || N > 16384) return DLLM_ERR_UNSUPPORTED_SHAPE;
-  if (B == 0 || N == 0) return DLLM_OK;
-  if (!conf || !pred || !tokens) return DLLM_ERR_INVALID_ARG;
-  if (gen_start > N) return DLLM_ERR_INVALID_ARG;
-  launch_unmask(conf, pred, tokens, B, N, mask_id, gen_start, block_len, n_unmask, pos_out,
-                nullptr, s);
-  return check_launch();
+  return dllm_unmask_tau(conf, pred, tokens, B, N, mask_id, gen_start, block_len, n_unmask, 0.f,
+                         pos_out, std::max(n_unmask, 0), stream);
 }
 
 extern "C" dllm_status dllm_get_device_status(void* ws, dllm_stream_t stream, int32_t* out) {
@@ -675,6 +700,9 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
   if (pol->k < 0 || pol->n_unmask < 0 || pol->gen_start < 0 || pol->gen_start > N ||
       pol->block_len < 1)
     return DLLM_ERR_INVALID_ARG;
+  if (pol->select_from < 0 || pol->select_from > N || !(pol->unmask_tau == pol->unmask_tau) ||
+      pol->unmask_tau == INFINITY || pol->refresh_every < 0)
+    return DLLM_ERR_INVALID_ARG;
   if (N > 16384 || pol->block_len > 1024) return DLLM_ERR_UNSUPPORTED_SHAPE;
   if ((forced_idx == nullptr) != (forced_count == nullptr)) return DLLM_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < dllm_step_workspace_size(c, B, N, pol))
@@ -729,15 +757,16 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
                                     h_src ? nullptr : tokens,
                                     static_cast<const __nv_bfloat16*>(cache->h_ref), B, N, d,
                                     cache->conf, nullptr, tokens, c->mask_id, pol->alpha,
-                                    pol->kind, w.scores, c->vocab, w.status, s);
+                                    pol->kind, w.scores, c->vocab, pol->select_from, w.status,
+                                    s);
       else
         launch_score<float>(static_cast<const float*>(h_src),
                             static_cast<const float*>(mw->embed), h_src ? nullptr : tokens,
                             static_cast<const float*>(cache->h_ref), B, N, d, cache->conf,
                             nullptr, tokens, c->mask_id, pol->alpha, pol->kind, w.scores,
-                            c->vocab, w.status, s);
-      launch_select(w.scores, B, N, pol->mode, pol->k, pol->tau, w.idx, w.count, k_cap, w.status,
-                    s);
+                            c->vocab, pol->select_from, w.status, s);
+      launch_select(w.scores, B, N, pol->select_from, pol->mode, pol->k, pol->tau, w.idx, w.count,
+                    k_cap, w.status, s);
     }
     launch_row_map(w.idx, w.count, B, k_cap, N, L.row_off, L.row_pos, L.row_seq, w.status, s);
   }
@@ -799,7 +828,8 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
 
   // 7. unmask
   launch_unmask(cache->conf, cache->pred, tokens, B, N, c->mask_id, pol->gen_start,
-                pol->block_len, pol->n_unmask, pos_out, forced_unmask_pos, s);
+                pol->block_len, pol->n_unmask, pol->unmask_tau, dllm_unmask_capacity(pol), pos_out,
+                forced_unmask_pos, s);
 
   if (!dense) {
     if (idx_out || count_out) {
@@ -818,4 +848,50 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
       return DLLM_ERR_CUDA;
   }
   return check_launch();
+}
+
+// ---------------------------------------------------------------- generation
+
+extern "C" size_t dllm_generate_workspace_size(const dllm_model_cfg* c, int B, int N,
+                                               const dllm_policy* pol) {
+  const size_t step = dllm_step_workspace_size(c, B, N, pol);
+  if (step == 0) return 0;
+  return round_up(step, 256) + round_up((size_t)std::max(B, 1) * sizeof(int32_t), 256);
+}
+
+extern "C" dllm_status dllm_generate(const dllm_model_cfg* c, const dllm_model_w* mw,
+                                     const dllm_cache* cache, int32_t* tokens, int B, int N,
+                                     const dllm_policy* pol, int n_steps, int32_t* pos_log,
+                                     uint8_t* dense_log, void* ws, size_t ws_bytes,
+                                     dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!c || !pol || n_steps < 0 || B < 0 || N < 0) return DLLM_ERR_INVALID_ARG;
+  if (pol->refresh_every < 0) return DLLM_ERR_INVALID_ARG;
+  if (n_steps == 0 || B == 0 || N == 0) return DLLM_OK;
+  const size_t step_ws = dllm_step_workspace_size(c, B, N, pol);
+  if (step_ws == 0) return check_cfg(c) != DLLM_OK ? check_cfg(c) : DLLM_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dllm_generate_workspace_size(c, B, N, pol))
+    return DLLM_ERR_WORKSPACE;
+  int32_t* d_blocks = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + round_up(step_ws, 256));
+  const int cap = dllm_unmask_capacity(pol);
+  std::vector<int32_t> prev(B), cur(B);
+  for (int t = 0; t < n_steps; ++t) {
+    bool dense = t == 0 || (pol->refresh_every > 0 && t % pol->refresh_every == 0);
+    if (pol->refresh_on_block) {
+      launch_block_start(tokens, B, N, c->mask_id, pol->gen_start, pol->block_len, d_blocks, s);
+      if (cudaMemcpyAsync(cur.data(), d_blocks, (size_t)B * sizeof(int32_t),
+                          cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+          cudaStreamSynchronize(s) != cudaSuccess)
+        return DLLM_ERR_CUDA;
+      if (t > 0 && cur != prev) dense = true;
+      prev.swap(cur);
+    }
+    const dllm_status st =
+        dllm_step(c, mw, cache, tokens, B, N, pol, dense ? 1 : 0, nullptr, nullptr, nullptr,
+                  nullptr, nullptr, pos_log ? pos_log + (size_t)t * B * cap : nullptr, nullptr,
+                  ws, step_ws, stream);
+    if (st != DLLM_OK) return st;
+    if (dense_log) dense_log[t] = dense ? 1 : 0;
+  }
+  return DLLM_OK;
 }

@@ -136,12 +136,15 @@ template <typename T>
 void launch_score(const T* h_cur, const T* embed, const int32_t* tokens, const T* h_ref, int B,
                   int N, int d, const float* conf, const uint8_t* masked,
                   const int32_t* mask_tokens, int mask_id, float alpha, int kind, float* scores,
-                  int vocab, int* status, cudaStream_t s);
-void launch_select(const float* scores, int B, int N, int mode, int k, float tau, int32_t* idx,
-                   int32_t* count, int k_cap, int* status, cudaStream_t s);
+                  int vocab, int lo, int* status, cudaStream_t s);
+// positions < lo are never candidates
+void launch_select(const float* scores, int B, int N, int lo, int mode, int k, float tau,
+                   int32_t* idx, int32_t* count, int k_cap, int* status, cudaStream_t s);
 void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
-                   int mask_id, int gen_start, int block_len, int n_unmask, int32_t* pos_out,
-                   const int32_t* forced, cudaStream_t s);
+                   int mask_id, int gen_start, int block_len, int n_unmask, float tau,
+                   int pos_cap, int32_t* pos_out, const int32_t* forced, cudaStream_t s);
+void launch_block_start(const int32_t* tokens, int B, int N, int mask_id, int gen_start,
+                        int block_len, int32_t* out, cudaStream_t s);
 void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
                      int32_t* dst_count, int B, int k_cap, cudaStream_t s);
 

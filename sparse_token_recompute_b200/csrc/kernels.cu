@@ -112,10 +112,14 @@ __global__ void __launch_bounds__(256) score_kernel(const T* __restrict__ h_cur,
                                                     const int32_t* __restrict__ mask_tokens,
                                                     int mask_id, float alpha, int kind,
                                                     float* __restrict__ scores, int vocab,
-                                                    int* status) {
+                                                    int lo, int* status) {
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
+  if (row % N < lo) {  // never a candidate (response-only step): not scored
+    if (lane == 0) scores[row] = -INFINITY;
+    return;
+  }
   const T* hc;
   if (tokens) {
     int t = tokens[row];
@@ -360,8 +364,11 @@ __global__ void __launch_bounds__(128) lm_merge_kernel(const float* __restrict__
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_MAX_PER_THREAD = 16;  // N <= 16384
 
+// Candidates are the positions >= lo (all of them for top-k, those with a score
+// above tau for the threshold mode); a bit per element marks them.
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __restrict__ scores,
-                                                             int N, int mode, int k, float tau,
+                                                             int N, int lo, int mode, int k,
+                                                             float tau,
                                                              int32_t* __restrict__ idx,
                                                              int32_t* __restrict__ count,
                                                              int k_cap, int* status) {
@@ -373,17 +380,17 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
   const int E = (N + SEL_THREADS - 1) / SEL_THREADS;
   const int i0 = threadIdx.x * E;  // contiguous chunk keeps position order for the scans
   uint32_t key[SEL_MAX_PER_THREAD];
+  uint32_t candm = 0u;
   int n_cand = 0;
 #pragma unroll
   for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
     key[e] = 0u;
-    if (e < E && i0 + e < N) {
-      const float x = sc[i0 + e];
-      if (mode == DLLM_SELECT_TOPK) {
+    const int i = i0 + e;
+    if (e < E && i < N && i >= lo) {
+      const float x = sc[i];
+      if (mode == DLLM_SELECT_TOPK || x > tau) {  // NaN compares false
         key[e] = order_key(x);
-        ++n_cand;
-      } else if (x > tau) {  // NaN compares false
-        key[e] = order_key(x);
+        candm |= 1u << e;
         ++n_cand;
       }
     }
@@ -391,7 +398,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
   int total = block_sum_int(n_cand, red);
   int keff;
   if (mode == DLLM_SELECT_TOPK) {
-    keff = min(min(k, N), k_cap);
+    keff = min(min(k, total), k_cap);
   } else {
     keff = min(total, k_cap);
     if (total > k_cap && threadIdx.x == 0) raise_status(status, DEV_CAPACITY);
@@ -408,9 +415,8 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
-      if (e < E && i0 + e < N) {
-        const bool cand = (mode == DLLM_SELECT_TOPK) || key[e] != 0u;
-        if (cand && (key[e] & pmask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1);
+      if ((candm >> e) & 1u) {
+        if ((key[e] & pmask) == prefix) atomicAdd(&hist[(key[e] >> shift) & 255u], 1);
       }
     }
     __syncthreads();
@@ -457,10 +463,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
   int n_tie = 0;
 #pragma unroll
   for (int e = 0; e < SEL_MAX_PER_THREAD; ++e)
-    if (e < E && i0 + e < N) {
-      const bool cand = (mode == DLLM_SELECT_TOPK) || key[e] != 0u;
-      n_tie += (cand && key[e] == T) ? 1 : 0;
-    }
+    n_tie += (((candm >> e) & 1u) && key[e] == T) ? 1 : 0;
   const int tie_incl = block_inclusive_scan(n_tie, red);
   int tie_rank = tie_incl - n_tie;
   bool sel[SEL_MAX_PER_THREAD];
@@ -468,11 +471,10 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
 #pragma unroll
   for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
     sel[e] = false;
-    if (e < E && i0 + e < N) {
-      const bool cand = (mode == DLLM_SELECT_TOPK) || key[e] != 0u;
-      if (cand && key[e] > T) {
+    if ((candm >> e) & 1u) {
+      if (key[e] > T) {
         sel[e] = true;
-      } else if (cand && key[e] == T) {
+      } else if (key[e] == T) {
         sel[e] = tie_rank < remaining;
         ++tie_rank;
       }
@@ -490,11 +492,15 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
 
 // ---------------------------------------------------------------- unmask
 
+// The n_unmask most confident masked positions of the current block; with
+// tau > 0, all masked positions with conf > tau when that is more (the top
+// max(n_unmask, #above) positions).  pos_out / forced rows hold pos_cap entries.
 __global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ conf,
                                                       const int32_t* __restrict__ pred,
                                                       int32_t* __restrict__ tokens, int N,
                                                       int mask_id, int gen_start, int block_len,
-                                                      int n_unmask, int32_t* __restrict__ pos_out,
+                                                      int n_unmask, float tau, int pos_cap,
+                                                      int32_t* __restrict__ pos_out,
                                                       const int32_t* __restrict__ forced) {
   __shared__ int red[33];
   __shared__ uint32_t skey[1024];
@@ -503,10 +509,10 @@ __global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ 
   int32_t* tk = tokens + (size_t)b * N;
   const float* cf = conf + (size_t)b * N;
   const int32_t* pr = pred + (size_t)b * N;
-  int32_t* po = pos_out ? pos_out + (size_t)b * n_unmask : nullptr;
+  int32_t* po = pos_out ? pos_out + (size_t)b * pos_cap : nullptr;
   if (forced) {
-    for (int j = threadIdx.x; j < n_unmask; j += blockDim.x) {
-      const int p = forced[(size_t)b * n_unmask + j];
+    for (int j = threadIdx.x; j < pos_cap; j += blockDim.x) {
+      const int p = forced[(size_t)b * pos_cap + j];
       if (p >= 0 && p < N) tk[p] = pr[p];
       if (po) po[j] = (p >= 0 && p < N) ? p : -1;
     }
@@ -518,7 +524,7 @@ __global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ 
   first = block_min_int(first, red);
   if (first >= N || n_unmask <= 0) {
     if (po)
-      for (int j = threadIdx.x; j < n_unmask; j += blockDim.x) po[j] = -1;
+      for (int j = threadIdx.x; j < pos_cap; j += blockDim.x) po[j] = -1;
     return;
   }
   const int blk = gen_start + ((first - gen_start) / block_len) * block_len;
@@ -533,6 +539,12 @@ __global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ 
     smask[t] = is_m ? 1 : 0;
   }
   __syncthreads();
+  int take = n_unmask;
+  if (tau > 0.f) {
+    const bool above = t < L && is_m && cf[blk + t] > tau;  // NaN compares false
+    take = max(take, block_sum_int(above ? 1 : 0, red));
+  }
+  take = min(take, pos_cap);
   bool sel = false;
   if (t < L && is_m) {
     int rank = 0;
@@ -541,7 +553,7 @@ __global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ 
       const uint32_t kj = skey[j];
       rank += (kj > mykey || (kj == mykey && j < t)) ? 1 : 0;
     }
-    sel = rank < n_unmask;
+    sel = rank < take;
   }
   const int incl = block_inclusive_scan(sel ? 1 : 0, red);
   __shared__ int s_total;
@@ -553,7 +565,24 @@ __global__ void __launch_bounds__(1024) unmask_kernel(const float* __restrict__ 
     if (po) po[incl - 1] = p;
   }
   if (po)
-    for (int j = s_total + threadIdx.x; j < n_unmask; j += blockDim.x) po[j] = -1;
+    for (int j = s_total + threadIdx.x; j < pos_cap; j += blockDim.x) po[j] = -1;
+}
+
+// start of each sequence's current block: the block holding the first masked
+// position >= gen_start (-1 when none is left)
+__global__ void __launch_bounds__(256) block_start_kernel(const int32_t* __restrict__ tokens,
+                                                          int N, int mask_id, int gen_start,
+                                                          int block_len,
+                                                          int32_t* __restrict__ out) {
+  __shared__ int red[33];
+  const int b = blockIdx.x;
+  const int32_t* tk = tokens + (size_t)b * N;
+  int first = N;
+  for (int p = gen_start + threadIdx.x; p < N; p += blockDim.x)
+    if (tk[p] == mask_id) first = min(first, p);
+  first = block_min_int(first, red);
+  if (threadIdx.x == 0)
+    out[b] = first >= N ? -1 : gen_start + ((first - gen_start) / block_len) * block_len;
 }
 
 // ---------------------------------------------------------------- row bookkeeping
@@ -963,21 +992,21 @@ template <typename T>
 void launch_score(const T* h_cur, const T* embed, const int32_t* tokens, const T* h_ref, int B,
                   int N, int d, const float* conf, const uint8_t* masked,
                   const int32_t* mask_tokens, int mask_id, float alpha, int kind, float* scores,
-                  int vocab, int* status, cudaStream_t s) {
+                  int vocab, int lo, int* status, cudaStream_t s) {
   const int rows = B * N;
   if (rows <= 0) return;
   ProfScope prof("score", s);
   score_kernel<T><<<(rows + 7) / 8, 256, 0, s>>>(h_cur, embed, tokens, h_ref, rows, N, d, conf,
                                                  masked, mask_tokens, mask_id, alpha, kind,
-                                                 scores, vocab, status);
+                                                 scores, vocab, lo, status);
 }
 template void launch_score<float>(const float*, const float*, const int32_t*, const float*, int,
                                   int, int, const float*, const uint8_t*, const int32_t*, int,
-                                  float, int, float*, int, int*, cudaStream_t);
+                                  float, int, float*, int, int, int*, cudaStream_t);
 template void launch_score<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
                                           const int32_t*, const __nv_bfloat16*, int, int, int,
                                           const float*, const uint8_t*, const int32_t*, int, float,
-                                          int, float*, int, int*, cudaStream_t);
+                                          int, float*, int, int, int*, cudaStream_t);
 
 template <typename T>
 void launch_confidence(const T* logits, const int32_t* logit_pos, int B, int Mm, int V, int N,
@@ -991,20 +1020,27 @@ template void launch_confidence<float>(const float*, const int32_t*, int, int, i
 template void launch_confidence<__nv_bfloat16>(const __nv_bfloat16*, const int32_t*, int, int, int,
                                                int, float*, int32_t*, cudaStream_t);
 
-void launch_select(const float* scores, int B, int N, int mode, int k, float tau, int32_t* idx,
-                   int32_t* count, int k_cap, int* status, cudaStream_t s) {
+void launch_select(const float* scores, int B, int N, int lo, int mode, int k, float tau,
+                   int32_t* idx, int32_t* count, int k_cap, int* status, cudaStream_t s) {
   if (B <= 0) return;
   ProfScope prof("select", s);
-  select_kernel<<<B, SEL_THREADS, 0, s>>>(scores, N, mode, k, tau, idx, count, k_cap, status);
+  select_kernel<<<B, SEL_THREADS, 0, s>>>(scores, N, lo, mode, k, tau, idx, count, k_cap, status);
 }
 
 void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
-                   int mask_id, int gen_start, int block_len, int n_unmask, int32_t* pos_out,
-                   const int32_t* forced, cudaStream_t s) {
+                   int mask_id, int gen_start, int block_len, int n_unmask, float tau,
+                   int pos_cap, int32_t* pos_out, const int32_t* forced, cudaStream_t s) {
   if (B <= 0) return;
   ProfScope prof("unmask", s);
   unmask_kernel<<<B, 1024, 0, s>>>(conf, pred, tokens, N, mask_id, gen_start, block_len, n_unmask,
-                                   pos_out, forced);
+                                   tau, pos_cap, pos_out, forced);
+}
+
+void launch_block_start(const int32_t* tokens, int B, int N, int mask_id, int gen_start,
+                        int block_len, int32_t* out, cudaStream_t s) {
+  if (B <= 0) return;
+  ProfScope prof("block_start", s);
+  block_start_kernel<<<B, 256, 0, s>>>(tokens, N, mask_id, gen_start, block_len, out);
 }
 
 void launch_row_map(const int32_t* idx, const int32_t* count, int B, int k_cap, int N,

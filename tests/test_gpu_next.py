@@ -1,0 +1,144 @@
+"""GPU parity of the step variants: over-threshold unmasking ("Accelerating
+Diffusion Large Language Models with SlowFast Sampling", German summary §2),
+response-only selection (DyLLM, French summary §2.C) and the periodic
+refresh of a generation (ES-dLLM, Dutch summary "Methodologie" item 3).
+Index work is compared bit-exactly on identical inputs; whole steps and
+generations against the oracle as in the step tests."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import dllm_synth as SY
+from _util import f64, max_abs_rel, TOL
+from test_gpu_step import Run, _small_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("tau", [0.0, 0.55, 0.97, 1e-30])
+def test_unmask_tau_matches_oracle(lib, tau):
+    g = torch.Generator().manual_seed(11)
+    B, N, gen_start, bl, n, mask_id = 3, 200, 40, 32, 4, 999
+    tokens = torch.randint(0, 900, (B, N), generator=g, dtype=torch.int32)
+    tokens[:, gen_start:] = torch.where(torch.rand(B, N - gen_start, generator=g) < 0.8,
+                                        torch.tensor(mask_id, dtype=torch.int32),
+                                        tokens[:, gen_start:])
+    tokens[1, gen_start:gen_start + 40] = 5          # sequence 1's first block is done
+    conf = torch.round(torch.rand(B, N, generator=g) * 20) / 20   # ties
+    pred = torch.randint(0, 900, (B, N), generator=g, dtype=torch.int32)
+    pos = torch.full((B, bl), -7, dtype=torch.int32)
+    t_gpu = tokens.cuda()
+    p_gpu = pos.cuda()
+    lib.dllm_unmask_tau(conf.cuda(), pred.cuda(), t_gpu, mask_id, gen_start, bl, n, tau, p_gpu)
+    torch.cuda.synchronize()
+    t_ora = f64(tokens).astype(np.int64)
+    tau32 = float(np.float32(tau))   # the threshold the library compares in fp32
+    p_ora = O.unmask(f64(conf), f64(pred).astype(np.int64), t_ora, mask_id, gen_start, bl, n,
+                     tau32)
+    cap = O.unmask_capacity(n, bl, tau)
+    got = p_gpu.cpu().numpy()
+    np.testing.assert_array_equal(got[:, :cap], p_ora)
+    assert np.all(got[:, cap:] == -1)
+    np.testing.assert_array_equal(t_gpu.cpu().numpy(), t_ora)
+
+
+@pytest.mark.parametrize("lo,k", [(0, 50), (37, 50), (190, 50), (200, 5)])
+def test_select_range_matches_oracle(lib, lo, k):
+    g = torch.Generator().manual_seed(12)
+    B, N = 4, 200
+    sc = torch.round(torch.randn(B, N, generator=g) * 4) / 4
+    sc[0, ::7] = float("nan")
+    sc[1, ::5] = -0.0
+    idx = torch.full((B, 64), -3, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+    lib.dllm_select_range(sc.cuda(), idx, cnt, lo, lib.DLLM_SELECT_TOPK, k)
+    torch.cuda.synchronize()
+    ora = O.select(f64(sc), O.SELECT_TOPK, k, 0.0, 64, lo)
+    for b in range(B):
+        c = int(cnt[b])
+        assert c == len(ora[b])
+        np.testing.assert_array_equal(idx[b, :c].cpu().numpy(), ora[b])
+
+
+def test_response_only_steps_tiny(lib):
+    r = Run(lib, SY.TINY, select_from=SY.TINY.prompt_len)
+    P = SY.TINY.prompt_len
+    r.gpu_step(True)
+    kv0 = [t[:, :P].clone() for t in r.cache.k + r.cache.v]
+    for t in range(1, 5):
+        tok_before = f64(r.tokens).astype(np.int64)
+        href_before = f64(r.cache.h_ref)
+        conf_before = f64(r.cache.conf)
+        idx, cnt, pos, sc = r.gpu_step(False)
+        masked = tok_before == r.ocfg.mask_id
+        h = r.ow.embed[tok_before]
+        ora = O.importance(O.variation(h, href_before, r.opol.kind), conf_before, masked,
+                           r.opol.alpha)
+        assert max_abs_rel(sc[:, P:], ora[:, P:]) < TOL["f32"]
+        assert np.all(np.isneginf(sc[:, :P]))
+        sel = O.select(sc, O.SELECT_TOPK, r.opol.k, 0.0, r.k_cap, P)
+        for b in range(r.B):
+            np.testing.assert_array_equal(idx[b, :cnt[b]], sel[b])
+            assert idx[b, :cnt[b]].min() >= P
+    for a, b in zip(kv0, [t[:, :P] for t in r.cache.k + r.cache.v]):
+        assert torch.equal(a, b)
+
+
+def test_threshold_unmask_inside_a_step(lib):
+    shape = _small_bf16()
+    r = Run(lib, shape)
+    r.gpu_step(True)
+    conf = f64(r.cache.conf)
+    tok = f64(r.tokens).astype(np.int64)
+    blk = O.current_block(tok[0], r.ocfg.mask_id, r.opol.gen_start, r.opol.block_len)
+    m = [p for p in range(*blk) if tok[0, p] == r.ocfg.mask_id]
+    tau = float(np.float32(np.quantile(conf[0, m], 0.3)))
+    r.pol.unmask_tau = tau
+    for t in range(2):
+        tok_before = f64(r.tokens).astype(np.int64)
+        idx, cnt, pos, sc = r.gpu_step(False)
+        t_ora = tok_before.copy()
+        p_ora = O.unmask(f64(r.cache.conf), f64(r.cache.pred).astype(np.int64), t_ora,
+                         r.ocfg.mask_id, r.opol.gen_start, r.opol.block_len, r.opol.n_unmask,
+                         tau)
+        np.testing.assert_array_equal(pos, p_ora)
+        np.testing.assert_array_equal(f64(r.tokens).astype(np.int64), t_ora)
+        if t == 0:
+            assert (p_ora[0] >= 0).sum() > r.opol.n_unmask   # the threshold did reveal more
+
+
+def test_generate_tiny_matches_oracle(lib):
+    shape = SY.with_(SY.TINY, block_len=16)
+    r = Run(lib, shape, refresh_every=3, refresh_on_block=True)
+    T = 8
+    cap = lib.dllm_unmask_capacity(r.pol)
+    pos_log = torch.full((T, r.B, cap), -9, dtype=torch.int32, device="cuda")
+    ws = lib.Workspace(lib.dllm_generate_workspace_size(r.model.cfg, r.B, r.N, r.pol))
+    dense = lib.dllm_generate(r.model, r.cache, r.tokens, r.pol, T, ws, pos_log=pos_log)
+    torch.cuda.synchronize()
+    assert ws.device_status() == 0
+    d_ora, p_ora = O.generate(r.ocfg, r.ow, r.st, r.opol, T)
+    assert dense == d_ora
+    assert dense == [True, False, True, True, True, False, True, False]
+    for t in range(T):
+        np.testing.assert_array_equal(pos_log[t].cpu().numpy(), p_ora[t])
+    np.testing.assert_array_equal(f64(r.tokens).astype(np.int64), r.st.tokens)
+    r.compare_state(TOL["f32"])
+
+
+def test_generate_equals_step_loop_bf16(lib):
+    shape = _small_bf16()
+    kw = dict(select_from=shape.prompt_len, refresh_every=2)
+    r1, r2 = Run(lib, shape, **kw), Run(lib, shape, **kw)
+    T = 5
+    ws = lib.Workspace(lib.dllm_generate_workspace_size(r1.model.cfg, r1.B, r1.N, r1.pol))
+    dense = lib.dllm_generate(r1.model, r1.cache, r1.tokens, r1.pol, T, ws)
+    assert dense == [True, False, True, False, True]
+    for t in range(T):
+        r2.gpu_step(dense[t])
+    torch.cuda.synchronize()
+    assert torch.equal(r1.tokens, r2.tokens)
+    for a, b in zip(r1.cache.k + r1.cache.v + [r1.cache.h_ref, r1.cache.conf, r1.cache.pred],
+                    r2.cache.k + r2.cache.v + [r2.cache.h_ref, r2.cache.conf, r2.cache.pred]):
+        assert torch.equal(a, b)

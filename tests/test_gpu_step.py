@@ -34,14 +34,18 @@ class Run:
         self.pol = lib.make_policy(score_layer=self.opol.score_layer, alpha=self.opol.alpha,
                                    kind=self.opol.kind, mode=self.opol.mode, k=self.opol.k,
                                    tau=self.opol.tau, n_unmask=self.opol.n_unmask,
-                                   gen_start=self.opol.gen_start, block_len=self.opol.block_len)
+                                   gen_start=self.opol.gen_start, block_len=self.opol.block_len,
+                                   select_from=self.opol.select_from,
+                                   unmask_tau=self.opol.unmask_tau,
+                                   refresh_every=self.opol.refresh_every,
+                                   refresh_on_block=self.opol.refresh_on_block)
         self.k_cap = max(1, min(self.opol.k, N))
         self.ws = lib.Workspace(lib.dllm_step_workspace_size(self.model.cfg, B, N, self.pol))
         self.st = O.empty_state(self.ocfg, f64(tok).astype(np.int64))
         self.B, self.N = B, N
 
     def gpu_step(self, dense, forced_idx=None, forced_unmask=None):
-        B, N, n = self.B, self.N, max(self.opol.n_unmask, 1)
+        B, N, n = self.B, self.N, max(self.lib.dllm_unmask_capacity(self.pol), 1)
         idx = torch.full((B, self.k_cap), -1, dtype=torch.int32, device="cuda")
         cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
         pos = torch.full((B, n), -5, dtype=torch.int32, device="cuda")
