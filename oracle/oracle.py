@@ -63,6 +63,14 @@ in the design notes):
   * Response-only steps [DyLLM §2.C]: rows before select_from (the prompt)
     are never selected in a partial step; their K/V stay as cached until a
     dense step injects the prompt again.
+  * Two skip points [ES-de §2.B "Strategie": layers 1/8 and 1/4]: with a
+    second score layer l2 > l_s, the rows selected at l_s run layers
+    l_s..l2-1; at l2 every one of them is scored again, on its input of
+    layer l2 against a second reference cache h_ref2 (its value at its last
+    pass through l2), with the same importance formula, and each sequence
+    keeps the top-k2 of its rows for layers l2..L-1 and the LM head.  Rows
+    dropped at l2 keep their fresh K/V below l2 and their cached K/V from l2
+    on.  A dense step writes h_ref2 for every row.
   * Periodic refresh [ES-nl Methodologie 3]: in a generation, a step is
     dense (every row recomputed, every cache rewritten) at step 0, every
     refresh_every steps, and, with refresh_on_block, at the first step at
@@ -190,6 +198,8 @@ class Policy:
     n_unmask: int = 1
     gen_start: int = 0
     block_len: int = 32
+    score_layer2: int = 0         # > score_layer: second skip point (0: none)
+    k2: int = 0                   # rows per sequence kept at the second skip point
     select_from: int = 0          # positions below it are never selected (partial steps)
     unmask_tau: float = 0.0       # > 0: over-threshold unmasking with top-n fallback
     refresh_every: int = 0        # generation: dense step every R steps (0: never)
@@ -205,11 +215,13 @@ class State:
     h_ref: np.ndarray                   # [B, N, d] hidden at the score layer, last recompute
     conf: np.ndarray                    # [B, N] cached confidence
     pred: np.ndarray                    # [B, N] cached argmax token
+    h_ref2: Optional[np.ndarray] = None  # [B, N, d] hidden at the second skip point
 
     def copy(self) -> "State":
         return State(self.tokens.copy(), [a.copy() for a in self.k],
                      [a.copy() for a in self.v], self.h_ref.copy(),
-                     self.conf.copy(), self.pred.copy())
+                     self.conf.copy(), self.pred.copy(),
+                     None if self.h_ref2 is None else self.h_ref2.copy())
 
 
 def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
@@ -219,7 +231,7 @@ def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
                  [np.zeros(kv) for _ in range(cfg.n_layers)],
                  [np.zeros(kv) for _ in range(cfg.n_layers)],
                  np.zeros((B, N, cfg.d)), np.zeros((B, N)),
-                 np.zeros((B, N), dtype=np.int64))
+                 np.zeros((B, N), dtype=np.int64), np.zeros((B, N, cfg.d)))
 
 
 # ---------------------------------------------------------------------------
@@ -497,6 +509,8 @@ class StepOut:
     scores: Optional[np.ndarray]   # [B, N] or None for a dense step
     unmasked: np.ndarray           # [B, n] padded with -1
     final_rows: List[np.ndarray] = field(default_factory=list)  # per sequence [k_b, d]
+    idx2: Optional[List[np.ndarray]] = None   # rows kept at the second skip point
+    scores2: Optional[List[np.ndarray]] = None  # their scores, per sequence in idx order
 
 
 def embed(W: ModelW, tokens: np.ndarray) -> np.ndarray:
@@ -514,8 +528,31 @@ def dense_layers(cfg: ModelCfg, W: ModelW, st: State, h: np.ndarray, upto: int) 
     return x.reshape(B, N, d)
 
 
+def narrow(st: State, pol: Policy, masked: np.ndarray, x: np.ndarray, b_of: np.ndarray,
+           p_of: np.ndarray, forced_idx2=None):
+    """The second skip point: score the compact rows on their input of layer
+    score_layer2 against h_ref2, keep each sequence's top-k2 (ES-de §2.A, §2.B).
+    Returns (kept positions per sequence, their scores per sequence, keep mask)."""
+    B = st.tokens.shape[0]
+    I2 = importance(variation(x, st.h_ref2[b_of, p_of], pol.kind), st.conf[b_of, p_of],
+                    masked[b_of, p_of], pol.alpha)
+    idx2, sc2 = [], []
+    for b in range(B):
+        rows = np.nonzero(b_of == b)[0]          # ascending positions
+        sc2.append(I2[rows])
+        if forced_idx2 is not None:
+            idx2.append(np.asarray(forced_idx2[b], dtype=np.int64))
+        else:
+            idx2.append(p_of[rows][select_topk(I2[rows], pol.k2)])
+    keep = np.zeros(len(b_of), dtype=bool)
+    for b in range(B):
+        keep |= (b_of == b) & np.isin(p_of, idx2[b])
+    return idx2, sc2, keep
+
+
 def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
-         forced_idx=None, forced_unmask=None, k_cap: Optional[int] = None) -> StepOut:
+         forced_idx=None, forced_unmask=None, k_cap: Optional[int] = None,
+         forced_idx2=None) -> StepOut:
     """One denoising step, in place on ``st``.
 
     1. embed the tokens; run layers below the score layer on every row;
@@ -546,7 +583,14 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
     p_of = np.concatenate(idx) if len(idx) else np.zeros(0, dtype=np.int64)
     x = h[b_of, p_of]
     st.h_ref[b_of, p_of] = x
+    l2 = pol.score_layer2 if pol.score_layer2 > ls else -1
+    idx2 = sc2 = None
     for l in range(ls, cfg.n_layers):
+        if l == l2:
+            if not dense:
+                idx2, sc2, keep = narrow(st, pol, masked, x, b_of, p_of, forced_idx2)
+                b_of, p_of, x = b_of[keep], p_of[keep], x[keep]
+            st.h_ref2[b_of, p_of] = x
         if len(b_of):
             x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l])
     sel_masked = masked[b_of, p_of]
@@ -563,10 +607,10 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
                      pol.block_len, pol.n_unmask, pol.unmask_tau)
     rows = []
     off = 0
-    for a in idx:
+    for a in (idx2 if idx2 is not None else idx):
         rows.append(x[off:off + len(a)].copy())
         off += len(a)
-    return StepOut(idx, scores, pos, rows)
+    return StepOut(idx, scores, pos, rows, idx2, sc2)
 
 
 def block_starts(cfg: ModelCfg, pol: Policy, tokens: np.ndarray) -> List[int]:

@@ -8,6 +8,11 @@
   at every step is the vanilla generation written out independently; no
   refresh is the plain loop of steps; block refreshes fall where the block
   index floor(t * n / block_len) changes when every step reveals n tokens.
+* Two skip points (ES-dLLM, German summary §2.B "Strategie"): keeping every
+  row at the second point is the one-point step; keeping none leaves the
+  layers from the second point on untouched; after a dense step a two-point
+  step is a fixed point; the rows kept at the second point dominate the
+  dropped ones by brute force.
 """
 import itertools
 
@@ -198,3 +203,80 @@ def test_block_refresh_schedule(block_len, n, R):
            for t in range(T)]
     assert dense_log == exp
     assert all((p >= 0).sum() == n for p in pos_log)
+
+
+# ----------------------------------------------------------------- two skip points
+
+
+def _two_point_setup(k2, **kw):
+    s, cfg, W, tok = _setup(n_layers=3, **kw)
+    st = O.empty_state(cfg, tok)
+    pol = oracle_policy(s, score_layer2=2, k2=k2)
+    O.step(cfg, W, st, pol, dense=True)
+    # change some generated tokens so the next step has real work
+    rng = np.random.default_rng(9)
+    P = s.prompt_len
+    ch = rng.choice(np.arange(P, s.seq_len), 12, replace=False)
+    st.tokens[0, ch] = rng.integers(0, cfg.vocab - 1, len(ch))
+    return s, cfg, W, st, pol
+
+
+def test_two_point_keeping_every_row_equals_one_point():
+    s, cfg, W, st, pol = _two_point_setup(k2=10 ** 6)
+    st1 = st.copy()
+    out2 = O.step(cfg, W, st, pol, dense=False)
+    pol1 = oracle_policy(s)
+    out1 = O.step(cfg, W, st1, pol1, dense=False)
+    for a, b in zip(out2.idx2, out1.idx):
+        np.testing.assert_array_equal(a, b)
+    for a, b in zip(st.k + st.v, st1.k + st1.v):
+        np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(st.tokens, st1.tokens)
+    np.testing.assert_array_equal(st.conf, st1.conf)
+
+
+def test_two_point_keeping_no_row_leaves_upper_layers():
+    s, cfg, W, st, pol = _two_point_setup(k2=0)
+    before = st.copy()
+    out = O.step(cfg, W, st, pol, dense=False)
+    assert all(len(a) == 0 for a in out.idx2)
+    for l in range(2, cfg.n_layers):
+        np.testing.assert_array_equal(st.k[l], before.k[l])
+        np.testing.assert_array_equal(st.v[l], before.v[l])
+    np.testing.assert_array_equal(st.conf, before.conf)
+    np.testing.assert_array_equal(st.h_ref2, before.h_ref2)
+    # the rows selected at the first point did run the layers below the second
+    changed = [l for l in range(2) if not np.array_equal(st.k[l], before.k[l])]
+    assert changed == [0, 1]
+
+
+def test_two_point_fixed_point_after_dense():
+    s, cfg, W, tok = _setup(n_layers=3)
+    st = O.empty_state(cfg, tok)
+    pol = oracle_policy(s, score_layer2=2, k2=9, n_unmask=0)
+    O.step(cfg, W, st, pol, dense=True)
+    ref = st.copy()
+    O.step(cfg, W, st, pol, dense=False)
+    for a, b in zip(st.k + st.v, ref.k + ref.v):
+        np.testing.assert_allclose(a, b, rtol=RT, atol=RT)
+    np.testing.assert_allclose(st.h_ref2, ref.h_ref2, rtol=RT, atol=RT)
+
+
+def test_two_point_selection_brute_force():
+    s, cfg, W, st, pol = _two_point_setup(k2=7)
+    out = O.step(cfg, W, st.copy(), pol, dense=False)
+    for b in range(len(out.idx)):
+        pos, sc = out.idx[b], out.scores2[b]
+        best = sorted(range(len(pos)), key=lambda j: _key(sc[j], pos[j]), reverse=True)[:7]
+        # brute force: every kept row ranks above every dropped row
+        kept = set(int(p) for p in out.idx2[b])
+        for j in range(len(pos)):
+            for i in range(len(pos)):
+                if int(pos[i]) in kept and int(pos[j]) not in kept:
+                    assert _key(sc[i], pos[i]) > _key(sc[j], pos[j])
+        assert kept == set(int(pos[j]) for j in best)
+
+
+def _key(v, p):
+    v = float(v)
+    return (0, 0.0, -int(p)) if np.isnan(v) else (1, v + 0.0, -int(p))
