@@ -124,6 +124,8 @@ typedef struct {
   void* h_ref;
   float* conf;
   int32_t* pred;
+  void* h_ref2;  /* [B, N, d]: each row's input of policy.score_layer2 at its last pass
+                  * through that layer; NULL unless the policy has a second skip point */
 } dllm_cache;
 
 typedef struct {
@@ -143,6 +145,12 @@ typedef struct {
                      /* block with conf > unmask_tau [SF-de 2, fast phase]*/
   int refresh_every; /* dllm_generate: dense step every R steps [ES-nl 3] */
   int refresh_on_block; /* dllm_generate: dense step when a block changes */
+  /* Second skip point [ES-de 2.B, "layers 1/8 and 1/4"]: when            */
+  /* score_layer < score_layer2 < n_layers, the rows selected at           */
+  /* score_layer are scored again on their input of score_layer2 (against */
+  /* cache.h_ref2) and each sequence keeps its top-k2 of them from there.  */
+  int score_layer2;  /* 0: no second skip point                         */
+  int k2;            /* rows per sequence kept at the second skip point  */
 } dllm_policy;
 
 /* Supported shapes for DLLM_BF16 layer work: d, n_heads*head_dim,
@@ -283,6 +291,45 @@ dllm_status dllm_partial_layer(const dllm_model_cfg* cfg, const dllm_layer_w* w,
  */
 size_t dllm_step_workspace_size(const dllm_model_cfg* cfg, int B, int N,
                                 const dllm_policy* policy);
+
+/* Optional inputs and outputs of dllm_step_ex; every pointer may be NULL.
+ * The first eight mean what the dllm_step arguments of the same names mean.
+ * forced_idx2 [B, k2_cap] + forced_count2 [B] (positions, a subset of each
+ * sequence's first selection) replace the choice at the second skip point;
+ * idx2_out [B, k2_cap] / count2_out [B] receive it, with k2_cap =
+ * max(1, min(policy.k2, k_cap)); scores2_out [B, k_cap] receives the second
+ * scores of each sequence's rows in the order of its first selection. */
+typedef struct {
+  const int32_t* forced_idx;
+  const int32_t* forced_count;
+  const int32_t* forced_unmask_pos;
+  int32_t* idx_out;
+  int32_t* count_out;
+  int32_t* pos_out;
+  float* scores_out;
+  const int32_t* forced_idx2;
+  const int32_t* forced_count2;
+  int32_t* idx2_out;
+  int32_t* count2_out;
+  float* scores2_out;
+} dllm_step_io;
+
+/*
+ * dllm_step_ex - dllm_step with the second skip point of [ES-de 2.B]: after
+ * layers score_layer .. score_layer2-1 on the rows of the first selection,
+ *  a. each of them is scored as in dllm_score on its input of layer
+ *     score_layer2 against cache.h_ref2 (c = cache.conf of masked rows);
+ *  b. each sequence keeps the top-k2 of its rows (dllm_select order);
+ *  c. cache.h_ref2 rows of the kept rows <- that input;
+ *  d. layers score_layer2 .. n_layers-1 and the LM head run on the kept rows.
+ * Dropped rows keep their new K/V below score_layer2 and their cached K/V
+ * from there on.  A dense step writes cache.h_ref2 for every row.  io may be
+ * NULL.  Same workspace as dllm_step for the same policy.
+ */
+dllm_status dllm_step_ex(const dllm_model_cfg* cfg, const dllm_model_w* w,
+                         const dllm_cache* cache, int32_t* tokens, int B, int N,
+                         const dllm_policy* policy, int dense, const dllm_step_io* io, void* ws,
+                         size_t ws_bytes, dllm_stream_t stream);
 dllm_status dllm_step(const dllm_model_cfg* cfg, const dllm_model_w* w, const dllm_cache* cache,
                       int32_t* tokens, int B, int N, const dllm_policy* policy, int dense,
                       const int32_t* forced_idx, const int32_t* forced_count,

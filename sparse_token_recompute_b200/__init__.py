@@ -55,7 +55,7 @@ class ModelW(C.Structure):
 
 class CacheS(C.Structure):
     _fields_ = [("k", C.POINTER(vp)), ("v", C.POINTER(vp)), ("h_ref", vp), ("conf", vp),
-                ("pred", vp)]
+                ("pred", vp), ("h_ref2", vp)]
 
 
 class Policy(C.Structure):
@@ -63,7 +63,14 @@ class Policy(C.Structure):
                 ("mode", C.c_int), ("k", C.c_int), ("tau", C.c_float), ("n_unmask", C.c_int),
                 ("gen_start", C.c_int), ("block_len", C.c_int), ("select_from", C.c_int),
                 ("unmask_tau", C.c_float), ("refresh_every", C.c_int),
-                ("refresh_on_block", C.c_int)]
+                ("refresh_on_block", C.c_int), ("score_layer2", C.c_int), ("k2", C.c_int)]
+
+
+class StepIO(C.Structure):
+    _fields_ = [("forced_idx", vp), ("forced_count", vp), ("forced_unmask_pos", vp),
+                ("idx_out", vp), ("count_out", vp), ("pos_out", vp), ("scores_out", vp),
+                ("forced_idx2", vp), ("forced_count2", vp), ("idx2_out", vp),
+                ("count2_out", vp), ("scores2_out", vp)]
 
 
 def _sig(name, res, args):
@@ -93,6 +100,9 @@ _step_ws = _sig("dllm_step_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i,
 _step = _sig("dllm_step", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS), vp,
                                _i, _i, C.POINTER(Policy), _i, vp, vp, vp, vp, vp, vp, vp, vp,
                                _sz, vp])
+_step_ex = _sig("dllm_step_ex", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS),
+                                     vp, _i, _i, C.POINTER(Policy), _i, C.POINTER(StepIO), vp,
+                                     _sz, vp])
 _gen_ws = _sig("dllm_generate_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i,
                                                      C.POINTER(Policy)])
 _gen = _sig("dllm_generate", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS), vp,
@@ -338,13 +348,15 @@ class Model:
 class Cache:
     """Per-layer K/V caches, hidden reference, cached confidence and argmax (torch memory)."""
 
-    def __init__(self, cfg: ModelCfg, B: int, N: int, device="cuda"):
+    def __init__(self, cfg: ModelCfg, B: int, N: int, device="cuda", second_ref: bool = False):
         import torch
         dt = torch.bfloat16 if cfg.dtype == DLLM_BF16 else torch.float32
         kv = (B, N, cfg.n_kv_heads, cfg.head_dim)
         self.k = [torch.zeros(kv, dtype=dt, device=device) for _ in range(cfg.n_layers)]
         self.v = [torch.zeros(kv, dtype=dt, device=device) for _ in range(cfg.n_layers)]
         self.h_ref = torch.zeros(B, N, cfg.d, dtype=dt, device=device)
+        # reference of the second skip point (policies with score_layer2 > 0)
+        self.h_ref2 = torch.zeros(B, N, cfg.d, dtype=dt, device=device) if second_ref else None
         self.conf = torch.zeros(B, N, dtype=torch.float32, device=device)
         self.pred = torch.zeros(B, N, dtype=torch.int32, device=device)
         self._refresh()
@@ -353,15 +365,16 @@ class Cache:
         L = max(len(self.k), 1)
         self._kp = (vp * L)(*[ptr(t) for t in self.k])
         self._vp = (vp * L)(*[ptr(t) for t in self.v])
-        self.s = CacheS(self._kp, self._vp, ptr(self.h_ref), ptr(self.conf), ptr(self.pred))
+        self.s = CacheS(self._kp, self._vp, ptr(self.h_ref), ptr(self.conf), ptr(self.pred),
+                        ptr(self.h_ref2))
 
 
 def make_policy(score_layer=0, alpha=0.5, kind=DLLM_SCORE_COS, mode=DLLM_SELECT_TOPK, k=1,
                 tau=0.0, n_unmask=1, gen_start=0, block_len=32, select_from=0, unmask_tau=0.0,
-                refresh_every=0, refresh_on_block=False) -> Policy:
+                refresh_every=0, refresh_on_block=False, score_layer2=0, k2=0) -> Policy:
     return Policy(score_layer, float(alpha), kind, mode, k, float(tau), n_unmask, gen_start,
                   block_len, int(select_from), float(unmask_tau), int(refresh_every),
-                  int(bool(refresh_on_block)))
+                  int(bool(refresh_on_block)), int(score_layer2), int(k2))
 
 
 def dllm_partial_layer_workspace_size(cfg: ModelCfg, B: int, N: int, k_cap: int) -> int:
@@ -408,6 +421,22 @@ def dllm_generate(model: Model, cache: Cache, tokens, pol: Policy, n_steps: int,
               _stream(stream))
     _check(st, "dllm_generate")
     return [bool(flags[t]) for t in range(int(n_steps))]
+
+
+def dllm_step_ex(model: Model, cache: Cache, tokens, pol: Policy, dense: bool, ws: Workspace,
+                 stream=None, **io):
+    """dllm_step with the second skip point; keyword tensors fill dllm_step_io
+    (forced_idx, forced_count, forced_unmask_pos, idx_out, count_out, pos_out,
+    scores_out, forced_idx2, forced_count2, idx2_out, count2_out, scores2_out)."""
+    B, N = tokens.shape
+    s = StepIO(*[ptr(io.get(name)) for name, _ in StepIO._fields_])
+    unknown = set(io) - {name for name, _ in StepIO._fields_}
+    if unknown:
+        raise TypeError(f"unknown dllm_step_io fields: {sorted(unknown)}")
+    st = _step_ex(C.byref(model.cfg), C.byref(model.s), C.byref(cache.s), ptr(tokens), B, N,
+                  C.byref(pol), int(bool(dense)), C.byref(s), ws.ptr, ws.nbytes,
+                  _stream(stream))
+    _check(st, "dllm_step_ex")
 
 
 def dllm_step_host(model: Model, cache: Cache, tokens_host, pol: Policy, dense: bool,

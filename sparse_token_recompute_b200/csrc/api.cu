@@ -631,12 +631,28 @@ struct StepWs {
   void* lmx;      // normalized LM rows [cap, d]
   float* lm_out;  // bf16: per-tile stats [cap, tiles, 3]; f32: logits [cap, V]
   int lm_tiles;
+  // second skip point (k2_cap > 0)
+  int k2_cap;
+  float* scores2;   // [B, k_cap]
+  int32_t* idx2;    // [B, k2_cap] indices within each sequence's segment
+  int32_t* count2;  // [B]
+  int32_t* pos2;    // [B, k2_cap] positions
+  int* row_off2;    // [B + 1]
+  int* row_pos2;    // [B * k2_cap]
+  int* row_seq2;    // [B * k2_cap]
+  void* x2;         // [B * k2_cap, d]
 };
+
+int k2_cap_of(const dllm_policy* pol, int N) {
+  const int k_cap = std::max(1, std::min(pol->k, N));
+  return pol->score_layer2 > 0 ? std::max(1, std::min(pol->k2, k_cap)) : 0;
+}
 
 // the LM-head GEMM uses column tiles of 128 or 256: size its statistics for 128
 int lm_tiles_for(const dllm_model_cfg* c) { return (c->vocab + 127) / 128; }
 
-void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, StepWs& w) {
+void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, int k2_cap,
+                 StepWs& w) {
   const size_t es = esize(c->dtype);
   const int cap = B * N;  // covers the dense step
   w.status = bp.take<int>(kHeader / sizeof(int));
@@ -657,6 +673,17 @@ void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, Ste
     w.lm_tiles = 0;
     w.lm_out = bp.take<float>((size_t)cap * c->vocab);
   }
+  w.k2_cap = k2_cap;
+  if (k2_cap > 0) {
+    w.scores2 = bp.take<float>((size_t)B * k_cap);
+    w.idx2 = bp.take<int32_t>((size_t)B * k2_cap);
+    w.count2 = bp.take<int32_t>(B);
+    w.pos2 = bp.take<int32_t>((size_t)B * k2_cap);
+    w.row_off2 = bp.take<int>((size_t)B + 1);
+    w.row_pos2 = bp.take<int>((size_t)B * k2_cap);
+    w.row_seq2 = bp.take<int>((size_t)B * k2_cap);
+    w.x2 = bp.take<char>((size_t)B * k2_cap * c->d * es);
+  }
 }
 
 }  // namespace
@@ -667,7 +694,7 @@ extern "C" size_t dllm_step_workspace_size(const dllm_model_cfg* c, int B, int N
   const int k_cap = std::max(1, std::min(pol->k, N));
   Bump bp(nullptr);
   StepWs w{};
-  layout_step(bp, c, B, N, k_cap, w);
+  layout_step(bp, c, B, N, k_cap, k2_cap_of(pol, N), w);
   return bp.off;
 }
 
@@ -678,7 +705,30 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
                                  int32_t* idx_out, int32_t* count_out, int32_t* pos_out,
                                  float* scores_out, void* ws, size_t ws_bytes,
                                  dllm_stream_t stream) {
+  dllm_step_io io{};
+  io.forced_idx = forced_idx;
+  io.forced_count = forced_count;
+  io.forced_unmask_pos = forced_unmask_pos;
+  io.idx_out = idx_out;
+  io.count_out = count_out;
+  io.pos_out = pos_out;
+  io.scores_out = scores_out;
+  return dllm_step_ex(c, mw, cache, tokens, B, N, pol, dense, &io, ws, ws_bytes, stream);
+}
+
+extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w* mw,
+                                    const dllm_cache* cache, int32_t* tokens, int B, int N,
+                                    const dllm_policy* pol, int dense, const dllm_step_io* io_in,
+                                    void* ws, size_t ws_bytes, dllm_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const dllm_step_io io = io_in ? *io_in : dllm_step_io{};
+  const int32_t* forced_idx = io.forced_idx;
+  const int32_t* forced_count = io.forced_count;
+  const int32_t* forced_unmask_pos = io.forced_unmask_pos;
+  int32_t* idx_out = io.idx_out;
+  int32_t* count_out = io.count_out;
+  int32_t* pos_out = io.pos_out;
+  float* scores_out = io.scores_out;
   dllm_status st = check_cfg(c);
   if (st != DLLM_OK) return st;
   if (!mw || !cache || !pol || !tokens) return DLLM_ERR_INVALID_ARG;
@@ -705,14 +755,21 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
     return DLLM_ERR_INVALID_ARG;
   if (N > 16384 || pol->block_len > 1024) return DLLM_ERR_UNSUPPORTED_SHAPE;
   if ((forced_idx == nullptr) != (forced_count == nullptr)) return DLLM_ERR_INVALID_ARG;
+  if ((io.forced_idx2 == nullptr) != (io.forced_count2 == nullptr)) return DLLM_ERR_INVALID_ARG;
+  const int l2 = pol->score_layer2;
+  if (l2 != 0) {
+    if (l2 <= pol->score_layer || l2 >= c->n_layers || pol->k2 < 0) return DLLM_ERR_INVALID_ARG;
+    if (!cache->h_ref2 || !aligned(cache->h_ref2, 16)) return DLLM_ERR_INVALID_ARG;
+  }
   if (!ws || !aligned(ws, 256) || ws_bytes < dllm_step_workspace_size(c, B, N, pol))
     return DLLM_ERR_WORKSPACE;
 
   const int k_cap = std::max(1, std::min(pol->k, N));
+  const int k2_cap = k2_cap_of(pol, N);
   const int d = c->d;
   Bump bp(ws);
   StepWs w{};
-  layout_step(bp, c, B, N, k_cap, w);
+  layout_step(bp, c, B, N, k_cap, k2_cap, w);
   LayerWs& L = w.L;
   const bool use_rope = c->rope_theta > 0.f;
   if (use_rope) launch_rope_table(L.rope, N, c->head_dim, c->rope_theta, s);
@@ -786,24 +843,75 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
                               L.row_pos, L.row_seq, M_dev, cap, N, d, static_cast<float*>(w.x),
                               static_cast<float*>(cache->h_ref), c->vocab, w.status, s);
 
-  // 5. remaining layers on the compact rows
+  // 5. remaining layers on the compact rows (narrowed at the second skip point)
+  void* xc = w.x;
+  int cap_c = cap, rps = rows_per_seq;
+  const int* M_c = M_dev;
   for (int l = ls; l < c->n_layers; ++l) {
-    st = layer_forward(c, &mw->layers[l], w.x, cap, M_dev, L, B, N, rows_per_seq, cache->k[l],
+    if (l2 > 0 && l == l2) {
+      if (dense) {
+        if (cudaMemcpyAsync(cache->h_ref2, xc, (size_t)B * N * d * esize(c->dtype),
+                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+          return DLLM_ERR_CUDA;
+      } else {
+        if (io.forced_idx2) {
+          launch_copy_idx(io.forced_idx2, io.forced_count2, w.pos2, w.count2, B, k2_cap, s);
+        } else {
+          if (bf)
+            launch_score_rows<__nv_bfloat16>(
+                static_cast<const __nv_bfloat16*>(xc),
+                static_cast<const __nv_bfloat16*>(cache->h_ref2), L.row_off, L.row_pos,
+                L.row_seq, M_c, cap_c, N, d, k_cap, cache->conf, tokens, c->mask_id, pol->alpha,
+                pol->kind, w.scores2, s);
+          else
+            launch_score_rows<float>(static_cast<const float*>(xc),
+                                     static_cast<const float*>(cache->h_ref2), L.row_off,
+                                     L.row_pos, L.row_seq, M_c, cap_c, N, d, k_cap, cache->conf,
+                                     tokens, c->mask_id, pol->alpha, pol->kind, w.scores2, s);
+          launch_select(w.scores2, B, k_cap, 0, DLLM_SELECT_TOPK, pol->k2, 0.f, w.idx2, w.count2,
+                        k2_cap, w.status, s, w.count);
+          launch_seg_positions(w.idx2, w.count2, L.row_off, L.row_pos, B, k2_cap, w.pos2, s);
+        }
+        launch_row_map(w.pos2, w.count2, B, k2_cap, N, w.row_off2, w.row_pos2, w.row_seq2,
+                       w.status, s);
+        const int cap2 = B * k2_cap;
+        if (bf)
+          launch_gather_narrow<__nv_bfloat16>(
+              static_cast<const __nv_bfloat16*>(xc), L.row_off, L.row_pos, w.row_off2,
+              w.row_pos2, w.row_seq2, w.row_off2 + B, cap2, N, d,
+              static_cast<__nv_bfloat16*>(w.x2), static_cast<__nv_bfloat16*>(cache->h_ref2),
+              w.status, s);
+        else
+          launch_gather_narrow<float>(static_cast<const float*>(xc), L.row_off, L.row_pos,
+                                      w.row_off2, w.row_pos2, w.row_seq2, w.row_off2 + B, cap2,
+                                      N, d, static_cast<float*>(w.x2),
+                                      static_cast<float*>(cache->h_ref2), w.status, s);
+        // the kept rows' maps replace the first selection's from here on
+        L.row_off = w.row_off2;
+        L.row_pos = w.row_pos2;
+        L.row_seq = w.row_seq2;
+        M_c = w.row_off2 + B;
+        xc = w.x2;
+        cap_c = cap2;
+        rps = k2_cap;
+      }
+    }
+    st = layer_forward(c, &mw->layers[l], xc, cap_c, M_c, L, B, N, rps, cache->k[l],
                        cache->v[l], use_rope, s);
     if (st != DLLM_OK) return st;
   }
 
   // 6. LM head on selected rows that are still masked
-  launch_masked_rows(tokens, c->mask_id, L.row_pos, L.row_seq, M_dev, cap, N, w.lm_rows, w.n_lm,
+  launch_masked_rows(tokens, c->mask_id, L.row_pos, L.row_seq, M_c, cap_c, N, w.lm_rows, w.n_lm,
                      s);
   if (bf) {
     using bfl = __nv_bfloat16;
-    launch_rmsnorm_rows<bfl>(static_cast<const bfl*>(w.x), static_cast<const bfl*>(mw->final_norm),
-                             static_cast<bfl*>(w.lmx), w.lm_rows, w.n_lm, cap, d, c->rms_eps, s);
+    launch_rmsnorm_rows<bfl>(static_cast<const bfl*>(xc), static_cast<const bfl*>(mw->final_norm),
+                             static_cast<bfl*>(w.lmx), w.lm_rows, w.n_lm, cap_c, d, c->rms_eps, s);
     GemmSpec g{};
     g.epi = EPI_LMHEAD;
     g.A = static_cast<const bfl*>(w.lmx);
-    g.M_cap = cap;
+    g.M_cap = cap_c;
     g.M_dev = w.n_lm;
     g.K = d;
     g.B[0] = static_cast<const bfl*>(mw->lm_head);
@@ -813,16 +921,16 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
     g.status = w.status;
     GemmPlan pl = gemm_plan(g);
     if (gemm_launch(g, s) != cudaSuccess) return DLLM_ERR_CUDA;
-    launch_lm_merge(w.lm_out, pl.tiles_n, w.lm_rows, w.n_lm, cap, L.row_pos, L.row_seq, N,
+    launch_lm_merge(w.lm_out, pl.tiles_n, w.lm_rows, w.n_lm, cap_c, L.row_pos, L.row_seq, N,
                     cache->conf, cache->pred, s);
   } else {
-    launch_rmsnorm_rows<float>(static_cast<const float*>(w.x),
+    launch_rmsnorm_rows<float>(static_cast<const float*>(xc),
                                static_cast<const float*>(mw->final_norm),
-                               static_cast<float*>(w.lmx), w.lm_rows, w.n_lm, cap, d, c->rms_eps,
+                               static_cast<float*>(w.lmx), w.lm_rows, w.n_lm, cap_c, d, c->rms_eps,
                                s);
     launch_gemm_f32(static_cast<const float*>(w.lmx), static_cast<const float*>(mw->lm_head),
-                    w.lm_out, nullptr, w.n_lm, cap, c->vocab, d, s);
-    launch_confidence_rows_f32(w.lm_out, c->vocab, w.lm_rows, w.n_lm, cap, L.row_pos, L.row_seq,
+                    w.lm_out, nullptr, w.n_lm, cap_c, c->vocab, d, s);
+    launch_confidence_rows_f32(w.lm_out, c->vocab, w.lm_rows, w.n_lm, cap_c, L.row_pos, L.row_seq,
                                N, cache->conf, cache->pred, s);
   }
 
@@ -846,6 +954,14 @@ extern "C" dllm_status dllm_step(const dllm_model_cfg* c, const dllm_model_w* mw
     if (scores_out && !forced_idx &&
         cudaMemcpyAsync(scores_out, w.scores, (size_t)B * N * 4, cudaMemcpyDeviceToDevice, s))
       return DLLM_ERR_CUDA;
+    if (l2 > 0) {
+      if (io.idx2_out && io.count2_out)
+        launch_copy_idx(w.pos2, w.count2, io.idx2_out, io.count2_out, B, k2_cap, s);
+      if (io.scores2_out && !io.forced_idx2 &&
+          cudaMemcpyAsync(io.scores2_out, w.scores2, (size_t)B * k_cap * 4,
+                          cudaMemcpyDeviceToDevice, s))
+        return DLLM_ERR_CUDA;
+    }
   }
   return check_launch();
 }

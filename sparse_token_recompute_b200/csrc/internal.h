@@ -137,9 +137,25 @@ void launch_score(const T* h_cur, const T* embed, const int32_t* tokens, const T
                   int N, int d, const float* conf, const uint8_t* masked,
                   const int32_t* mask_tokens, int mask_id, float alpha, int kind, float* scores,
                   int vocab, int lo, int* status, cudaStream_t s);
-// positions < lo are never candidates
+// positions < lo (and >= lens[b] when lens is given) are never candidates
 void launch_select(const float* scores, int B, int N, int lo, int mode, int k, float tau,
-                   int32_t* idx, int32_t* count, int k_cap, int* status, cudaStream_t s);
+                   int32_t* idx, int32_t* count, int k_cap, int* status, cudaStream_t s,
+                   const int* lens = nullptr);
+// second skip point: scores of the compact rows into [B, k_cap] segments
+template <typename T>
+void launch_score_rows(const T* x, const T* h_ref, const int* row_off, const int* row_pos,
+                       const int* row_seq, const int* M, int cap, int N, int d, int k_cap,
+                       const float* conf, const int32_t* tokens, int mask_id, float alpha,
+                       int kind, float* scores, cudaStream_t s);
+// positions of the kept rows from their indices within each sequence's segment
+void launch_seg_positions(const int32_t* seg_idx, const int32_t* count, const int* row_off,
+                          const int* row_pos, int B, int k2_cap, int32_t* pos, cudaStream_t s);
+// narrowed compact rows (and their h_ref2 refresh) from the previous compact rows
+template <typename T>
+void launch_gather_narrow(const T* x, const int* row_off, const int* row_pos,
+                          const int* row_off2, const int* row_pos2, const int* row_seq2,
+                          const int* M2, int cap2, int N, int d, T* x2, T* h_ref2, int* status,
+                          cudaStream_t s);
 void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
                    int mask_id, int gen_start, int block_len, int n_unmask, float tau,
                    int pos_cap, int32_t* pos_out, const int32_t* forced, cudaStream_t s);

@@ -99,39 +99,13 @@ __device__ __forceinline__ void load_vec8<float>(const float* p, float* f) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-// One warp per row.  Accumulates |h|^2, |r|^2, |h-r|^2, |h-r|_1 and bitwise
+// Variation of one row against its reference, by one warp (every lane gets
+// the result).  Accumulates |h|^2, |r|^2, |h-r|^2, |h-r|_1 and bitwise
 // equality; 1 - cos is evaluated as (|h-r|^2 - (|h|-|r|)^2) / (2 |h| |r|),
 // which equals 1 - h.r/(|h||r|) and stays accurate when the rows are close.
 template <typename T>
-__global__ void __launch_bounds__(256) score_kernel(const T* __restrict__ h_cur,
-                                                    const T* __restrict__ embed,
-                                                    const int32_t* __restrict__ tokens,
-                                                    const T* __restrict__ h_ref, int rows, int N,
-                                                    int d, const float* __restrict__ conf,
-                                                    const uint8_t* __restrict__ masked,
-                                                    const int32_t* __restrict__ mask_tokens,
-                                                    int mask_id, float alpha, int kind,
-                                                    float* __restrict__ scores, int vocab,
-                                                    int lo, int* status) {
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  if (row % N < lo) {  // never a candidate (response-only step): not scored
-    if (lane == 0) scores[row] = -INFINITY;
-    return;
-  }
-  const T* hc;
-  if (tokens) {
-    int t = tokens[row];
-    if (t < 0 || t >= vocab) {
-      if (lane == 0) raise_status(status, DEV_BAD_INDEX);
-      t = t < 0 ? 0 : vocab - 1;
-    }
-    hc = embed + (size_t)t * d;
-  } else {
-    hc = h_cur + (size_t)row * d;
-  }
-  const T* hr = h_ref + (size_t)row * d;
+__device__ __forceinline__ float row_variation(const T* __restrict__ hc, const T* __restrict__ hr,
+                                               int d, int kind, int lane) {
   float nc = 0.f, nr = 0.f, dd = 0.f, l1 = 0.f;
   int eq = 1;
   // U vector pairs per lane in flight before any arithmetic
@@ -166,27 +140,83 @@ __global__ void __launch_bounds__(256) score_kernel(const T* __restrict__ h_cur,
   dd = warp_sum(dd);
   l1 = warp_sum(l1);
   eq = warp_and(eq);
-  if (lane == 0) {
-    float v;
-    if (eq) {
-      v = 0.0f;
-    } else if (kind == DLLM_SCORE_COS) {
-      const float a = sqrtf(nc), b = sqrtf(nr);
-      const float nn = a * b;
-      if (nn > 0.0f) {
-        const float t = a - b;
-        v = (dd - t * t) / (2.0f * nn);
-        v = fminf(fmaxf(v, 0.0f), 2.0f);
-      } else {
-        v = 1.0f;
-      }
+  float v;
+  if (eq) {
+    v = 0.0f;
+  } else if (kind == DLLM_SCORE_COS) {
+    const float a = sqrtf(nc), b = sqrtf(nr);
+    const float nn = a * b;
+    if (nn > 0.0f) {
+      const float t = a - b;
+      v = (dd - t * t) / (2.0f * nn);
+      v = fminf(fmaxf(v, 0.0f), 2.0f);
     } else {
-      v = nr > 0.0f ? l1 / (sqrtf((float)d) * sqrtf(nr)) : INFINITY;
+      v = 1.0f;
     }
+  } else {
+    v = nr > 0.0f ? l1 / (sqrtf((float)d) * sqrtf(nr)) : INFINITY;
+  }
+  return v;
+}
+
+// One warp per row of [B, N].
+template <typename T>
+__global__ void __launch_bounds__(256) score_kernel(const T* __restrict__ h_cur,
+                                                    const T* __restrict__ embed,
+                                                    const int32_t* __restrict__ tokens,
+                                                    const T* __restrict__ h_ref, int rows, int N,
+                                                    int d, const float* __restrict__ conf,
+                                                    const uint8_t* __restrict__ masked,
+                                                    const int32_t* __restrict__ mask_tokens,
+                                                    int mask_id, float alpha, int kind,
+                                                    float* __restrict__ scores, int vocab,
+                                                    int lo, int* status) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  if (row % N < lo) {  // never a candidate (response-only step): not scored
+    if (lane == 0) scores[row] = -INFINITY;
+    return;
+  }
+  const T* hc;
+  if (tokens) {
+    int t = tokens[row];
+    if (t < 0 || t >= vocab) {
+      if (lane == 0) raise_status(status, DEV_BAD_INDEX);
+      t = t < 0 ? 0 : vocab - 1;
+    }
+    hc = embed + (size_t)t * d;
+  } else {
+    hc = h_cur + (size_t)row * d;
+  }
+  const float v = row_variation<T>(hc, h_ref + (size_t)row * d, d, kind, lane);
+  if (lane == 0) {
     const bool is_m =
         masked ? (masked[row] != 0) : (mask_tokens ? mask_tokens[row] == mask_id : false);
     const float c = is_m ? conf[row] : 0.0f;
     scores[row] = alpha * c + (1.0f - alpha) * v;
+  }
+}
+
+// The second skip point: one warp per compact row r < M (device count) of
+// sequence b = row_seq[r] at position p = row_pos[r]; x[r] against
+// h_ref[b, p]; the score lands at scores[b * k_cap + (r - row_off[b])].
+template <typename T>
+__global__ void __launch_bounds__(256) score_rows_kernel(
+    const T* __restrict__ x, const T* __restrict__ h_ref, const int* __restrict__ row_off,
+    const int* __restrict__ row_pos, const int* __restrict__ row_seq, const int* __restrict__ M,
+    int cap, int N, int d, int k_cap, const float* __restrict__ conf,
+    const int32_t* __restrict__ tokens, int mask_id, float alpha, int kind,
+    float* __restrict__ scores) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= cap || r >= *M) return;
+  const int b = row_seq[r], p = row_pos[r];
+  const size_t g = (size_t)b * N + p;
+  const float v = row_variation<T>(x + (size_t)r * d, h_ref + g * d, d, kind, lane);
+  if (lane == 0) {
+    const float c = tokens[g] == mask_id ? conf[g] : 0.0f;
+    scores[(size_t)b * k_cap + (r - row_off[b])] = alpha * c + (1.0f - alpha) * v;
   }
 }
 
@@ -364,11 +394,13 @@ __global__ void __launch_bounds__(128) lm_merge_kernel(const float* __restrict__
 constexpr int SEL_THREADS = 1024;
 constexpr int SEL_MAX_PER_THREAD = 16;  // N <= 16384
 
-// Candidates are the positions >= lo (all of them for top-k, those with a score
-// above tau for the threshold mode); a bit per element marks them.
+// Candidates are the positions lo <= i < len (len = lens[b], or N without
+// lens): all of them for top-k, those with a score above tau for the
+// threshold mode; a bit per element marks them.
 __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __restrict__ scores,
-                                                             int N, int lo, int mode, int k,
-                                                             float tau,
+                                                             int N, int lo,
+                                                             const int* __restrict__ lens,
+                                                             int mode, int k, float tau,
                                                              int32_t* __restrict__ idx,
                                                              int32_t* __restrict__ count,
                                                              int k_cap, int* status) {
@@ -378,6 +410,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
   const int b = blockIdx.x;
   const float* sc = scores + (size_t)b * N;
   const int E = (N + SEL_THREADS - 1) / SEL_THREADS;
+  const int len = lens ? min(max(lens[b], 0), N) : N;
   const int i0 = threadIdx.x * E;  // contiguous chunk keeps position order for the scans
   uint32_t key[SEL_MAX_PER_THREAD];
   uint32_t candm = 0u;
@@ -386,7 +419,7 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
   for (int e = 0; e < SEL_MAX_PER_THREAD; ++e) {
     key[e] = 0u;
     const int i = i0 + e;
-    if (e < E && i < N && i >= lo) {
+    if (e < E && i < len && i >= lo) {
       const float x = sc[i];
       if (mode == DLLM_SELECT_TOPK || x > tau) {  // NaN compares false
         key[e] = order_key(x);
@@ -488,6 +521,66 @@ __global__ void __launch_bounds__(SEL_THREADS) select_kernel(const float* __rest
   for (int e = 0; e < SEL_MAX_PER_THREAD; ++e)
     if (sel[e]) out[o++] = i0 + e;
   if (threadIdx.x == blockDim.x - 1) count[b] = sel_incl;
+}
+
+// ---------------------------------------------------------------- second skip point
+
+// positions of the rows kept at the second skip point: seg_idx[b, i] indexes
+// sequence b's compact segment; pos[b, i] = row_pos[row_off[b] + seg_idx[b, i]]
+__global__ void __launch_bounds__(256) seg_positions_kernel(const int32_t* __restrict__ seg_idx,
+                                                            const int32_t* __restrict__ count,
+                                                            const int* __restrict__ row_off,
+                                                            const int* __restrict__ row_pos,
+                                                            int k2_cap, int32_t* __restrict__ pos) {
+  const int b = blockIdx.x;
+  const int n = min(count[b], k2_cap), base = row_off[b], len = row_off[b + 1] - base;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int j = seg_idx[(size_t)b * k2_cap + i];
+    pos[(size_t)b * k2_cap + i] = (j >= 0 && j < len) ? row_pos[base + j] : -1;
+  }
+}
+
+// x2[r2] = x[r] for the old compact row r of the same sequence and position
+// (binary search in the old segment, ascending by position); h_ref2 of the row
+// is refreshed with it.  A position not in the old segment raises DEV_BAD_INDEX
+// and leaves the row zero.
+template <typename T>
+__global__ void __launch_bounds__(128) gather_narrow_kernel(
+    const T* __restrict__ x, const int* __restrict__ row_off, const int* __restrict__ row_pos,
+    const int* __restrict__ row_off2, const int* __restrict__ row_pos2,
+    const int* __restrict__ row_seq2, const int* __restrict__ M2, int N, int d,
+    T* __restrict__ x2, T* __restrict__ h_ref2, int* status) {
+  const int r2 = blockIdx.x;
+  if (r2 >= *M2) return;
+  const int b = row_seq2[r2], p = row_pos2[r2];
+  int lo = row_off[b], hi = row_off[b + 1] - 1, src = -1;
+  while (lo <= hi) {
+    const int mid = (lo + hi) >> 1;
+    const int q = row_pos[mid];
+    if (q == p) {
+      src = mid;
+      break;
+    }
+    if (q < p) lo = mid + 1; else hi = mid - 1;
+  }
+  T* dst = x2 + (size_t)r2 * d;
+  T* ref = h_ref2 + ((size_t)b * N + p) * d;
+  if (src < 0) {
+    if (threadIdx.x == 0) raise_status(status, DEV_BAD_INDEX);
+    for (int i = threadIdx.x; i < d; i += blockDim.x) dst[i] = T(0.f);
+    return;
+  }
+  const T* a = x + (size_t)src * d;
+  constexpr int V = 16 / sizeof(T);
+  if (d % V == 0) {
+    for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
+      const uint4 v = *reinterpret_cast<const uint4*>(a + i);
+      *reinterpret_cast<uint4*>(dst + i) = v;
+      *reinterpret_cast<uint4*>(ref + i) = v;
+    }
+  } else {
+    for (int i = threadIdx.x; i < d; i += blockDim.x) dst[i] = ref[i] = a[i];
+  }
 }
 
 // ---------------------------------------------------------------- unmask
@@ -1021,11 +1114,56 @@ template void launch_confidence<__nv_bfloat16>(const __nv_bfloat16*, const int32
                                                int, float*, int32_t*, cudaStream_t);
 
 void launch_select(const float* scores, int B, int N, int lo, int mode, int k, float tau,
-                   int32_t* idx, int32_t* count, int k_cap, int* status, cudaStream_t s) {
+                   int32_t* idx, int32_t* count, int k_cap, int* status, cudaStream_t s,
+                   const int* lens) {
   if (B <= 0) return;
   ProfScope prof("select", s);
-  select_kernel<<<B, SEL_THREADS, 0, s>>>(scores, N, lo, mode, k, tau, idx, count, k_cap, status);
+  select_kernel<<<B, SEL_THREADS, 0, s>>>(scores, N, lo, lens, mode, k, tau, idx, count, k_cap,
+                                          status);
 }
+
+template <typename T>
+void launch_score_rows(const T* x, const T* h_ref, const int* row_off, const int* row_pos,
+                       const int* row_seq, const int* M, int cap, int N, int d, int k_cap,
+                       const float* conf, const int32_t* tokens, int mask_id, float alpha,
+                       int kind, float* scores, cudaStream_t s) {
+  if (cap <= 0) return;
+  ProfScope prof("score2", s);
+  score_rows_kernel<T><<<(cap + 7) / 8, 256, 0, s>>>(x, h_ref, row_off, row_pos, row_seq, M, cap,
+                                                     N, d, k_cap, conf, tokens, mask_id, alpha,
+                                                     kind, scores);
+}
+template void launch_score_rows<float>(const float*, const float*, const int*, const int*,
+                                       const int*, const int*, int, int, int, int, const float*,
+                                       const int32_t*, int, float, int, float*, cudaStream_t);
+template void launch_score_rows<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*,
+                                               const int*, const int*, const int*, const int*,
+                                               int, int, int, int, const float*, const int32_t*,
+                                               int, float, int, float*, cudaStream_t);
+
+void launch_seg_positions(const int32_t* seg_idx, const int32_t* count, const int* row_off,
+                          const int* row_pos, int B, int k2_cap, int32_t* pos, cudaStream_t s) {
+  if (B <= 0) return;
+  seg_positions_kernel<<<B, 256, 0, s>>>(seg_idx, count, row_off, row_pos, k2_cap, pos);
+}
+
+template <typename T>
+void launch_gather_narrow(const T* x, const int* row_off, const int* row_pos,
+                          const int* row_off2, const int* row_pos2, const int* row_seq2,
+                          const int* M2, int cap2, int N, int d, T* x2, T* h_ref2, int* status,
+                          cudaStream_t s) {
+  if (cap2 <= 0) return;
+  ProfScope prof("gather", s);
+  gather_narrow_kernel<T><<<cap2, 128, 0, s>>>(x, row_off, row_pos, row_off2, row_pos2, row_seq2,
+                                               M2, N, d, x2, h_ref2, status);
+}
+template void launch_gather_narrow<float>(const float*, const int*, const int*, const int*,
+                                          const int*, const int*, const int*, int, int, int,
+                                          float*, float*, int*, cudaStream_t);
+template void launch_gather_narrow<__nv_bfloat16>(const __nv_bfloat16*, const int*, const int*,
+                                                  const int*, const int*, const int*, const int*,
+                                                  int, int, int, __nv_bfloat16*, __nv_bfloat16*,
+                                                  int*, cudaStream_t);
 
 void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int B, int N,
                    int mask_id, int gen_start, int block_len, int n_unmask, float tau,

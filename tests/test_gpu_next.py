@@ -142,3 +142,75 @@ def test_generate_equals_step_loop_bf16(lib):
     for a, b in zip(r1.cache.k + r1.cache.v + [r1.cache.h_ref, r1.cache.conf, r1.cache.pred],
                     r2.cache.k + r2.cache.v + [r2.cache.h_ref, r2.cache.conf, r2.cache.pred]):
         assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------- two skip points
+
+
+def _pad(rows, width, fill=-1):
+    a = np.full((len(rows), width), fill, dtype=np.int32)
+    for b, r in enumerate(rows):
+        a[b, :len(r)] = r
+    return torch.from_numpy(a).cuda()
+
+
+def _two_point_run(lib, shape, k2):
+    r = Run(lib, shape, score_layer2=2, k2=k2)
+    r.pol.score_layer2, r.pol.k2 = 2, k2
+    r.cache = lib.Cache(r.model.cfg, r.B, r.N, second_ref=True)
+    r.ws = lib.Workspace(lib.dllm_step_workspace_size(r.model.cfg, r.B, r.N, r.pol))
+    r.k2_cap = max(1, min(k2, r.k_cap))
+    return r
+
+
+def _two_point_forced(lib, shape, k2, tol, steps):
+    r = _two_point_run(lib, shape, k2)
+    for t in range(steps):
+        out = O.step(r.ocfg, r.ow, r.st, r.opol, dense=(t == 0))
+        io = {"forced_unmask_pos": _pad(out.unmasked, out.unmasked.shape[1])}
+        if t > 0:
+            io.update(forced_idx=_pad(out.idx, r.k_cap),
+                      forced_count=torch.tensor([len(a) for a in out.idx], dtype=torch.int32,
+                                                device="cuda"),
+                      forced_idx2=_pad(out.idx2, r.k2_cap),
+                      forced_count2=torch.tensor([len(a) for a in out.idx2], dtype=torch.int32,
+                                                 device="cuda"))
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, t == 0, r.ws, **io)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        final_idx = out.idx2 if out.idx2 is not None else out.idx
+        r.compare_state(tol, out.final_rows, final_idx)
+        assert max_abs_rel(f64(r.cache.h_ref2), r.st.h_ref2) < tol
+        r.tokens.copy_(torch.from_numpy(r.st.tokens.astype(np.int32)))
+    return r
+
+
+def test_two_point_tiny_f32_forced(lib):
+    _two_point_forced(lib, SY.with_(SY.TINY, n_layers=3), 12, TOL["f32"], 5)
+
+
+def test_two_point_bf16_forced(lib):
+    _two_point_forced(lib, _small_bf16(n_layers=4), 10, TOL["bf16"], 4)
+
+
+def test_two_point_own_decisions_follow_the_rule(lib):
+    shape = SY.with_(SY.TINY, n_layers=3)
+    r = _two_point_run(lib, shape, 12)
+    lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, True, r.ws)
+    for t in range(1, 4):
+        B = r.B
+        idx = torch.full((B, r.k_cap), -1, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+        idx2 = torch.full((B, r.k2_cap), -1, dtype=torch.int32, device="cuda")
+        cnt2 = torch.zeros(B, dtype=torch.int32, device="cuda")
+        sc2 = torch.zeros(B, r.k_cap, dtype=torch.float32, device="cuda")
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, False, r.ws, idx_out=idx,
+                         count_out=cnt, idx2_out=idx2, count2_out=cnt2, scores2_out=sc2)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        for b in range(B):
+            c = int(cnt[b])
+            first = idx[b, :c].cpu().numpy()
+            s2 = sc2[b, :c].cpu().numpy()
+            keep = first[O.select_topk(s2, 12)]
+            np.testing.assert_array_equal(idx2[b, :int(cnt2[b])].cpu().numpy(), keep)
