@@ -290,6 +290,39 @@ def gqa_measure(S, steps, warmup):
     return out
 
 
+def es_two_point_measure(S, model, shape, rank, steps, warmup):
+    """The two skip points of ES-dLLM at layers NL/8 and NL/4: every row runs the
+    first NL/8 layers, 2k rows per sequence the next NL/8, k rows the rest."""
+    import torch
+    stream = torch.cuda.current_stream()
+    l1, l2 = shape.n_layers // 8, shape.n_layers // 4
+    k1 = min(2 * shape.k, shape.seq_len)
+    pol = S.make_policy(score_layer=l1, alpha=shape.alpha, k=k1, n_unmask=shape.n_unmask,
+                        gen_start=shape.prompt_len, block_len=shape.block_len,
+                        score_layer2=l2, k2=shape.k)
+    tokens = rank_inputs(shape, rank)
+    cache = S.Cache(model.cfg, shape.batch, shape.seq_len, second_ref=True)
+    ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+    S.dllm_step_ex(model, cache, tokens, pol, True, ws)
+    for _ in range(warmup):
+        S.dllm_step_ex(model, cache, tokens, pol, False, ws)
+    torch.cuda.synchronize()
+    K = min(steps, 10)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        S.dllm_step_ex(model, cache, tokens, pol, False, ws, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / K
+    st = ws.device_status()
+    del cache, ws
+    return {"score_layers": [l1, l2], "rows_per_seq": [shape.seq_len, k1, shape.k],
+            "ms_per_step": round(ms, 4), "steps_per_s": round(1000.0 / ms, 3),
+            "tokens_per_s": round(shape.batch * shape.n_unmask * 1000.0 / ms, 2),
+            "device_status": st}
+
+
 def cpu_baseline_sample(W, cache, tokens, shape):
     """The oracle on one sequence, one layer and that sequence's LM-head rows,
     scaled to a full step: per step = 32 sequences x (32 layers x t_layer + t_lm)."""
@@ -389,6 +422,26 @@ def run_ours(args):
     n_gen = shape.gen_len // shape.n_unmask
     gen_s = (ms_dense + (n_gen - 1) * ms_step) / 1000.0
 
+    # a whole generation through dllm_generate: response-only partial steps (the
+    # prompt is never selected) with a dense step injecting the prompt every 16 steps
+    R = 16
+    pol_g = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k, n_unmask=shape.n_unmask,
+                          gen_start=shape.prompt_len, block_len=shape.block_len,
+                          select_from=shape.prompt_len, refresh_every=R)
+    tok_g = rank_inputs(shape, rank)
+    ws_g = S.Workspace(S.dllm_generate_workspace_size(model.cfg, shape.batch, shape.seq_len,
+                                                      pol_g))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    dense_flags = S.dllm_generate(model, cache, tok_g, pol_g, n_gen, ws_g, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_gen_ro = max_over_ranks(e0.elapsed_time(e1), world)
+    left = int((tok_g[:, shape.prompt_len:] == shape.mask_id).sum().item())
+    barrier(world)
+    del ws_g
+
     # roofline of the dominant kernel: the tensor-core GEMM of the layer projections
     M = shape.batch * shape.k
     q = shape.n_heads * shape.head_dim
@@ -436,6 +489,15 @@ def run_ours(args):
             "steps_per_s": round(n_gen / gen_s, 3),
             "how": f"step 0 dense + {n_gen - 1} partial steps at the timed per-step cost; "
                    f"tokens = sequences x {shape.gen_len} generated"},
+        "generation_response_only": {
+            "steps": n_gen, "refresh_every": R, "dense_steps": int(sum(dense_flags)),
+            "total_s": round(ms_gen_ro / 1000.0, 4),
+            "tokens_per_s": round(world * shape.batch * shape.gen_len / (ms_gen_ro / 1000.0), 2),
+            "steps_per_s": round(n_gen / (ms_gen_ro / 1000.0), 3),
+            "masked_left": left,
+            "how": "one dllm_generate call timed with CUDA events: partial steps select only "
+                   "generated positions, a dense step every 16 steps refreshes every cache "
+                   "(prompt injection)"},
         "e2e": {"value": round(job_tokens_per_s(world, tok_per_step, ms_e2e), 2), "unit": "tokens/s",
                 "ms_per_step": round(ms_e2e, 4),
                 "h2d_bytes_per_step": tokens.numel() * 4,
@@ -446,6 +508,9 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline_sample(W, cache, tokens, shape)
+    if not args.layers and world == 1:
+        result["es_two_point"] = es_two_point_measure(S, model, shape, rank, args.steps,
+                                                      args.warmup)
     if not args.no_bs1 and not args.layers:
         del cache, ws
         torch.cuda.empty_cache()
