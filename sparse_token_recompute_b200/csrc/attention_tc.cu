@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int off = p.row_off[b];
   const int cnt = p.row_off[b + 1] - off;
   const int q0 = blockIdx.x * (NTILE * BT);
+  griddep_launch_dependents();  // the next GEMM may start streaming its weights
   if (q0 >= cnt) return;
   const int T = (p.Nseq + BKV - 1) / BKV;
   const int nq = (cnt - q0 > BT) ? 2 : 1;  // query tiles holding rows in this CTA

@@ -85,6 +85,22 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+
+// Lets the next kernel of the stream, when it was launched with programmatic
+// stream serialization, start its CTAs (on SMs this grid leaves free) before
+// this grid has finished.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Waits until every grid this one depends on has completed and its memory
+// operations are visible; returns at once for a grid launched without
+// programmatic stream serialization.  A kernel launched with it reads no data
+// produced by earlier kernels before this call.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- shared memory / mbarrier
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

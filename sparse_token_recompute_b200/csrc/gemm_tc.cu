@@ -65,6 +65,7 @@ struct Params {
   float* lm_part;
   int V;
   int a_tx;  // bytes one A box delivers (fewer than a full 128-row tile when M_cap < 128)
+  int prefetch_b;  // issue the first unit's weight tiles before waiting on the previous kernel
   int* status;
 };
 
@@ -293,17 +294,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  int M = p.M_cap;
-  if (p.M_dev) {
-    M = *p.M_dev;
-    if (M > p.M_cap || M < 0) {
-      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, DEV_BAD_SHAPE);
-      M = M < 0 ? 0 : p.M_cap;
-    }
-  }
-  const int m_tiles = (M + BM - 1) / BM;
-  const int n_units = m_tiles * p.tiles_n * p.splits;
-
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
   auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
   auto tfull_bar = [&](int a) { return smem_u32(&bars[2 * STAGES + a]); };
@@ -337,20 +327,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the next kernel may start its CTAs on SMs this grid leaves free
+  griddep_launch_dependents();
+
+  // weight (B) tile of k-block kb of output tile n into a stage
+  auto load_b = [&](uint32_t b_dst, uint32_t bar, int kb, int n) {
+    if constexpr (EPI == EPI_SWIGLU) {
+      tma_load_2d(b_dst, &tmB0, bar, kb * BK, n * (BN / 2));
+      tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB1, bar, kb * BK, n * (BN / 2));
+    } else if constexpr (EPI == EPI_QKV) {
+      const int n0 = n * BN;
+      if (n0 < p.seg0)
+        tma_load_2d(b_dst, &tmB0, bar, kb * BK, n0);
+      else if (n0 < p.seg1)
+        tma_load_2d(b_dst, &tmB1, bar, kb * BK, n0 - p.seg0);
+      else
+        tma_load_2d(b_dst, &tmB2, bar, kb * BK, n0 - p.seg1);
+    } else {
+      tma_load_2d(b_dst, &tmB0, bar, kb * BK, n * BN);
+    }
+  };
+
+  // Weights never depend on earlier kernels: with a single row tile by
+  // capacity, the producer starts streaming this CTA's first weight tiles
+  // before it waits for the kernel that writes A (and the row count).
+  int npre = 0, pre_n = 0, pre_kb0 = 0;
+  if (p.prefetch_b && warp == 0 && lane == 0 && (int)blockIdx.x < p.tiles_n * p.splits) {
+    int m, s;
+    decode_unit(blockIdx.x, 1, p.tiles_n, p.splits, m, pre_n, s);
+    pre_kb0 = s * p.kb_per_split;
+    npre = max(0, min(STAGES, min(pre_kb0 + p.kb_per_split, p.kb_total) - pre_kb0));
+    for (int i = 0; i < npre; ++i) {  // fresh stages: no empty wait
+      mbar_arrive_expect_tx(full_bar(i), (uint32_t)p.a_tx + B_BYTES);
+      load_b(smem_u32(sB + i * B_BYTES), full_bar(i), pre_kb0 + i, pre_n);
+    }
+  }
+  griddep_wait();
+
+  int M = p.M_cap;
+  if (p.M_dev) {
+    M = *p.M_dev;
+    if (M > p.M_cap || M < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, DEV_BAD_SHAPE);
+      M = M < 0 ? 0 : p.M_cap;
+    }
+  }
+  const int m_tiles = (M + BM - 1) / BM;
+  const int n_units = m_tiles * p.tiles_n * p.splits;
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      int stage = npre % STAGES;
+      uint32_t phase = npre == STAGES ? 1u : 0u;
       uint32_t issued = 0;
       uint32_t issue_phase = 0;
       bool ok = true;
+      // the A halves of the pre-issued stages (row tile 0); when this CTA has no
+      // unit after all (no rows), they only complete the stages before exit
+      for (int i = 0; i < npre; ++i) {
+        tma_load_2d(smem_u32(sA + i * A_BYTES), &tmA, full_bar(i), (pre_kb0 + i) * BK, 0);
+        issued |= 1u << i;
+      }
+      if (npre > 0 && (int)blockIdx.x >= n_units) {
+        for (int i = 0; i < npre; ++i) mbar_wait_drain(full_bar(i), 0);
+        npre = 0;
+      }
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int m, n, s;
         decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
-        const int kb0 = s * p.kb_per_split;
-        const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
+        const int kb0 = s * p.kb_per_split + (u == (int)blockIdx.x ? npre : 0);
+        const int kb1 = min(s * p.kb_per_split + p.kb_per_split, p.kb_total);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
             ok = false;
@@ -360,20 +407,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_dst = smem_u32(sA + stage * A_BYTES);
           const uint32_t b_dst = smem_u32(sB + stage * B_BYTES);
           tma_load_2d(a_dst, &tmA, full_bar(stage), kb * BK, m * BM);
-          if constexpr (EPI == EPI_SWIGLU) {
-            tma_load_2d(b_dst, &tmB0, full_bar(stage), kb * BK, n * (BN / 2));
-            tma_load_2d(b_dst + (BN / 2) * BK * 2, &tmB1, full_bar(stage), kb * BK, n * (BN / 2));
-          } else if constexpr (EPI == EPI_QKV) {
-            const int n0 = n * BN;
-            if (n0 < p.seg0)
-              tma_load_2d(b_dst, &tmB0, full_bar(stage), kb * BK, n0);
-            else if (n0 < p.seg1)
-              tma_load_2d(b_dst, &tmB1, full_bar(stage), kb * BK, n0 - p.seg0);
-            else
-              tma_load_2d(b_dst, &tmB2, full_bar(stage), kb * BK, n0 - p.seg1);
-          } else {
-            tma_load_2d(b_dst, &tmB0, full_bar(stage), kb * BK, n * BN);
-          }
+          load_b(b_dst, full_bar(stage), kb, n);
           issued |= 1u << stage;
           if (phase) issue_phase |= 1u << stage; else issue_phase &= ~(1u << stage);
           if (++stage == STAGES) {
@@ -552,6 +586,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------- host side
 
 // [rows, cols] bf16 row-major, box (64 cols, box_rows rows), 128-byte swizzle
+// programmatic dependent launch of the GEMMs; DLLM_PDL=0 turns it off (cross-check)
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DLLM_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows) {
   if (rows <= 0 || cols <= 0) return false;
   return tmap_bf16_2d(m, ptr, (uint64_t)rows, (uint64_t)cols, (uint32_t)box_rows);
@@ -568,23 +611,30 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (p.splits == 1) {
-    gemm_tc_kernel<BN, EPI><<<grid, NUM_THREADS, smem, s>>>(a, b0, b1, b2, p);
-    return cudaGetLastError();
-  }
-  // split K: one unit per CTA, the `splits` CTAs of a tile in one cluster
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)p.splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  if (p.splits > 1) {
+    // split K: one unit per CTA, the `splits` CTAs of a tile in one cluster
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = (unsigned)p.splits;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  if (pdl_enabled()) {
+    // may start while the previous kernel finishes; the kernel waits for it
+    // (griddepcontrol.wait) before reading anything that kernel writes
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, EPI>, a, b0, b1, b2, p);
 }
 
@@ -631,24 +681,39 @@ GemmPlan gemm_plan(const GemmSpec& g) {
   };
   const bool weight_bound = g.M_cap < 256;
   if (!bn && weight_bound) {
-    // Weight streaming (fewer than 256 rows): each CTA keeps a ring of 32 KB
-    // weight boxes in flight, and about 64 streaming CTAs saturate HBM (ncu and
-    // split sweeps on the 77-row projections of the 8B shape: O-proj 23 -> 15 us
-    // at 4 splits, down 60 -> 25 us; QKV and gate/up fastest unsplit with 48 and
-    // 96 tiles).  So: the widest tile the epilogue allows, then split K across a
-    // cluster until ~64 CTAs stream.
-    for (int c : {256, 128, 64}) {
-      if (bn_ok(c)) {
-        bn = c;
-        break;
-      }
+    // Weight streaming (fewer than 256 rows): a CTA streams its weight boxes at
+    // roughly 40-60 GB/s, so the GEMM wants ~96-148 streaming CTAs in one wave,
+    // with as few K splits as reach that (each split adds a cluster reduction)
+    // and at least 16 k-blocks per split.  Measured with cold weights at 77 and
+    // 192 rows of the 8B projections (us): QKV 12288x4096 tile 128 unsplit 24.5
+    // (tile 256: 32.7, 2 splits 31.7); O 4096x4096 tile 128 x 4 splits 13.6
+    // (tile 256 x 4: 17.6); down 4096x12288 tile 128 x 4 splits 24.7 (tile 256
+    // x 4: 31.7); gate/up 24576x4096 tile 256 unsplit 39.8 (tile 128: 47.6); at
+    // 192 rows QKV tile 256 unsplit 35.0 and down tile 256 x 4 splits 33.7.
+    // A single row tile prefers 128-wide tiles (more CTAs), two row tiles 256.
+    const int order1[2] = {128, 256}, order2[2] = {256, 128};
+    const int* order = pl.m_tiles_cap == 1 ? order1 : order2;
+    for (int i = 0; i < 2 && !bn; ++i) {
+      const int c = order[i];
+      if (!bn_ok(c)) continue;
+      const int t1 = tiles_for(c);
+      if (t1 > sms) continue;
+      int sp = 1;
+      if (t1 < 96 && g.epi != EPI_LMHEAD)
+        while (sp < 8 && t1 * (sp + 1) <= sms && kb_total / (sp + 1) >= 16) ++sp;
+      bn = c;
+      if (!splits) splits = sp;
     }
-    if (!bn) bn = 64;
-    const int tiles = tiles_for(bn);
-    int sp = 1;
-    if (g.epi != EPI_LMHEAD) sp = std::max(1, std::min(8, (64 + tiles / 2) / std::max(tiles, 1)));
-    while (sp > 1 && kb_total / sp < 4) --sp;
-    if (!splits) splits = sp;
+    if (!bn) {
+      // more tiles than SMs even at 256 columns: persistent CTAs, no split
+      for (int c : {256, 128, 64}) {
+        if (bn_ok(c)) {
+          bn = c;
+          break;
+        }
+      }
+      if (!bn) bn = 64;
+    }
   } else if (!bn) {
     // Tensor-bound: time ~ waves x main loop of a tile; no split.
     const int cands[3] = {256, 128, 64};
@@ -722,6 +787,7 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   // reads 128 smem rows, but rows >= M_cap only feed output rows that are never stored
   const int a_rows = g.M_cap < BM ? ((g.M_cap + 15) / 16) * 16 : BM;
   p.a_tx = a_rows * BK * 2;
+  p.prefetch_b = (g.M_cap <= BM && pdl_enabled()) ? 1 : 0;
   if (!make_map(&ta, g.A, g.M_cap, g.K, a_rows)) return cudaErrorInvalidValue;
   const int bbox = (g.epi == EPI_SWIGLU) ? pl.bn / 2 : pl.bn;
   if (!make_map(&tb0, g.B[0], g.seg_cols[0], g.K, bbox)) return cudaErrorInvalidValue;

@@ -841,6 +841,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x,
                                                       const T* __restrict__ g, T* __restrict__ o,
                                                       const int* __restrict__ M_dev, int M_cap,
                                                       int d, float eps) {
+  griddep_launch_dependents();  // the next GEMM may start streaming its weights
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
   if (r >= M) return;
