@@ -26,6 +26,9 @@ pytestmark = pytest.mark.gpu
     (129, 200, 72, 1, False),
     (1000, 1024, 1024, 0, False),
     (2048, 2048, 2048, 1, False),
+    (500, 1024, 4096, 0, False),     # four row tiles, few column tiles
+    (400, 4096, 12288, 0, True),     # four row tiles, deep K, residual accumulate
+    (257, 8192, 1024, 0, False),     # three row tiles, the last one holding one row
 ])
 def test_gemm_bf16(lib, M, N, K, splits, acc):
     A = SY.normal((M, K), 1.0, 11 + M, "cuda", "bf16")
@@ -39,12 +42,13 @@ def test_gemm_bf16(lib, M, N, K, splits, acc):
     assert err < 1e-2, err
 
 
-def test_gemm_split_k_is_deterministic(lib):
-    A = SY.normal((77, 4096), 1.0, 3, "cuda", "bf16")
+@pytest.mark.parametrize("M", [77, 300])
+def test_gemm_split_k_is_deterministic(lib, M):
+    A = SY.normal((M, 4096), 1.0, 3, "cuda", "bf16")
     Bm = SY.normal((4096, 4096), 0.02, 4, "cuda", "bf16")
     outs = []
     for _ in range(3):
-        Cm = torch.zeros(77, 4096, dtype=torch.bfloat16, device="cuda")
+        Cm = torch.zeros(M, 4096, dtype=torch.bfloat16, device="cuda")
         lib.dllm_gemm_bf16(A, Bm, Cm, splits=4)
         outs.append(Cm)
     torch.cuda.synchronize()
