@@ -71,6 +71,12 @@ in the design notes):
     keeps the top-k2 of its rows for layers l2..L-1 and the LM head.  Rows
     dropped at l2 keep their fresh K/V below l2 and their cached K/V from l2
     on.  A dense step writes h_ref2 for every row.
+  * Approximate attention of stable rows [DyLLM §2.B]: a row that is not
+    recomputed keeps its query and the statistics (max, sum, output) of its
+    last exact attention; when some keys change, their old terms are taken
+    out of the softmax sums and their new terms put in (reference max raised
+    to cover the new scores).  Exact when the query is current; DyLLM's
+    approximation when the query is stale.
   * Periodic refresh [ES-nl Methodologie 3]: in a generation, a step is
     dense (every row recomputed, every cache rewritten) at step 0, every
     refresh_every steps, and, with refresh_on_block, at the first step at
@@ -292,6 +298,62 @@ def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
         p = softmax_rows((q[:, h, :] @ K[:, g, :].T) * scale)
         out[:, h, :] = p @ V[:, g, :]
     return out
+
+
+def attention_stats(q: np.ndarray, K: np.ndarray, V: np.ndarray):
+    """attention() together with each row's softmax statistics, per query head:
+    m = max_j s_j and l = sum_j exp(s_j - m), s_j = q . k_j / sqrt(hd).
+    Returns (m [R, Hq], l [R, Hq], o [R, Hq, hd])."""
+    R, Hq, hd = q.shape
+    Hkv = K.shape[1]
+    m = np.empty((R, Hq))
+    l = np.empty((R, Hq))
+    o = np.empty((R, Hq, hd))
+    scale = 1.0 / math.sqrt(hd)
+    for h in range(Hq):
+        g = (h * Hkv) // Hq
+        s = (q[:, h, :] @ K[:, g, :].T) * scale
+        m[:, h] = np.max(s, axis=1)
+        e = np.exp(s - m[:, h:h + 1])
+        l[:, h] = np.sum(e, axis=1)
+        o[:, h, :] = (e @ V[:, g, :]) / l[:, h:h + 1]
+    return m, l, o
+
+
+def attention_update(q, m, l, o, K_old, V_old, K_new, V_new):
+    """Attention of stable rows after some keys changed [DyLLM §2.B].
+
+    The rows' queries q [R, Hq, hd] and statistics (m, l, o) from their last
+    exact attention are reused; only the changed keys contribute work: their
+    old terms are taken out of the softmax sums and their new terms put in,
+    against the reference max(m, new scores).  K_old, V_old, K_new, V_new
+    [A, Hkv, hd] are the changed keys' values before and after the step.  When
+    (m, l, o) are exact for the old keys and q is the row's current query, the
+    result is the exact attention over the updated keys; with a stale q it is
+    DyLLM's approximation (weights of unchanged keys reused).
+    Returns (m', l', o')."""
+    R, Hq, hd = q.shape
+    Hkv = K_new.shape[1]
+    scale = 1.0 / math.sqrt(hd)
+    m2 = np.empty((R, Hq))
+    l2 = np.empty((R, Hq))
+    o2 = np.empty((R, Hq, hd))
+    for h in range(Hq):
+        g = (h * Hkv) // Hq
+        s_old = (q[:, h, :] @ K_old[:, g, :].T) * scale
+        s_new = (q[:, h, :] @ K_new[:, g, :].T) * scale
+        mh = m[:, h]
+        if s_new.shape[1]:
+            mh = np.maximum(mh, np.max(s_new, axis=1))
+        w = l[:, h] * np.exp(m[:, h] - mh)
+        e_old = np.exp(s_old - mh[:, None])
+        e_new = np.exp(s_new - mh[:, None])
+        lh = w - e_old.sum(axis=1) + e_new.sum(axis=1)
+        num = w[:, None] * o[:, h, :] - e_old @ V_old[:, g, :] + e_new @ V_new[:, g, :]
+        m2[:, h] = mh
+        l2[:, h] = lh
+        o2[:, h, :] = num / lh[:, None]
+    return m2, l2, o2
 
 
 def silu(x: np.ndarray) -> np.ndarray:

@@ -13,6 +13,11 @@
   layers from the second point on untouched; after a dense step a two-point
   step is a fixed point; the rows kept at the second point dominate the
   dropped ones by brute force.
+* Incremental attention of stable rows (DyLLM, French summary §2.B): after
+  some keys change, updating the cached statistics with the changed keys'
+  old and new terms equals the attention over the updated keys computed
+  directly; no change, every key changed and a key replaced by itself are
+  the limits.
 """
 import itertools
 
@@ -280,3 +285,51 @@ def test_two_point_selection_brute_force():
 def _key(v, p):
     v = float(v)
     return (0, 0.0, -int(p)) if np.isnan(v) else (1, v + 0.0, -int(p))
+
+
+# ----------------------------------------------------------------- incremental attention
+
+
+def _kv(rng, N, Hkv, hd, scale=1.0):
+    return rng.normal(0, scale, (N, Hkv, hd)), rng.normal(0, 1.0, (N, Hkv, hd))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2)])
+def test_attention_update_equals_attention_on_updated_keys(Hq, Hkv):
+    rng = np.random.default_rng(21)
+    N, hd, R = 40, 16, 7
+    K, V = _kv(rng, N, Hkv, hd)
+    q = rng.normal(0, 1.0, (R, Hq, hd))
+    m, l, o = O.attention_stats(q, K, V)
+    np.testing.assert_allclose(o, O.attention(q, K, V), rtol=1e-12, atol=1e-12)
+    A = np.array([3, 9, 10, 27, 39])
+    K2, V2 = K.copy(), V.copy()
+    K2[A] = rng.normal(0, 2.0, (len(A), Hkv, hd))     # some new scores exceed the old max
+    V2[A] = rng.normal(0, 1.0, (len(A), Hkv, hd))
+    m2, l2, o2 = O.attention_update(q, m, l, o, K[A], V[A], K2[A], V2[A])
+    me, le, oe = O.attention_stats(q, K2, V2)
+    np.testing.assert_allclose(o2, oe, rtol=1e-10, atol=1e-10)
+    # the same softmax: l e^m agrees (the reference max may stay above the new max)
+    np.testing.assert_allclose(l2 * np.exp(m2 - me), le, rtol=1e-10)
+    assert np.all(m2 >= me - 1e-12)
+
+
+def test_attention_update_limits():
+    rng = np.random.default_rng(22)
+    N, Hkv, hd, R = 12, 2, 8, 5
+    K, V = _kv(rng, N, Hkv, hd)
+    q = rng.normal(0, 1.0, (R, 2, hd))
+    m, l, o = O.attention_stats(q, K, V)
+    # no key changed: nothing moves
+    e = np.zeros((0, Hkv, hd))
+    m2, l2, o2 = O.attention_update(q, m, l, o, e, e, e, e)
+    np.testing.assert_allclose(o2, o, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(l2, l, rtol=1e-13)
+    # every key changed: the attention over the new keys
+    K2, V2 = _kv(rng, N, Hkv, hd)
+    m2, l2, o2 = O.attention_update(q, m, l, o, K, V, K2, V2)
+    np.testing.assert_allclose(o2, O.attention(q, K2, V2), rtol=1e-9, atol=1e-9)
+    # a changed key replaced by itself: nothing moves
+    A = np.array([0, 5])
+    m2, l2, o2 = O.attention_update(q, m, l, o, K[A], V[A], K[A], V[A])
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
