@@ -378,6 +378,48 @@ dllm_status dllm_attention_bf16(const void* q, const void* k_cache, const void* 
                                 dllm_stream_t stream);
 
 /*
+ * dllm_attention_stats_bf16 - dllm_attention_bf16 that also returns each
+ * row's softmax statistics per query head, in natural-log units: a reference
+ * m and l = sum_j exp(q.k_j / sqrt(head_dim) - m), so that m + log(l) is the
+ * log-sum-exp of the row's scores.  m is the largest score up to the kernel's
+ * lazy raise (it can sit below the maximum by at most 8 ln 2, which keeps
+ * every exp(s - m) <= 256).  m, l: [B*k_cap, n_heads] f32, rows packed like q
+ * and o.  They are what dllm_attention_update_bf16 keeps up to date for rows
+ * that are not recomputed.
+ */
+dllm_status dllm_attention_stats_bf16(const void* q, const void* k_cache, const void* v_cache,
+                                      void* o, float* m, float* l, const int32_t* count, int B,
+                                      int k_cap, int N, int n_heads, int n_kv_heads, int head_dim,
+                                      void* ws, size_t ws_bytes, dllm_stream_t stream);
+
+/*
+ * dllm_attention_update_bf16 - the approximate attention of rows that are not
+ * recomputed [DyLLM 2.B]: such a row keeps its query and the statistics
+ * (m, l, o) of its last exact attention; when some of its sequence's keys
+ * change, only those keys are visited: each one's old term leaves the softmax
+ * sums and its new term enters them (reference maximum raised to cover the
+ * new scores).  With the row's current query this equals the attention over
+ * the updated keys; with a stale one it is DyLLM's reuse of the unchanged
+ * keys' weights.  Cost O(rows x changed keys) instead of O(rows x N).
+ * q: [B*r_cap, n_heads*head_dim] bf16, the stable rows' cached queries packed
+ *    by sequence (r_count[b] rows for sequence b, as in dllm_attention_bf16);
+ * o: same layout, in/out (the cached outputs, then the updated ones);
+ * m, l: [B*r_cap, n_heads] f32 in/out, natural-log units as above;
+ * k_new, v_new, k_old, v_old: [B*a_cap, n_kv_heads, head_dim] bf16, the changed
+ *    keys' values after and before the change, packed by sequence
+ *    (a_count[b] keys for sequence b).
+ * Rows of a sequence with no changed key are left untouched.  head_dim 64 or
+ * 128.  ws: dllm_attention_update_workspace_size(B) bytes.
+ */
+size_t dllm_attention_update_workspace_size(int B);
+dllm_status dllm_attention_update_bf16(const void* q, void* o, float* m, float* l,
+                                       const int32_t* r_count, int B, int r_cap,
+                                       const void* k_new, const void* v_new, const void* k_old,
+                                       const void* v_old, const int32_t* a_count, int a_cap,
+                                       int n_heads, int n_kv_heads, int head_dim, void* ws,
+                                       size_t ws_bytes, dllm_stream_t stream);
+
+/*
  * dllm_attention_bf16_noalloc - dllm_attention_bf16 without a workspace, for
  * callers that cannot allocate device memory: code running while a CUDA
  * graph is captured (cudaMalloc cannot be captured and may synchronise the

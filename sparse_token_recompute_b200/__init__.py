@@ -112,6 +112,11 @@ _devstat = _sig("dllm_get_device_status", _i, [vp, vp, C.POINTER(C.c_int32)])
 _attn_noalloc = _sig("dllm_attention_bf16_noalloc", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i,
                                                          _i, vp])
 _attn_ws = _sig("dllm_attention_workspace_size", _sz, [_i])
+_attn_stats = _sig("dllm_attention_stats_bf16", _i, [vp, vp, vp, vp, vp, vp, vp, _i, _i, _i, _i,
+                                                     _i, _i, vp, _sz, vp])
+_attn_upd_ws = _sig("dllm_attention_update_workspace_size", _sz, [_i])
+_attn_upd = _sig("dllm_attention_update_bf16", _i, [vp, vp, vp, vp, vp, _i, _i, vp, vp, vp, vp,
+                                                    vp, _i, _i, _i, _i, vp, _sz, vp])
 _attn = _sig("dllm_attention_bf16", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i, _i, vp, _sz,
                                          vp])
 _gemm_ws = _sig("dllm_gemm_workspace_size", _sz, [_i, _i, _i, _i])
@@ -280,6 +285,36 @@ def dllm_attention_bf16(q, k_cache, v_cache, o, count, k_cap: int, ws: Workspace
     st = _attn(ptr(q), ptr(k_cache), ptr(v_cache), ptr(o), ptr(count), B, int(k_cap), N, Hq, Hkv,
                hd, ws.ptr, ws.nbytes, _stream(stream))
     _check(st, "dllm_attention_bf16")
+    return ws
+
+
+def dllm_attention_stats_bf16(q, k_cache, v_cache, o, m, l, count, k_cap: int,
+                              ws: Workspace = None, stream=None):
+    """dllm_attention_bf16 plus each row's softmax statistics m, l [B*k_cap, Hq] (f32)."""
+    B, N, Hkv, hd = k_cache.shape
+    Hq = q.shape[1] // hd
+    if ws is None:
+        ws = Workspace(dllm_attention_workspace_size(B), q.device)
+    st = _attn_stats(ptr(q), ptr(k_cache), ptr(v_cache), ptr(o), ptr(m), ptr(l), ptr(count), B,
+                     int(k_cap), N, Hq, Hkv, hd, ws.ptr, ws.nbytes, _stream(stream))
+    _check(st, "dllm_attention_stats_bf16")
+    return ws
+
+
+def dllm_attention_update_bf16(q, o, m, l, r_count, r_cap: int, k_new, v_new, k_old, v_old,
+                               a_count, a_cap: int, n_kv_heads: int, ws: Workspace = None,
+                               stream=None):
+    """Incremental attention of stable rows (see include/dllm.h); q/o [B*r_cap, Hq*hd],
+    m/l [B*r_cap, Hq] updated in place; changed keys [B*a_cap, Hkv, hd]."""
+    B = r_count.shape[0]
+    hd = k_new.shape[-1]
+    Hq = q.shape[1] // hd
+    if ws is None:
+        ws = Workspace(int(_attn_upd_ws(B)), q.device)
+    st = _attn_upd(ptr(q), ptr(o), ptr(m), ptr(l), ptr(r_count), B, int(r_cap), ptr(k_new),
+                   ptr(v_new), ptr(k_old), ptr(v_old), ptr(a_count), int(a_cap), Hq,
+                   int(n_kv_heads), hd, ws.ptr, ws.nbytes, _stream(stream))
+    _check(st, "dllm_attention_update_bf16")
     return ws
 
 

@@ -558,6 +558,74 @@ extern "C" dllm_status dllm_attention_bf16(const void* q, const void* k_cache,
   return e == cudaSuccess ? check_launch() : DLLM_ERR_CUDA;
 }
 
+extern "C" dllm_status dllm_attention_stats_bf16(const void* q, const void* k_cache,
+                                                 const void* v_cache, void* o, float* m, float* l,
+                                                 const int32_t* count, int B, int k_cap, int N,
+                                                 int n_heads, int n_kv_heads, int head_dim,
+                                                 void* ws, size_t ws_bytes, dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B < 0 || k_cap < 1 || N < 0 || n_heads <= 0 || n_kv_heads <= 0) return DLLM_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || N == 0) return DLLM_OK;
+  if (!q || !k_cache || !v_cache || !o || !count || !m || !l) return DLLM_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16))
+    return DLLM_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dllm_attention_workspace_size(B))
+    return DLLM_ERR_WORKSPACE;
+  Bump bp(ws);
+  int* status = bp.take<int>(kHeader / sizeof(int));
+  int* row_off = bp.take<int>((size_t)B + 1);
+  launch_row_map(nullptr, count, B, k_cap, N, row_off, nullptr, nullptr, status, s);
+  const cudaError_t e = launch_attention_tc(
+      static_cast<const __nv_bfloat16*>(q), B * k_cap, static_cast<const __nv_bfloat16*>(k_cache),
+      static_cast<const __nv_bfloat16*>(v_cache), static_cast<__nv_bfloat16*>(o), row_off, B,
+      k_cap, N, n_heads, n_kv_heads, head_dim, status, s, m, l);
+  return e == cudaSuccess ? check_launch() : DLLM_ERR_CUDA;
+}
+
+extern "C" size_t dllm_attention_update_workspace_size(int B) {
+  Bump bp(nullptr);
+  bp.take<char>(kHeader);
+  bp.take<int>((size_t)std::max(B, 0) + 1);
+  bp.take<int>((size_t)std::max(B, 0) + 1);
+  return bp.off;
+}
+
+extern "C" dllm_status dllm_attention_update_bf16(const void* q, void* o, float* m, float* l,
+                                                  const int32_t* r_count, int B, int r_cap,
+                                                  const void* k_new, const void* v_new,
+                                                  const void* k_old, const void* v_old,
+                                                  const int32_t* a_count, int a_cap, int n_heads,
+                                                  int n_kv_heads, int head_dim, void* ws,
+                                                  size_t ws_bytes, dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (B < 0 || r_cap < 1 || a_cap < 1 || n_heads <= 0 || n_kv_heads <= 0)
+    return DLLM_ERR_INVALID_ARG;
+  if (n_heads % n_kv_heads) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (head_dim != 64 && head_dim != 128) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0) return DLLM_OK;
+  if (!q || !o || !m || !l || !r_count || !k_new || !v_new || !k_old || !v_old || !a_count)
+    return DLLM_ERR_INVALID_ARG;
+  for (const void* ptr : {q, static_cast<const void*>(o), k_new, v_new, k_old, v_old})
+    if (!aligned(ptr, 16)) return DLLM_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dllm_attention_update_workspace_size(B))
+    return DLLM_ERR_WORKSPACE;
+  Bump bp(ws);
+  int* status = bp.take<int>(kHeader / sizeof(int));
+  int* r_off = bp.take<int>((size_t)B + 1);
+  int* a_off = bp.take<int>((size_t)B + 1);
+  launch_row_map(nullptr, r_count, B, r_cap, r_cap, r_off, nullptr, nullptr, status, s);
+  launch_row_map(nullptr, a_count, B, a_cap, a_cap, a_off, nullptr, nullptr, status, s);
+  const cudaError_t e = launch_attention_update(
+      static_cast<const __nv_bfloat16*>(q), B * r_cap, static_cast<__nv_bfloat16*>(o), m, l,
+      r_off, r_cap, static_cast<const __nv_bfloat16*>(k_new),
+      static_cast<const __nv_bfloat16*>(v_new), static_cast<const __nv_bfloat16*>(k_old),
+      static_cast<const __nv_bfloat16*>(v_old), a_off, B * a_cap, B, n_heads, n_kv_heads,
+      head_dim, status, s);
+  return e == cudaSuccess ? check_launch() : DLLM_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- partial layer
 
 extern "C" size_t dllm_partial_layer_workspace_size(const dllm_model_cfg* c, int B, int N,

@@ -66,6 +66,11 @@ struct AttnParams {
   int Nseq, Hq, Hkv, ldo;
   float scale_log2;
   int* status;
+  // per query row and head, natural-log units: m = max score, l = sum exp(s - m);
+  // written by the attention when non-null, read and updated by the update mode
+  float* st_m;
+  float* st_l;
+  const int* a_off;  // update mode: changed keys of sequence b at rows a_off[b]..a_off[b+1]
 };
 
 // 32 columns without the trailing wait: several loads in flight before one wait
@@ -156,23 +161,40 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
-template <int HD>
+// UPD = false: attention of the selected rows over the sequence's N cached keys.
+// UPD = true: the incremental update of stable rows [DyLLM 2.B]: the "keys"
+// are the sequence's changed keys, first with their new values (tmK, tmV), then
+// with their old values (tmK2, tmV2) entering the sums with a negative sign; the
+// reference maximum starts at the row's cached m, and the epilogue merges the
+// sums into the cached (m, l, o).
+template <int HD, bool UPD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
+                   const __grid_constant__ CUtensorMap tmV2, const AttnParams p) {
   using L = Smem<HD>;
   constexpr int NB = HD / 64;  // 64-column boxes per row of Q/K/V
+  constexpr float kLog2e = 1.4426950408889634f;
   const int b = blockIdx.z, h = blockIdx.y;
   const int off = p.row_off[b];
   const int cnt = p.row_off[b + 1] - off;
   const int q0 = blockIdx.x * (NTILE * BT);
   griddep_launch_dependents();  // the next GEMM may start streaming its weights
   if (q0 >= cnt) return;
-  const int T = (p.Nseq + BKV - 1) / BKV;
+  // update mode: a_cnt changed keys -> TH tiles of new values, then TH of old
+  const int a_base = UPD ? p.a_off[b] : 0;
+  const int a_cnt = UPD ? p.a_off[b + 1] - a_base : 0;
+  const int TH = UPD ? (a_cnt + BKV - 1) / BKV : 0;
+  const int T = UPD ? 2 * TH : (p.Nseq + BKV - 1) / BKV;
+  if (T == 0) return;  // no changed key: the cached statistics stand
+  // keys of K/V tile t that exist (the rest score -inf)
+  auto tile_keys = [&](int t) {
+    return UPD ? min(BKV, a_cnt - (t % TH) * BKV) : min(BKV, p.Nseq - t * BKV);
+  };
   const int nq = (cnt - q0 > BT) ? 2 : 1;  // query tiles holding rows in this CTA
   // A lone query tile splits the keys instead: group A takes K/V tiles [0, TA),
   // group B [TA, T), and the two partial softmax results are merged at the end.
-  const bool split = nq == 1 && T >= 2;
+  const bool split = !UPD && nq == 1 && T >= 2;
   const int TA = split ? (T + 1) / 2 : T;
   const int TB = split ? T - TA : T;
   const int ngroups = (nq == 2 || split) ? 2 : 1;
@@ -237,6 +259,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if (UPD) {
+      tma_prefetch_desc(&tmK2);
+      tma_prefetch_desc(&tmV2);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -256,10 +282,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t u = use_par(n);
         if (!mbar_wait(empty(sl), u ^ 1u, abort_flag, p.status)) return false;
         mbar_arrive_expect_tx(full(sl), L::KV_BYTES);
-        const CUtensorMap* tm = is_v ? &tmV : &tmK;
+        const bool old = UPD && tile >= TH;
+        const CUtensorMap* tm = is_v ? (old ? &tmV2 : &tmV) : (old ? &tmK2 : &tmK);
+        const int row = UPD ? a_base + (tile - (old ? TH : 0)) * BKV : krow0 + tile * BKV;
         for (int c = 0; c < NB; ++c)
           tma_load_2d(sRing + sl * L::KV_BYTES + c * BKV * 128, tm, full(sl), g * HD + c * 64,
-                      krow0 + tile * BKV);
+                      row);
         issued |= 1u << sl;
         issue_par = (issue_par & ~(1u << sl)) | (u << sl);
         ++n;
@@ -397,6 +425,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (x < ngroups && quad < live_warps(x)) {
       const float sc = p.scale_log2;
       float m_ref = -INFINITY, lsum = 0.f;  // reference maximum in the exp2 domain
+      const int row_x = q0 + qtile(x) * BT + r;  // this thread's row in the sequence
+      const size_t st_i = (size_t)(off + row_x) * p.Hq + h;
+      if (UPD) m_ref = row_x < cnt ? p.st_m[st_i] * kLog2e : 0.f;  // the cached maximum
       bool ok = true;
       const int nj = ntiles(x);
       for (int j = 0; j < nj; ++j) {
@@ -407,10 +438,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int c = 0; c < BKV; c += 32) tmem_ld32_nowait(tS(x) + lane_off + c, s + c);
         tmem_wait_ld();
-        const int kbase = (kv_first(x) + j) * BKV;
-        if (kbase + BKV > p.Nseq) {
+        const int nkeys = tile_keys(kv_first(x) + j);
+        if (nkeys < BKV) {
 #pragma unroll
-          for (int i = 0; i < BKV; ++i) s[i] = (kbase + i < p.Nseq) ? s[i] : -INFINITY;
+          for (int i = 0; i < BKV; ++i) s[i] = (i < nkeys) ? s[i] : -INFINITY;
         }
         // the maximum of the raw scores (the scale is positive)
         float mxv[4];
@@ -420,14 +451,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < BKV; i += 2) mxv[(i >> 1) & 3] = fmax3(mxv[(i >> 1) & 3], s[i], s[i + 1]);
         const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])) * sc;
         // raise the reference maximum only when this tile exceeds it by > 2^8
-        const bool need = (j == 0) || (mx > m_ref + kRescaleLog2);
+        // (the update mode starts from the cached maximum, not from tile 0)
+        const bool first = !UPD && j == 0;
+        const bool need = first || (mx > m_ref + kRescaleLog2);
         const bool rescale_o = __any_sync(0xffffffffu, need && j > 0);
         float alpha = 1.f;
         if (need) {
-          alpha = (j == 0) ? 0.f : ex2_approx(m_ref - mx);
+          alpha = first ? 0.f : ex2_approx(m_ref - mx);
           m_ref = mx;
         }
-        lsum *= (j == 0) ? 0.f : alpha;
+        lsum *= first ? 0.f : alpha;
         if (rescale_o) {
           // S_X(j) complete implies PV_X(j-1) complete: O_X is stable until P_X(j) is ready
 #pragma unroll 1
@@ -449,7 +482,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
         for (int i = 0; i < BKV; i += 2) {
           const float x0 = fmaf(s[i], sc, neg_m), x1 = fmaf(s[i + 1], sc, neg_m);
-          const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+          if (UPD && j >= TH) {  // an old key's term leaves the sums
+            e0 = -e0;
+            e1 = -e1;
+          }
           rsv[i & 7] += e0;
           rsv[(i + 1) & 7] += e1;
           pk[i >> 1] = pack_bf2(e0, e1);
@@ -474,18 +511,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_after();
       }
       if (ok && (x == 0 || !split)) {
-        const int row = q0 + qtile(x) * BT + r;
-        float wa = 1.f, wb = 0.f;
+        const int row = row_x;
+        float wa = 1.f, wb = 0.f, m_out = m_ref, w_old = 0.f;
         if (split) {
           const float mb = stat[r], lb = stat[BT + r];
           const float mm = fmaxf(m_ref, mb);
           wa = ex2_approx(m_ref - mm);
           wb = ex2_approx(mb - mm);
           lsum = lsum * wa + lb * wb;
+          m_out = mm;
+        }
+        if (UPD && row < cnt) {
+          // the cached sum and output, brought to the final reference
+          w_old = p.st_l[st_i] * ex2_approx(p.st_m[st_i] * kLog2e - m_ref);
+          lsum += w_old;
         }
         const float inv = 1.0f / lsum;
         wa *= inv;
         wb *= inv;
+        w_old *= inv;
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           float o[32], ob[32];
@@ -499,9 +543,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               float f[8];
 #pragma unroll
               for (int t = 0; t < 8; ++t) f[t] = split ? o[i + t] * wa + ob[i + t] * wb : o[i + t] * wa;
+              if (UPD) {
+                float prev[8];
+                unpack8(*reinterpret_cast<const uint4*>(dst + i), prev);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) f[t] = fmaf(w_old, prev[t], f[t]);
+              }
               *reinterpret_cast<uint4*>(dst + i) = pack8(f);
             }
           }
+        }
+        if (row < cnt && p.st_m) {
+          p.st_m[st_i] = m_out / kLog2e;
+          p.st_l[st_i] = lsum;
         }
       }
     }
@@ -515,18 +569,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int HD>
+template <int HD, bool UPD>
 cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                      const AttnParams& p, dim3 grid, cudaStream_t s) {
+                      const CUtensorMap& k2, const CUtensorMap& v2, const AttnParams& p, dim3 grid,
+                      cudaStream_t s) {
   constexpr int smem = Smem<HD>::TOTAL;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD>,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, UPD>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  attn_tc_kernel<HD><<<grid, NTHREADS, smem, s>>>(q, k, v, p);
+  attn_tc_kernel<HD, UPD><<<grid, NTHREADS, smem, s>>>(q, k, v, k2, v2, p);
   return cudaGetLastError();
 }
 
@@ -535,7 +590,7 @@ cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensor
 cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
                                 const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
                                 int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
-                                cudaStream_t s) {
+                                cudaStream_t s, float* st_m, float* st_l) {
   if (B <= 0 || k_cap <= 0 || M_cap <= 0) return cudaSuccess;
   if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv;
@@ -544,10 +599,36 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
     return cudaErrorInvalidValue;
   if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
     return cudaErrorInvalidValue;
-  AttnParams p{row_off, o, Nseq, Hq, Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd), status};
+  AttnParams p{row_off, o,      Nseq, Hq,      Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
+               status,  st_m,   st_l, nullptr};
   dim3 grid((k_cap + NTILE * BT - 1) / (NTILE * BT), Hq, B);
   ProfScope prof("attention", s);
-  return hd == 128 ? launch_hd<128>(tq, tk, tv, p, grid, s) : launch_hd<64>(tq, tk, tv, p, grid, s);
+  return hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
+                   : launch_hd<64, false>(tq, tk, tv, tk, tv, p, grid, s);
+}
+
+cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bfloat16* o,
+                                    float* st_m, float* st_l, const int* r_off, int r_cap,
+                                    const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                                    const __nv_bfloat16* k_old, const __nv_bfloat16* v_old,
+                                    const int* a_off, int A_cap, int B, int Hq, int Hkv, int hd,
+                                    int* status, cudaStream_t s) {
+  if (B <= 0 || r_cap <= 0 || R_cap <= 0 || A_cap <= 0) return cudaSuccess;
+  if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv, tk2, tv2;
+  const uint64_t cols = (uint64_t)Hkv * hd;
+  if (!tmap_bf16_2d(&tq, q, (uint64_t)R_cap, (uint64_t)Hq * hd, BT) ||
+      !tmap_bf16_2d(&tk, k_new, (uint64_t)A_cap, cols, BKV) ||
+      !tmap_bf16_2d(&tv, v_new, (uint64_t)A_cap, cols, BKV) ||
+      !tmap_bf16_2d(&tk2, k_old, (uint64_t)A_cap, cols, BKV) ||
+      !tmap_bf16_2d(&tv2, v_old, (uint64_t)A_cap, cols, BKV))
+    return cudaErrorInvalidValue;
+  AttnParams p{r_off, o,    0,    Hq,   Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
+               status, st_m, st_l, a_off};
+  dim3 grid((r_cap + NTILE * BT - 1) / (NTILE * BT), Hq, B);
+  ProfScope prof("attention_update", s);
+  return hd == 128 ? launch_hd<128, true>(tq, tk, tv, tk2, tv2, p, grid, s)
+                   : launch_hd<64, true>(tq, tk, tv, tk2, tv2, p, grid, s);
 }
 
 }  // namespace dllm

@@ -115,11 +115,21 @@ void launch_confidence_rows_f32(const float* logits, int V, const int* lm_rows, 
                                 float* conf, int32_t* pred, cudaStream_t s);
 
 // ----- bf16 attention -----
-// tcgen05 flash attention (Q compact [M_cap, Hq*hd], caches [B, N, Hkv, hd])
+// tcgen05 flash attention (Q compact [M_cap, Hq*hd], caches [B, N, Hkv, hd]); with st_m/st_l
+// non-null also each row's softmax statistics [M_cap, Hq] (max score, sum of exp(s - max))
 cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
                                 const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
                                 int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
-                                cudaStream_t s);
+                                cudaStream_t s, float* st_m = nullptr, float* st_l = nullptr);
+// incremental attention of stable rows: q [R_cap, Hq*hd] with cached o, st_m, st_l (in/out),
+// rows of sequence b at r_off[b].. (at most r_cap); changed keys' new and old K/V
+// [A_cap, Hkv*hd] compact, sequence b at rows a_off[b]..a_off[b+1]
+cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bfloat16* o,
+                                    float* st_m, float* st_l, const int* r_off, int r_cap,
+                                    const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
+                                    const __nv_bfloat16* k_old, const __nv_bfloat16* v_old,
+                                    const int* a_off, int A_cap, int B, int Hq, int Hkv, int hd,
+                                    int* status, cudaStream_t s);
 // warp-level MMA flash attention (mma.sync), kept for comparison
 void launch_attention_bf16(const __nv_bfloat16* q, const __nv_bfloat16* kc,
                            const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,

@@ -83,6 +83,32 @@ def case_attention(a):
             "kv_bytes": 2 * a.B * a.N * a.kv_heads * hd * 2}
 
 
+def case_attention_update(a):
+    """Incremental attention of the stable rows of one 8B layer: B sequences, N - k
+    stable rows each, k changed keys each (the rows the step recomputed)."""
+    H, hd, Hkv = a.heads, 128, a.kv_heads
+    R = a.N - a.k
+    q = SY.normal((a.B * R, H * hd), 1.0, 1, "cuda", "bf16")
+    o = SY.normal((a.B * R, H * hd), 0.05, 2, "cuda", "bf16")
+    m = torch.zeros(a.B * R, H, dtype=torch.float32, device="cuda")
+    l = torch.full((a.B * R, H), float(a.N), dtype=torch.float32, device="cuda")
+    kv = [SY.normal((a.B * a.k, Hkv, hd), 1.0, 3 + i, "cuda", "bf16") for i in range(4)]
+    rc = torch.full((a.B,), R, dtype=torch.int32, device="cuda")
+    ac = torch.full((a.B,), a.k, dtype=torch.int32, device="cuda")
+    ws = S.Workspace(S._attn_upd_ws(a.B))
+    m0, l0, o0 = m.clone(), l.clone(), o.clone()
+
+    def run():
+        m.copy_(m0), l.copy_(l0), o.copy_(o0)
+        S.dllm_attention_update_bf16(q, o, m, l, rc, R, kv[0], kv[1], kv[2], kv[3], ac, a.k, Hkv,
+                                     ws=ws)
+    reset_ms = _time(lambda: (m.copy_(m0), l.copy_(l0), o.copy_(o0)), a.warmup, a.iters)
+    ms = _time(run, a.warmup, a.iters) - reset_ms
+    fl = 2.0 * 2 * (2 * a.k) * R * H * hd * a.B   # QK and PV over old + new keys
+    return {"case": "attention_update", "stable_rows": R, "changed": a.k, "ms": ms,
+            "tflops": fl / ms / 1e9}
+
+
 def case_step(a):
     """Whole partial denoising steps of the 8B model at batch B, N tokens, ratio r:
     one dense step, `--warmup` partial steps, then `--iters` timed partial steps."""
@@ -123,7 +149,8 @@ def case_layer(a):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "score", "layer", "attention", "step"])
+    ap.add_argument("case", choices=["gemm", "score", "layer", "attention", "attention_update",
+                                     "step"])
     ap.add_argument("--ratio", type=float, default=0.10)
     ap.add_argument("--heads", type=int, default=32)
     ap.add_argument("--kv-heads", dest="kv_heads", type=int, default=32)
@@ -142,11 +169,12 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     a = ap.parse_args()
     if a.k is None:
-        a.k = 308 if a.case in ("layer", "attention") else 256
-    if a.case in ("layer", "attention"):
+        a.k = 308 if a.case in ("layer", "attention", "attention_update") else 256
+    if a.case in ("layer", "attention", "attention_update"):
         a.N = 1536 if a.N == 12288 else a.N
     out = {"gemm": case_gemm, "score": case_score, "layer": case_layer,
-           "attention": case_attention, "step": case_step}[a.case](a)
+           "attention": case_attention, "attention_update": case_attention_update,
+           "step": case_step}[a.case](a)
     print(json.dumps(out))
 
 

@@ -214,3 +214,66 @@ def test_two_point_own_decisions_follow_the_rule(lib):
             s2 = sc2[b, :c].cpu().numpy()
             keep = first[O.select_topk(s2, 12)]
             np.testing.assert_array_equal(idx2[b, :int(cnt2[b])].cpu().numpy(), keep)
+
+
+# ----------------------------------------------------------------- incremental attention
+
+
+def _lse(m, l):
+    return np.asarray(m, dtype=np.float64) + np.log(np.asarray(l, dtype=np.float64))
+
+
+@pytest.mark.parametrize("Hq,Hkv,hd", [(4, 2, 128), (2, 2, 64)])
+def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
+    g = torch.Generator().manual_seed(31)
+    B, N, r_cap, a_cap = 3, 300, 150, 40
+    r_count = [150, 70, 33]
+    a_count = [40, 7, 0]          # the last sequence has no changed key
+    kc = SY.normal((B, N, Hkv, hd), 1.0, 41, "cuda", "bf16")
+    vc = SY.normal((B, N, Hkv, hd), 1.0, 42, "cuda", "bf16")
+    q = SY.normal((B * r_cap, Hq * hd), 1.0, 43, "cuda", "bf16")
+    o = torch.zeros_like(q)
+    m = torch.zeros(B * r_cap, Hq, dtype=torch.float32, device="cuda")
+    l = torch.zeros_like(m)
+    rc = torch.tensor(r_count, dtype=torch.int32, device="cuda")
+    lib.dllm_attention_stats_bf16(q, kc, vc, o, m, l, rc, r_cap)
+    torch.cuda.synchronize()
+    # statistics of the exact attention: the same log-sum-exp as the oracle's
+    off = 0
+    for b, c in enumerate(r_count):
+        qb = f64(q[off:off + c]).reshape(c, Hq, hd)
+        om, ol, oo = O.attention_stats(qb, f64(kc[b]), f64(vc[b]))
+        assert np.max(np.abs(_lse(m[off:off + c].cpu(), l[off:off + c].cpu()) - _lse(om, ol))) < 2e-2
+        assert max_abs_rel(f64(o[off:off + c]), O.store(oo, "bf16").reshape(c, -1)) < TOL["bf16"]
+        off += c
+    # change a_count[b] keys of each sequence (new keys larger: new scores pass the old max)
+    k_new = torch.zeros(B * a_cap, Hkv, hd, dtype=torch.bfloat16, device="cuda")
+    v_new, k_old, v_old = torch.zeros_like(k_new), torch.zeros_like(k_new), torch.zeros_like(k_new)
+    kc2, vc2 = kc.clone(), vc.clone()
+    aoff = 0
+    for b, a in enumerate(a_count):
+        pos = torch.randperm(N, generator=g)[:a].sort()[0].cuda()
+        kn = (torch.randn(a, Hkv, hd, generator=g) * 1.8).to(torch.bfloat16).cuda()
+        vn = torch.randn(a, Hkv, hd, generator=g).to(torch.bfloat16).cuda()
+        k_old[aoff:aoff + a], v_old[aoff:aoff + a] = kc[b, pos], vc[b, pos]
+        k_new[aoff:aoff + a], v_new[aoff:aoff + a] = kn, vn
+        kc2[b, pos], vc2[b, pos] = kn, vn
+        aoff += a
+    ac = torch.tensor(a_count, dtype=torch.int32, device="cuda")
+    o_before, m_before, l_before = o.clone(), m.clone(), l.clone()
+    ws = lib.dllm_attention_update_bf16(q, o, m, l, rc, r_cap, k_new, v_new, k_old, v_old, ac,
+                                        a_cap, Hkv)
+    torch.cuda.synchronize()
+    assert ws.device_status() == 0
+    off = 0
+    for b, c in enumerate(r_count):
+        sl = slice(off, off + c)
+        if a_count[b] == 0:
+            assert torch.equal(o[sl], o_before[sl]) and torch.equal(m[sl], m_before[sl])
+            assert torch.equal(l[sl], l_before[sl])
+        else:
+            qb = f64(q[sl]).reshape(c, Hq, hd)
+            em, el, eo = O.attention_stats(qb, f64(kc2[b]), f64(vc2[b]))
+            assert max_abs_rel(f64(o[sl]), O.store(eo, "bf16").reshape(c, -1)) < TOL["bf16"]
+            assert np.max(np.abs(_lse(m[sl].cpu(), l[sl].cpu()) - _lse(em, el))) < 2e-2
+        off += c
