@@ -71,6 +71,13 @@ in the design notes):
     keeps the top-k2 of its rows for layers l2..L-1 and the LM head.  Rows
     dropped at l2 keep their fresh K/V below l2 and their cached K/V from l2
     on.  A dense step writes h_ref2 for every row.
+  * FFN gating [DyLLM §2.A]: with ffn_gate on, each recomputed row compares
+    its attention output of the layer (the context C_{t,l}, as stored) with
+    the one cached at its last pass (1 - cos); above ffn_tau the row is
+    salient and runs the FFN, else it adds the FFN output cached at its last
+    salient pass.  The FFN output is a stored tensor (rounded before the
+    residual add) so that both branches add the same kind of value.  Dense
+    steps treat every row as salient and fill both caches.
   * Approximate attention of stable rows [DyLLM §2.B]: a row that is not
     recomputed keeps its query and the statistics (max, sum, output) of its
     last exact attention; when some keys change, their old terms are taken
@@ -207,6 +214,8 @@ class Policy:
     score_layer2: int = 0         # > score_layer: second skip point (0: none)
     k2: int = 0                   # rows per sequence kept at the second skip point
     select_from: int = 0          # positions below it are never selected (partial steps)
+    ffn_gate: bool = False        # DyLLM FFN gating on the attention context
+    ffn_tau: float = 0.0          # salient when 1 - cos(context, cached context) > ffn_tau
     unmask_tau: float = 0.0       # > 0: over-threshold unmasking with top-n fallback
     refresh_every: int = 0        # generation: dense step every R steps (0: never)
     refresh_on_block: bool = False  # generation: dense step when a block changes
@@ -222,12 +231,16 @@ class State:
     conf: np.ndarray                    # [B, N] cached confidence
     pred: np.ndarray                    # [B, N] cached argmax token
     h_ref2: Optional[np.ndarray] = None  # [B, N, d] hidden at the second skip point
+    ctx: Optional[List[np.ndarray]] = None  # per layer [B, N, Hq*hd] attention output
+    ffn: Optional[List[np.ndarray]] = None  # per layer [B, N, d] FFN output
 
     def copy(self) -> "State":
+        cp = lambda a: None if a is None else [x.copy() for x in a]
         return State(self.tokens.copy(), [a.copy() for a in self.k],
                      [a.copy() for a in self.v], self.h_ref.copy(),
                      self.conf.copy(), self.pred.copy(),
-                     None if self.h_ref2 is None else self.h_ref2.copy())
+                     None if self.h_ref2 is None else self.h_ref2.copy(), cp(self.ctx),
+                     cp(self.ffn))
 
 
 def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
@@ -237,7 +250,9 @@ def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
                  [np.zeros(kv) for _ in range(cfg.n_layers)],
                  [np.zeros(kv) for _ in range(cfg.n_layers)],
                  np.zeros((B, N, cfg.d)), np.zeros((B, N)),
-                 np.zeros((B, N), dtype=np.int64), np.zeros((B, N, cfg.d)))
+                 np.zeros((B, N), dtype=np.int64), np.zeros((B, N, cfg.d)),
+                 [np.zeros((B, N, cfg.n_heads * cfg.head_dim)) for _ in range(cfg.n_layers)],
+                 [np.zeros((B, N, cfg.d)) for _ in range(cfg.n_layers)])
 
 
 # ---------------------------------------------------------------------------
@@ -360,8 +375,21 @@ def silu(x: np.ndarray) -> np.ndarray:
     return x / (1.0 + np.exp(-x))
 
 
+@dataclass
+class FfnGate:
+    """The DyLLM FFN gate of one layer: its context and FFN-output caches
+    [B, N, .], the threshold, whether every row counts as salient (dense
+    steps), and (out) the salient flags of the rows."""
+    ctx: np.ndarray
+    ffn: np.ndarray
+    tau: float
+    all_rows: bool = False
+    salient: Optional[np.ndarray] = None
+
+
 def layer_rows(cfg: ModelCfg, w: LayerW, x: np.ndarray, b_of_row: np.ndarray,
-               pos_of_row: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray) -> np.ndarray:
+               pos_of_row: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+               gate: Optional[FfnGate] = None) -> np.ndarray:
     """One transformer layer on a set of rows; updates the layer's K/V cache.
 
     ``x`` [R, d] are the rows' layer inputs; row r belongs to sequence
@@ -387,8 +415,20 @@ def layer_rows(cfg: ModelCfg, w: LayerW, x: np.ndarray, b_of_row: np.ndarray,
     o = store(o.reshape(R, Hq * hd), dt)
     x = store(x + o @ w.wo.T, dt)
     n2 = store(rms_norm(x, w.ffn_norm, cfg.rms_eps), dt)
-    a = store(silu(n2 @ w.w_gate.T) * (n2 @ w.w_up.T), dt)
-    return store(x + a @ w.w_down.T, dt)
+    if gate is None:
+        a = store(silu(n2 @ w.w_gate.T) * (n2 @ w.w_up.T), dt)
+        return store(x + a @ w.w_down.T, dt)
+    # DyLLM §2.A: salient rows (context moved) run the FFN, the rest reuse it
+    v = variation(o, gate.ctx[b_of_row, pos_of_row], SCORE_COS)
+    sal = np.ones(R, dtype=bool) if gate.all_rows else v > gate.tau
+    gate.ctx[b_of_row, pos_of_row] = o
+    f = gate.ffn[b_of_row, pos_of_row].copy()
+    if np.any(sal):
+        a = store(silu(n2[sal] @ w.w_gate.T) * (n2[sal] @ w.w_up.T), dt)
+        f[sal] = store(a @ w.w_down.T, dt)
+        gate.ffn[b_of_row[sal], pos_of_row[sal]] = f[sal]
+    gate.salient = sal
+    return store(x + f, dt)
 
 
 # ---------------------------------------------------------------------------
@@ -573,20 +613,23 @@ class StepOut:
     final_rows: List[np.ndarray] = field(default_factory=list)  # per sequence [k_b, d]
     idx2: Optional[List[np.ndarray]] = None   # rows kept at the second skip point
     scores2: Optional[List[np.ndarray]] = None  # their scores, per sequence in idx order
+    ffn_rows: Optional[List[int]] = None  # FFN gating: salient rows per recomputed layer
 
 
 def embed(W: ModelW, tokens: np.ndarray) -> np.ndarray:
     return np.asarray(W.embed, dtype=np.float64)[tokens]
 
 
-def dense_layers(cfg: ModelCfg, W: ModelW, st: State, h: np.ndarray, upto: int) -> np.ndarray:
+def dense_layers(cfg: ModelCfg, W: ModelW, st: State, h: np.ndarray, upto: int,
+                 gate_on: bool = False) -> np.ndarray:
     """Layers 0 .. upto-1 on every row (writes every row's K/V there)."""
     B, N, d = h.shape
     b_of = np.repeat(np.arange(B), N)
     p_of = np.tile(np.arange(N), B)
     x = h.reshape(B * N, d)
     for l in range(upto):
-        x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l])
+        gate = FfnGate(st.ctx[l], st.ffn[l], 0.0, True) if gate_on else None
+        x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l], gate)
     return x.reshape(B, N, d)
 
 
@@ -630,7 +673,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
     ls = pol.score_layer
     masked = st.tokens == cfg.mask_id
     h = embed(W, st.tokens)
-    h = dense_layers(cfg, W, st, h, ls)
+    h = dense_layers(cfg, W, st, h, ls, pol.ffn_gate)
     scores = None
     if dense:
         idx = [np.arange(N, dtype=np.int64) for _ in range(B)]
@@ -647,6 +690,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
     st.h_ref[b_of, p_of] = x
     l2 = pol.score_layer2 if pol.score_layer2 > ls else -1
     idx2 = sc2 = None
+    ffn_rows = [] if pol.ffn_gate else None
     for l in range(ls, cfg.n_layers):
         if l == l2:
             if not dense:
@@ -654,7 +698,10 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
                 b_of, p_of, x = b_of[keep], p_of[keep], x[keep]
             st.h_ref2[b_of, p_of] = x
         if len(b_of):
-            x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l])
+            gate = FfnGate(st.ctx[l], st.ffn[l], pol.ffn_tau, dense) if pol.ffn_gate else None
+            x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l], gate)
+            if gate is not None:
+                ffn_rows.append(int(np.sum(gate.salient)))
     sel_masked = masked[b_of, p_of]
     if np.any(sel_masked):
         n = store(rms_norm(x[sel_masked], W.final_norm, cfg.rms_eps), cfg.dtype)
@@ -672,7 +719,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
     for a in (idx2 if idx2 is not None else idx):
         rows.append(x[off:off + len(a)].copy())
         off += len(a)
-    return StepOut(idx, scores, pos, rows, idx2, sc2)
+    return StepOut(idx, scores, pos, rows, idx2, sc2, ffn_rows)
 
 
 def block_starts(cfg: ModelCfg, pol: Policy, tokens: np.ndarray) -> List[int]:

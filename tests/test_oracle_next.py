@@ -18,6 +18,11 @@
   old and new terms equals the attention over the updated keys computed
   directly; no change, every key changed and a key replaced by itself are
   the limits.
+* FFN gating on the attention context (DyLLM, French summary §2.A): every
+  row salient is the plain layer; no row salient adds the cached FFN output
+  to the post-attention residual (taken from the same model with its FFN
+  output weight zeroed); after a dense step a gated step is a fixed point
+  that runs no FFN.
 """
 import itertools
 
@@ -333,3 +338,74 @@ def test_attention_update_limits():
     A = np.array([0, 5])
     m2, l2, o2 = O.attention_update(q, m, l, o, K[A], V[A], K[A], V[A])
     np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- FFN gating
+
+
+def _gated_setup(**kw):
+    s, cfg, W, tok = _setup(n_layers=2, **kw)
+    st = O.empty_state(cfg, tok)
+    return s, cfg, W, tok, st
+
+
+def test_ffn_gate_every_row_salient_is_the_plain_layer():
+    s, cfg, W, tok, st = _gated_setup()
+    pol = oracle_policy(s, ffn_gate=True, ffn_tau=-1.0)
+    plain = O.empty_state(cfg, tok)
+    O.step(cfg, W, st, pol, dense=True)
+    O.step(cfg, W, plain, oracle_policy(s), dense=True)
+    for t in range(3):
+        out = O.step(cfg, W, st, pol, dense=False)
+        ref = O.step(cfg, W, plain, oracle_policy(s), dense=False)
+        assert out.ffn_rows == [sum(len(a) for a in out.idx)] * cfg.n_layers
+        for a, b in zip(out.final_rows, ref.final_rows):
+            np.testing.assert_array_equal(a, b)   # f32 storage: the same sums, exactly
+    np.testing.assert_array_equal(st.tokens, plain.tokens)
+
+
+def test_ffn_gate_no_row_salient_reuses_the_cached_ffn():
+    import dataclasses
+    s, cfg, W, tok = _setup(n_layers=1)
+    st = O.empty_state(cfg, tok)
+    pol = oracle_policy(s, ffn_gate=True, ffn_tau=2.5)      # 1 - cos never exceeds 2
+    O.step(cfg, W, st, pol, dense=True)
+    st.tokens[0, s.prompt_len + 3] = 5                      # something to recompute
+    ffn0 = st.ffn[0].copy()
+    # the post-attention residual, from the plain layer of a model without FFN output
+    W0 = dataclasses.replace(W, layers=[dataclasses.replace(W.layers[0],
+                                                            w_down=np.zeros_like(W.layers[0].w_down))])
+    st0 = st.copy()
+    mid = O.step(cfg, W0, st0, oracle_policy(s), dense=False)
+    out = O.step(cfg, W, st, pol, dense=False)
+    assert out.ffn_rows == [0]
+    np.testing.assert_array_equal(st.ffn[0], ffn0)
+    np.testing.assert_array_equal(out.idx[0], mid.idx[0])
+    np.testing.assert_allclose(out.final_rows[0], mid.final_rows[0] + ffn0[0, out.idx[0]],
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_ffn_gate_fixed_point_after_dense():
+    s, cfg, W, tok, st = _gated_setup(n_unmask=0)
+    pol = oracle_policy(s, ffn_gate=True, ffn_tau=1e-9, n_unmask=0)
+    O.step(cfg, W, st, pol, dense=True)
+    ref = st.copy()
+    out = O.step(cfg, W, st, pol, dense=False)
+    # unchanged tokens: every context reproduces its cache, no FFN runs, and the rows
+    # still come out as the dense pass computed them
+    assert out.ffn_rows == [0] * cfg.n_layers
+    for a, b in zip(st.k + st.v + st.ctx, ref.k + ref.v + ref.ctx):
+        np.testing.assert_allclose(a, b, rtol=RT, atol=RT)
+    full = O.dense_forward(cfg, W, tok)
+    np.testing.assert_allclose(out.final_rows[0], full[0, out.idx[0]], rtol=RT, atol=RT)
+
+
+def test_ffn_gate_threshold_splits_rows_by_context_change():
+    s, cfg, W, tok, st = _gated_setup(n_unmask=0)
+    pol = oracle_policy(s, ffn_gate=True, ffn_tau=0.0, n_unmask=0, alpha=0.0, k=32)
+    O.step(cfg, W, st, pol, dense=True)
+    st.tokens[0, s.prompt_len:s.prompt_len + 4] = [11, 12, 13, 14]
+    out = O.step(cfg, W, st, pol, dense=False)
+    # with tau 0 exactly the rows whose context moved at all run the FFN: in the first
+    # recomputed layer every selected row sees the four changed keys
+    assert 0 < out.ffn_rows[0] <= 32
