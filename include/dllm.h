@@ -126,6 +126,11 @@ typedef struct {
   int32_t* pred;
   void* h_ref2;  /* [B, N, d]: each row's input of policy.score_layer2 at its last pass
                   * through that layer; NULL unless the policy has a second skip point */
+  /* DyLLM FFN gate (policy.ffn_gate); HOST arrays of n_layers device pointers,
+   * NULL when the gate is off: */
+  void* const* ctx;  /* [B, N, n_heads*head_dim] each row's attention output at its
+                      * last pass through the layer */
+  void* const* ffn;  /* [B, N, d] each row's FFN output at its last salient pass */
 } dllm_cache;
 
 typedef struct {
@@ -151,6 +156,12 @@ typedef struct {
   /* cache.h_ref2) and each sequence keeps its top-k2 of them from there.  */
   int score_layer2;  /* 0: no second skip point                         */
   int k2;            /* rows per sequence kept at the second skip point  */
+  /* FFN gate [DyLLM 2.A]: a recomputed row runs a layer's FFN only when its */
+  /* attention output moved since its last pass, 1 - cos > ffn_tau; else it  */
+  /* adds the FFN output cached at its last salient pass (cache.ctx/ffn).    */
+  /* Dense steps run every FFN and fill both caches.                         */
+  int ffn_gate;      /* 0: off                                           */
+  float ffn_tau;
 } dllm_policy;
 
 /* Supported shapes for DLLM_BF16 layer work: d, n_heads*head_dim,
@@ -312,6 +323,8 @@ typedef struct {
   int32_t* idx2_out;
   int32_t* count2_out;
   float* scores2_out;
+  int32_t* ffn_rows_out;  /* [n_layers] device: rows that ran each layer's FFN under the
+                           * FFN gate (layers the step did not run are left untouched) */
 } dllm_step_io;
 
 /*

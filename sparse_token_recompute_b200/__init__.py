@@ -55,7 +55,7 @@ class ModelW(C.Structure):
 
 class CacheS(C.Structure):
     _fields_ = [("k", C.POINTER(vp)), ("v", C.POINTER(vp)), ("h_ref", vp), ("conf", vp),
-                ("pred", vp), ("h_ref2", vp)]
+                ("pred", vp), ("h_ref2", vp), ("ctx", C.POINTER(vp)), ("ffn", C.POINTER(vp))]
 
 
 class Policy(C.Structure):
@@ -63,14 +63,15 @@ class Policy(C.Structure):
                 ("mode", C.c_int), ("k", C.c_int), ("tau", C.c_float), ("n_unmask", C.c_int),
                 ("gen_start", C.c_int), ("block_len", C.c_int), ("select_from", C.c_int),
                 ("unmask_tau", C.c_float), ("refresh_every", C.c_int),
-                ("refresh_on_block", C.c_int), ("score_layer2", C.c_int), ("k2", C.c_int)]
+                ("refresh_on_block", C.c_int), ("score_layer2", C.c_int), ("k2", C.c_int),
+                ("ffn_gate", C.c_int), ("ffn_tau", C.c_float)]
 
 
 class StepIO(C.Structure):
     _fields_ = [("forced_idx", vp), ("forced_count", vp), ("forced_unmask_pos", vp),
                 ("idx_out", vp), ("count_out", vp), ("pos_out", vp), ("scores_out", vp),
                 ("forced_idx2", vp), ("forced_count2", vp), ("idx2_out", vp),
-                ("count2_out", vp), ("scores2_out", vp)]
+                ("count2_out", vp), ("scores2_out", vp), ("ffn_rows_out", vp)]
 
 
 def _sig(name, res, args):
@@ -383,7 +384,8 @@ class Model:
 class Cache:
     """Per-layer K/V caches, hidden reference, cached confidence and argmax (torch memory)."""
 
-    def __init__(self, cfg: ModelCfg, B: int, N: int, device="cuda", second_ref: bool = False):
+    def __init__(self, cfg: ModelCfg, B: int, N: int, device="cuda", second_ref: bool = False,
+                 ffn_gate: bool = False):
         import torch
         dt = torch.bfloat16 if cfg.dtype == DLLM_BF16 else torch.float32
         kv = (B, N, cfg.n_kv_heads, cfg.head_dim)
@@ -392,6 +394,12 @@ class Cache:
         self.h_ref = torch.zeros(B, N, cfg.d, dtype=dt, device=device)
         # reference of the second skip point (policies with score_layer2 > 0)
         self.h_ref2 = torch.zeros(B, N, cfg.d, dtype=dt, device=device) if second_ref else None
+        # DyLLM FFN gate: per layer, attention outputs and FFN outputs of every row
+        q = cfg.n_heads * cfg.head_dim
+        self.ctx = [torch.zeros(B, N, q, dtype=dt, device=device)
+                    for _ in range(cfg.n_layers)] if ffn_gate else None
+        self.ffn = [torch.zeros(B, N, cfg.d, dtype=dt, device=device)
+                    for _ in range(cfg.n_layers)] if ffn_gate else None
         self.conf = torch.zeros(B, N, dtype=torch.float32, device=device)
         self.pred = torch.zeros(B, N, dtype=torch.int32, device=device)
         self._refresh()
@@ -400,16 +408,20 @@ class Cache:
         L = max(len(self.k), 1)
         self._kp = (vp * L)(*[ptr(t) for t in self.k])
         self._vp = (vp * L)(*[ptr(t) for t in self.v])
+        self._cp = (vp * L)(*[ptr(t) for t in self.ctx]) if self.ctx else None
+        self._fp = (vp * L)(*[ptr(t) for t in self.ffn]) if self.ffn else None
         self.s = CacheS(self._kp, self._vp, ptr(self.h_ref), ptr(self.conf), ptr(self.pred),
-                        ptr(self.h_ref2))
+                        ptr(self.h_ref2), self._cp, self._fp)
 
 
 def make_policy(score_layer=0, alpha=0.5, kind=DLLM_SCORE_COS, mode=DLLM_SELECT_TOPK, k=1,
                 tau=0.0, n_unmask=1, gen_start=0, block_len=32, select_from=0, unmask_tau=0.0,
-                refresh_every=0, refresh_on_block=False, score_layer2=0, k2=0) -> Policy:
+                refresh_every=0, refresh_on_block=False, score_layer2=0, k2=0, ffn_gate=False,
+                ffn_tau=0.0) -> Policy:
     return Policy(score_layer, float(alpha), kind, mode, k, float(tau), n_unmask, gen_start,
                   block_len, int(select_from), float(unmask_tau), int(refresh_every),
-                  int(bool(refresh_on_block)), int(score_layer2), int(k2))
+                  int(bool(refresh_on_block)), int(score_layer2), int(k2), int(bool(ffn_gate)),
+                  float(ffn_tau))
 
 
 def dllm_partial_layer_workspace_size(cfg: ModelCfg, B: int, N: int, k_cap: int) -> int:

@@ -243,9 +243,24 @@ bool attention_legacy() {
 }
 
 // One transformer layer over the compact rows in x (in place).
+// DyLLM FFN gate of one layer (see launch_ffn_gate)
+struct LayerGate {
+  void* ctx;          // [B, N, n_heads*head_dim] attention outputs at each row's last pass
+  void* ffn;          // [B, N, d] FFN outputs at each row's last salient pass
+  float tau;          // salient when 1 - cos > tau
+  int all_rows;       // every row salient (dense steps)
+  int* flag;          // [cap] scratch
+  int* list;          // [cap] salient rows
+  int* inv;           // [cap] row -> place in the list, or -1
+  int* n_sal;         // [1] salient rows
+  void* f_new;        // [cap, d] FFN outputs of the salient rows
+  int32_t* rows_out;  // this layer's salient-row count (device), or null
+};
+
 dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void* x, int M_cap,
                           const int* M_dev, const LayerWs& w, int B, int N, int k_cap,
-                          void* k_cache, void* v_cache, bool use_rope, cudaStream_t s) {
+                          void* k_cache, void* v_cache, bool use_rope, cudaStream_t s,
+                          const LayerGate* gate = nullptr) {
   const int d = c->d, q = c->n_heads * c->head_dim, kv = c->n_kv_heads * c->head_dim;
   const int F = c->ffn, hd = c->head_dim;
   const float2* rope = use_rope ? w.rope : nullptr;
@@ -301,6 +316,43 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     go.out = xb;
     go.ldo = d;
     if (gemm_launch(go, s) != cudaSuccess) return DLLM_ERR_CUDA;
+    if (gate) {
+      // DyLLM: the FFN only on rows whose attention output moved, the rest reuse it
+      launch_ffn_gate<bf>(static_cast<const bf*>(w.o), static_cast<bf*>(gate->ctx), w.row_pos,
+                          w.row_seq, M_dev, M_cap, N, q, gate->tau, gate->all_rows, gate->flag,
+                          gate->list, gate->inv, gate->n_sal, s);
+      launch_rmsnorm_rows<bf>(xb, static_cast<const bf*>(lw->ffn_norm), nb, gate->list,
+                              gate->n_sal, M_cap, d, c->rms_eps, s);
+      GemmSpec gu = g;
+      gu.epi = EPI_SWIGLU;
+      gu.A = nb;
+      gu.M_dev = gate->n_sal;
+      gu.K = d;
+      gu.B[0] = static_cast<const bf*>(lw->w_gate);
+      gu.B[1] = static_cast<const bf*>(lw->w_up);
+      gu.seg_cols[0] = F;
+      gu.seg_cols[1] = F;
+      gu.n_seg = 2;
+      gu.out = static_cast<bf*>(w.act);
+      gu.ldo = F;
+      if (gemm_launch(gu, s) != cudaSuccess) return DLLM_ERR_CUDA;
+      GemmSpec gd = gu;
+      gd.epi = EPI_STORE;
+      gd.A = static_cast<const bf*>(w.act);
+      gd.K = F;
+      gd.B[0] = static_cast<const bf*>(lw->w_down);
+      gd.seg_cols[0] = d;
+      gd.n_seg = 1;
+      gd.out = static_cast<bf*>(gate->f_new);
+      gd.ldo = d;
+      if (gemm_launch(gd, s) != cudaSuccess) return DLLM_ERR_CUDA;
+      launch_ffn_combine<bf>(xb, static_cast<const bf*>(gate->f_new), static_cast<bf*>(gate->ffn),
+                             gate->inv, w.row_pos, w.row_seq, M_dev, M_cap, N, d, s);
+      if (gate->rows_out && cudaMemcpyAsync(gate->rows_out, gate->n_sal, sizeof(int32_t),
+                                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return DLLM_ERR_CUDA;
+      return check_launch();
+    }
     launch_rmsnorm<bf>(xb, static_cast<const bf*>(lw->ffn_norm), nb, M_dev, M_cap, d, c->rms_eps,
                        s);
     GemmSpec gu = g;
@@ -343,6 +395,27 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
                          M_dev, M_cap, N, c->n_heads, c->n_kv_heads, hd, s);
     launch_gemm_f32(static_cast<const float*>(w.o), static_cast<const float*>(lw->wo), xf, xf,
                     M_dev, M_cap, d, q, s);
+    if (gate) {
+      launch_ffn_gate<float>(static_cast<const float*>(w.o), static_cast<float*>(gate->ctx),
+                             w.row_pos, w.row_seq, M_dev, M_cap, N, q, gate->tau, gate->all_rows,
+                             gate->flag, gate->list, gate->inv, gate->n_sal, s);
+      launch_rmsnorm_rows<float>(xf, static_cast<const float*>(lw->ffn_norm), nf, gate->list,
+                                 gate->n_sal, M_cap, d, c->rms_eps, s);
+      launch_gemm_f32(nf, static_cast<const float*>(lw->w_gate), w.graw, nullptr, gate->n_sal,
+                      M_cap, F, d, s);
+      launch_gemm_f32(nf, static_cast<const float*>(lw->w_up), w.uraw, nullptr, gate->n_sal,
+                      M_cap, F, d, s);
+      launch_swiglu_f32(w.graw, w.uraw, static_cast<float*>(w.act), gate->n_sal, M_cap, F, s);
+      launch_gemm_f32(static_cast<const float*>(w.act), static_cast<const float*>(lw->w_down),
+                      static_cast<float*>(gate->f_new), nullptr, gate->n_sal, M_cap, d, F, s);
+      launch_ffn_combine<float>(xf, static_cast<const float*>(gate->f_new),
+                                static_cast<float*>(gate->ffn), gate->inv, w.row_pos, w.row_seq,
+                                M_dev, M_cap, N, d, s);
+      if (gate->rows_out && cudaMemcpyAsync(gate->rows_out, gate->n_sal, sizeof(int32_t),
+                                            cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return DLLM_ERR_CUDA;
+      return check_launch();
+    }
     launch_rmsnorm<float>(xf, static_cast<const float*>(lw->ffn_norm), nf, M_dev, M_cap, d,
                           c->rms_eps, s);
     launch_gemm_f32(nf, static_cast<const float*>(lw->w_gate), w.graw, nullptr, M_dev, M_cap, F,
@@ -709,6 +782,12 @@ struct StepWs {
   int* row_pos2;    // [B * k2_cap]
   int* row_seq2;    // [B * k2_cap]
   void* x2;         // [B * k2_cap, d]
+  // DyLLM FFN gate (policy.ffn_gate)
+  int* g_flag;      // [cap]
+  int* g_list;      // [cap]
+  int* g_inv;       // [cap]
+  int* g_n;         // [1]
+  void* g_f;        // [cap, d]
 };
 
 int k2_cap_of(const dllm_policy* pol, int N) {
@@ -720,7 +799,7 @@ int k2_cap_of(const dllm_policy* pol, int N) {
 int lm_tiles_for(const dllm_model_cfg* c) { return (c->vocab + 127) / 128; }
 
 void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, int k2_cap,
-                 StepWs& w) {
+                 bool gate, StepWs& w) {
   const size_t es = esize(c->dtype);
   const int cap = B * N;  // covers the dense step
   w.status = bp.take<int>(kHeader / sizeof(int));
@@ -752,6 +831,13 @@ void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, int
     w.row_seq2 = bp.take<int>((size_t)B * k2_cap);
     w.x2 = bp.take<char>((size_t)B * k2_cap * c->d * es);
   }
+  if (gate) {
+    w.g_flag = bp.take<int>(cap);
+    w.g_list = bp.take<int>(cap);
+    w.g_inv = bp.take<int>(cap);
+    w.g_n = bp.take<int>(1);
+    w.g_f = bp.take<char>((size_t)cap * c->d * es);
+  }
 }
 
 }  // namespace
@@ -762,7 +848,7 @@ extern "C" size_t dllm_step_workspace_size(const dllm_model_cfg* c, int B, int N
   const int k_cap = std::max(1, std::min(pol->k, N));
   Bump bp(nullptr);
   StepWs w{};
-  layout_step(bp, c, B, N, k_cap, k2_cap_of(pol, N), w);
+  layout_step(bp, c, B, N, k_cap, k2_cap_of(pol, N), pol->ffn_gate != 0, w);
   return bp.off;
 }
 
@@ -824,6 +910,14 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
   if (N > 16384 || pol->block_len > 1024) return DLLM_ERR_UNSUPPORTED_SHAPE;
   if ((forced_idx == nullptr) != (forced_count == nullptr)) return DLLM_ERR_INVALID_ARG;
   if ((io.forced_idx2 == nullptr) != (io.forced_count2 == nullptr)) return DLLM_ERR_INVALID_ARG;
+  if (pol->ffn_gate) {
+    if (!(pol->ffn_tau == pol->ffn_tau)) return DLLM_ERR_INVALID_ARG;
+    if (!cache->ctx || !cache->ffn) return DLLM_ERR_INVALID_ARG;
+    for (int l = 0; l < c->n_layers; ++l)
+      if (!cache->ctx[l] || !cache->ffn[l] || !aligned(cache->ctx[l], 16) ||
+          !aligned(cache->ffn[l], 16))
+        return DLLM_ERR_INVALID_ARG;
+  }
   const int l2 = pol->score_layer2;
   if (l2 != 0) {
     if (l2 <= pol->score_layer || l2 >= c->n_layers || pol->k2 < 0) return DLLM_ERR_INVALID_ARG;
@@ -837,13 +931,20 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
   const int d = c->d;
   Bump bp(ws);
   StepWs w{};
-  layout_step(bp, c, B, N, k_cap, k2_cap, w);
+  layout_step(bp, c, B, N, k_cap, k2_cap, pol->ffn_gate != 0, w);
   LayerWs& L = w.L;
   const bool use_rope = c->rope_theta > 0.f;
   if (use_rope) launch_rope_table(L.rope, N, c->head_dim, c->rope_theta, s);
   const bool bf = c->dtype == DLLM_BF16;
   const int ls = pol->score_layer;
   const int* M_dev = L.row_off + B;
+  auto gate_of = [&](int l, bool all_rows, LayerGate& gt) -> const LayerGate* {
+    if (!pol->ffn_gate) return nullptr;
+    gt = LayerGate{cache->ctx[l], cache->ffn[l], pol->ffn_tau, all_rows ? 1 : 0, w.g_flag,
+                   w.g_list, w.g_inv, w.g_n, w.g_f,
+                   io.ffn_rows_out ? io.ffn_rows_out + l : nullptr};
+    return &gt;
+  };
 
   // 1. hidden at the score layer: embeddings, then dense layers below it
   const void* h_src = nullptr;  // [B, N, d] source of the score-layer hidden, or null = embed
@@ -859,8 +960,9 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
                                 L.row_seq, M_dev, B * N, N, d, static_cast<float*>(w.h_full),
                                 nullptr, c->vocab, w.status, s);
     for (int l = 0; l < ls; ++l) {
+      LayerGate gt;
       st = layer_forward(c, &mw->layers[l], w.h_full, B * N, M_dev, L, B, N, N, cache->k[l],
-                         cache->v[l], use_rope, s);
+                         cache->v[l], use_rope, s, gate_of(l, true, gt));
       if (st != DLLM_OK) return st;
     }
     h_src = w.h_full;
@@ -964,8 +1066,9 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
         rps = k2_cap;
       }
     }
+    LayerGate gt;
     st = layer_forward(c, &mw->layers[l], xc, cap_c, M_c, L, B, N, rps, cache->k[l],
-                       cache->v[l], use_rope, s);
+                       cache->v[l], use_rope, s, gate_of(l, dense != 0, gt));
     if (st != DLLM_OK) return st;
   }
 

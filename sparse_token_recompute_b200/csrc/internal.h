@@ -171,6 +171,17 @@ void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int 
                    int pos_cap, int32_t* pos_out, const int32_t* forced, cudaStream_t s);
 void launch_block_start(const int32_t* tokens, int B, int N, int mask_id, int gen_start,
                         int block_len, int32_t* out, cudaStream_t s);
+// DyLLM FFN gate: flag rows whose attention output moved (1 - cos > tau, or all rows),
+// refresh the context cache, compact the salient rows (list, inverse map, count)
+template <typename T>
+void launch_ffn_gate(const T* o, T* ctx, const int* row_pos, const int* row_seq,
+                     const int* M_dev, int M_cap, int N, int q, float tau, int all_rows,
+                     int* flag, int* list, int* inv, int* n_sal, cudaStream_t s);
+// x[r] += FFN output: the new one of a salient row (cached too) or the cached one
+template <typename T>
+void launch_ffn_combine(T* x, const T* f_new, T* f_cache, const int* inv, const int* row_pos,
+                        const int* row_seq, const int* M_dev, int M_cap, int N, int d,
+                        cudaStream_t s);
 void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
                      int32_t* dst_count, int B, int k_cap, cudaStream_t s);
 

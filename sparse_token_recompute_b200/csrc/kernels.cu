@@ -898,6 +898,87 @@ __global__ void __launch_bounds__(1024) masked_rows_kernel(const int32_t* __rest
   if (threadIdx.x == 0) *n_out = s_carry;
 }
 
+// ---------------------------------------------------------------- DyLLM FFN gate
+
+// One warp per compact row r < M: the row's attention output o[r] against the
+// context cached at its last pass, ctx[b, p] (1 - cos); salient when all_rows
+// or 1 - cos > tau; the cache takes o[r].
+template <typename T>
+__global__ void __launch_bounds__(256) ffn_gate_kernel(const T* __restrict__ o, T* __restrict__ ctx,
+                                                       const int* __restrict__ row_pos,
+                                                       const int* __restrict__ row_seq,
+                                                       const int* __restrict__ M_dev, int M_cap,
+                                                       int N, int q, float tau, int all_rows,
+                                                       int* __restrict__ flag) {
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  const T* a = o + (size_t)r * q;
+  T* c = ctx + ((size_t)row_seq[r] * N + row_pos[r]) * q;
+  const float v = row_variation<T>(a, c, q, DLLM_SCORE_COS, lane);
+  __syncwarp();
+  for (int i = lane; i < q; i += 32) c[i] = a[i];
+  if (lane == 0) flag[r] = (all_rows || v > tau) ? 1 : 0;
+}
+
+// rows r < M with flag[r] -> list (ascending) and count; inv[r] = position in the
+// list or -1
+__global__ void __launch_bounds__(1024) flag_compact_kernel(const int* __restrict__ flag,
+                                                            const int* __restrict__ M_dev,
+                                                            int M_cap, int* __restrict__ list,
+                                                            int* __restrict__ inv,
+                                                            int* __restrict__ n_out) {
+  __shared__ int red[33];
+  __shared__ int s_carry;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int r0 = 0; r0 < M; r0 += blockDim.x) {
+    const int r = r0 + threadIdx.x;
+    const int f = (r < M && flag[r]) ? 1 : 0;
+    const int incl = block_inclusive_scan(f, red);
+    const int carry = s_carry;
+    if (r < M) {
+      inv[r] = f ? carry + incl - 1 : -1;
+      if (f) list[carry + incl - 1] = r;
+    }
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) s_carry = carry + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *n_out = s_carry;
+}
+
+// x[r] = x[r] + f, with f = the FFN output just computed for a salient row (also
+// written to the row's cache) or the cached one; one block per row
+template <typename T>
+__global__ void __launch_bounds__(128) ffn_combine_kernel(T* __restrict__ x,
+                                                          const T* __restrict__ f_new,
+                                                          T* __restrict__ f_cache,
+                                                          const int* __restrict__ inv,
+                                                          const int* __restrict__ row_pos,
+                                                          const int* __restrict__ row_seq,
+                                                          const int* __restrict__ M_dev,
+                                                          int M_cap, int N, int d) {
+  const int r = blockIdx.x;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  const int j = inv[r];
+  T* fc = f_cache + ((size_t)row_seq[r] * N + row_pos[r]) * d;
+  T* xr = x + (size_t)r * d;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) {
+    T f;
+    if (j >= 0) {
+      f = f_new[(size_t)j * d + i];
+      fc[i] = f;
+    } else {
+      f = fc[i];
+    }
+    xr[i] = T((float)xr[i] + (float)f);
+  }
+}
+
 __global__ void copy_idx_kernel(const int32_t* src_idx, const int32_t* src_count,
                                 int32_t* dst_idx, int32_t* dst_count, int B, int k_cap) {
   const size_t total = (size_t)B * k_cap;
@@ -1194,6 +1275,38 @@ void launch_row_map_dense(int B, int N, int* row_off, int* row_pos, int* row_seq
   row_map_dense_kernel<<<grid_for((size_t)B * N, 256), 256, 0, s>>>(B, N, row_off, row_pos,
                                                                     row_seq);
 }
+
+template <typename T>
+void launch_ffn_gate(const T* o, T* ctx, const int* row_pos, const int* row_seq,
+                     const int* M_dev, int M_cap, int N, int q, float tau, int all_rows,
+                     int* flag, int* list, int* inv, int* n_sal, cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("ffn_gate", s);
+  ffn_gate_kernel<T><<<(M_cap + 7) / 8, 256, 0, s>>>(o, ctx, row_pos, row_seq, M_dev, M_cap, N, q,
+                                                     tau, all_rows, flag);
+  flag_compact_kernel<<<1, 1024, 0, s>>>(flag, M_dev, M_cap, list, inv, n_sal);
+}
+template void launch_ffn_gate<float>(const float*, float*, const int*, const int*, const int*, int,
+                                     int, int, float, int, int*, int*, int*, int*, cudaStream_t);
+template void launch_ffn_gate<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, const int*,
+                                             const int*, const int*, int, int, int, float, int,
+                                             int*, int*, int*, int*, cudaStream_t);
+
+template <typename T>
+void launch_ffn_combine(T* x, const T* f_new, T* f_cache, const int* inv, const int* row_pos,
+                        const int* row_seq, const int* M_dev, int M_cap, int N, int d,
+                        cudaStream_t s) {
+  if (M_cap <= 0) return;
+  ProfScope prof("ffn_combine", s);
+  ffn_combine_kernel<T><<<M_cap, 128, 0, s>>>(x, f_new, f_cache, inv, row_pos, row_seq, M_dev,
+                                              M_cap, N, d);
+}
+template void launch_ffn_combine<float>(float*, const float*, float*, const int*, const int*,
+                                        const int*, const int*, int, int, int, cudaStream_t);
+template void launch_ffn_combine<__nv_bfloat16>(__nv_bfloat16*, const __nv_bfloat16*,
+                                                __nv_bfloat16*, const int*, const int*,
+                                                const int*, const int*, int, int, int,
+                                                cudaStream_t);
 
 void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
                      int32_t* dst_count, int B, int k_cap, cudaStream_t s) {

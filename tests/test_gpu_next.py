@@ -277,3 +277,63 @@ def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
             assert max_abs_rel(f64(o[sl]), O.store(eo, "bf16").reshape(c, -1)) < TOL["bf16"]
             assert np.max(np.abs(_lse(m[sl].cpu(), l[sl].cpu()) - _lse(em, el))) < 2e-2
         off += c
+
+
+# ----------------------------------------------------------------- FFN gate
+
+
+def _gated_run(lib, shape, tau):
+    r = Run(lib, shape, ffn_gate=True, ffn_tau=tau)
+    r.pol.ffn_gate, r.pol.ffn_tau = 1, tau
+    r.cache = lib.Cache(r.model.cfg, r.B, r.N, ffn_gate=True)
+    r.ws = lib.Workspace(lib.dllm_step_workspace_size(r.model.cfg, r.B, r.N, r.pol))
+    return r
+
+
+def _gated_forced(lib, shape, tau, tol, steps):
+    r = _gated_run(lib, shape, tau)
+    L = r.ocfg.n_layers
+    for t in range(steps):
+        out = O.step(r.ocfg, r.ow, r.st, r.opol, dense=(t == 0))
+        rows = torch.full((L,), -1, dtype=torch.int32, device="cuda")
+        io = {"forced_unmask_pos": _pad(out.unmasked, out.unmasked.shape[1]), "ffn_rows_out": rows}
+        if t > 0:
+            io.update(forced_idx=_pad(out.idx, r.k_cap),
+                      forced_count=torch.tensor([len(a) for a in out.idx], dtype=torch.int32,
+                                                device="cuda"))
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, t == 0, r.ws, **io)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        assert rows.cpu().tolist() == out.ffn_rows
+        r.compare_state(tol, out.final_rows, out.idx)
+        for l in range(L):
+            assert max_abs_rel(f64(r.cache.ctx[l]), r.st.ctx[l]) < tol, ("ctx", l)
+            assert max_abs_rel(f64(r.cache.ffn[l]), r.st.ffn[l]) < tol, ("ffn", l)
+        r.tokens.copy_(torch.from_numpy(r.st.tokens.astype(np.int32)))
+    return r
+
+
+@pytest.mark.parametrize("tau", [-1.0, 2.5])
+def test_ffn_gate_tiny_f32_forced(lib, tau):
+    _gated_forced(lib, SY.with_(SY.TINY, n_layers=2), tau, TOL["f32"], 5)
+
+
+@pytest.mark.parametrize("tau", [-1.0, 2.5])
+def test_ffn_gate_bf16_forced(lib, tau):
+    _gated_forced(lib, _small_bf16(), tau, TOL["bf16"], 4)
+
+
+def test_ffn_gate_fixed_point_bf16(lib):
+    """After a dense step, a gated step over unchanged tokens finds every context
+    where it was (up to rounding), runs no FFN and reproduces the dense rows."""
+    shape = _small_bf16(n_unmask=0)
+    r = _gated_run(lib, shape, 1e-3)
+    lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, True, r.ws)
+    kv0 = [t.clone() for t in r.cache.k + r.cache.v]
+    rows = torch.full((r.ocfg.n_layers,), -1, dtype=torch.int32, device="cuda")
+    lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, False, r.ws, ffn_rows_out=rows)
+    torch.cuda.synchronize()
+    assert r.ws.device_status() == 0
+    assert rows.cpu().tolist() == [0] * r.ocfg.n_layers
+    for a, b in zip(kv0, r.cache.k + r.cache.v):
+        assert max_abs_rel(f64(b), f64(a)) < TOL["bf16"]
