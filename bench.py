@@ -323,6 +323,45 @@ def es_two_point_measure(S, model, shape, rank, steps, warmup):
             "device_status": st}
 
 
+def ffn_gate_measure(S, model, shape, rank, steps, warmup):
+    """DyLLM's FFN gate on the 8B workload: partial steps whose recomputed rows run a
+    layer's FFN only when their attention output moved (1 - cos > tau)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    tokens = rank_inputs(shape, rank)
+    cache = S.Cache(model.cfg, shape.batch, shape.seq_len, ffn_gate=True)
+    out = {}
+    for tau in (-1.0, 1e-3):
+        pol = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k, n_unmask=shape.n_unmask,
+                            gen_start=shape.prompt_len, block_len=shape.block_len,
+                            ffn_gate=True, ffn_tau=tau)
+        ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+        S.dllm_step_ex(model, cache, tokens, pol, True, ws)
+        for _ in range(warmup):
+            S.dllm_step_ex(model, cache, tokens, pol, False, ws)
+        rows = torch.zeros(shape.n_layers, dtype=torch.int32, device="cuda")
+        torch.cuda.synchronize()
+        K = min(steps, 10)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            S.dllm_step_ex(model, cache, tokens, pol, False, ws, stream=stream, ffn_rows_out=rows)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / K
+        frac = float(rows.float().mean().item()) / (shape.batch * shape.k)
+        out[f"tau_{tau:g}"] = {"ms_per_step": round(ms, 4),
+                               "tokens_per_s": round(shape.batch * shape.n_unmask * 1000.0 / ms, 2),
+                               "ffn_row_fraction_last_step": round(frac, 4),
+                               "device_status": ws.device_status()}
+        del ws
+    del cache
+    out["how"] = ("tau -1: every recomputed row is salient (the gate's own cost); tau 1e-3: "
+                  "rows whose attention output moved by more than 1e-3 (1 - cos) run the FFN; "
+                  "random-init weights, so the fraction says nothing about trained models")
+    return out
+
+
 def cpu_baseline_sample(W, cache, tokens, shape):
     """The oracle on one sequence, one layer and that sequence's LM-head rows,
     scaled to a full step: per step = 32 sequences x (32 layers x t_layer + t_lm)."""
@@ -511,6 +550,8 @@ def run_ours(args):
     if not args.layers and world == 1:
         result["es_two_point"] = es_two_point_measure(S, model, shape, rank, args.steps,
                                                       args.warmup)
+        result["dyllm_ffn_gate"] = ffn_gate_measure(S, model, shape, rank, args.steps,
+                                                    args.warmup)
     if not args.no_bs1 and not args.layers:
         del cache, ws
         torch.cuda.empty_cache()
