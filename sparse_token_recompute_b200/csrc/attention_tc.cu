@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   using L = Smem<HD>;
   constexpr int NB = HD / 64;  // 64-column boxes per row of Q/K/V
   constexpr float kLog2e = 1.4426950408889634f;
+  griddep_wait();  // everything below reads what earlier kernels wrote
   const int b = blockIdx.z, h = blockIdx.y;
   const int off = p.row_off[b];
   const int cnt = p.row_off[b + 1] - off;
@@ -581,8 +582,17 @@ cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensor
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  attn_tc_kernel<HD, UPD><<<grid, NTHREADS, smem, s>>>(q, k, v, k2, v2, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<HD, UPD>, q, k, v, k2, v2, p);
 }
 
 }  // namespace

@@ -586,15 +586,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // ---------------------------------------------------------------- host side
 
 // [rows, cols] bf16 row-major, box (64 cols, box_rows rows), 128-byte swizzle
-// programmatic dependent launch of the GEMMs; DLLM_PDL=0 turns it off (cross-check)
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("DLLM_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
 bool make_map(CUtensorMap* m, const void* ptr, int rows, int cols, int box_rows) {
   if (rows <= 0 || cols <= 0) return false;
   return tmap_bf16_2d(m, ptr, (uint64_t)rows, (uint64_t)cols, (uint32_t)box_rows);
@@ -649,6 +640,15 @@ cudaError_t launch_bn(int bn, const CUtensorMap& a, const CUtensorMap& b0, const
 }
 
 }  // namespace
+
+// programmatic dependent launch (GEMMs, norms, attention); DLLM_PDL=0 turns it off
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DLLM_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
 
 int gemm_total_cols(const GemmSpec& g) {
   int n = 0;

@@ -61,6 +61,10 @@ struct GemmSpec {
   int force_splits;  // 0: choose
 };
 
+// launch kernels with programmatic stream serialization (they griddepcontrol.wait
+// before reading what earlier kernels wrote); DLLM_PDL=0 turns it off
+bool pdl_enabled();
+
 struct GemmPlan {
   int bn, splits, tiles_n, m_tiles_cap, units_cap, grid;
 };

@@ -842,6 +842,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x,
                                                       const int* __restrict__ M_dev, int M_cap,
                                                       int d, float eps) {
   griddep_launch_dependents();  // the next GEMM may start streaming its weights
+  griddep_wait();               // x is written by the kernel before
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
   if (r >= M) return;
@@ -1338,7 +1339,16 @@ void launch_rmsnorm(const T* x, const T* g, T* out, const int* M_dev, int M_cap,
                     cudaStream_t s) {
   if (M_cap <= 0) return;
   ProfScope prof("rmsnorm", s);
-  rmsnorm_kernel<T><<<(M_cap + 7) / 8, 256, 0, s>>>(x, g, out, M_dev, M_cap, d, eps);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((M_cap + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  cudaLaunchKernelEx(&cfg, rmsnorm_kernel<T>, x, g, out, M_dev, M_cap, d, eps);
 }
 template void launch_rmsnorm<float>(const float*, const float*, float*, const int*, int, int,
                                     float, cudaStream_t);
