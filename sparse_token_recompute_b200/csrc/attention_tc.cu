@@ -27,6 +27,8 @@
 // block's outstanding copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -71,6 +73,7 @@ struct AttnParams {
   float* st_m;
   float* st_l;
   const int* a_off;  // update mode: changed keys of sequence b at rows a_off[b]..a_off[b+1]
+  int ppc;           // pairs of query tiles per CTA (consecutive; > 1 only without key splits)
 };
 
 // 32 columns without the trailing wait: several loads in flight before one wait
@@ -179,9 +182,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int b = blockIdx.z, h = blockIdx.y;
   const int off = p.row_off[b];
   const int cnt = p.row_off[b + 1] - off;
-  const int q0 = blockIdx.x * (NTILE * BT);
   griddep_launch_dependents();  // the next GEMM may start streaming its weights
-  if (q0 >= cnt) return;
+  // this CTA's pairs of query tiles: pair i starts at row pair_q0(i) of the sequence
+  // (several pairs per CTA only in the update mode, whose key streams are short)
+  constexpr bool multi = UPD;
+  const int ppc = UPD ? p.ppc : 1;
+  const int pair0 = blockIdx.x * ppc;
+  auto pair_q0 = [&](int i) { return (pair0 + i) * (NTILE * BT); };
+  const int npairs = UPD ? min(ppc, (cnt - pair_q0(0) + NTILE * BT - 1) / (NTILE * BT))
+                         : (pair_q0(0) < cnt ? 1 : 0);
+  if (npairs <= 0) return;
+  const int q0 = pair_q0(0);
   // update mode: a_cnt changed keys -> TH tiles of new values, then TH of old
   const int a_base = UPD ? p.a_off[b] : 0;
   const int a_cnt = UPD ? p.a_off[b + 1] - a_base : 0;
@@ -192,21 +203,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto tile_keys = [&](int t) {
     return UPD ? min(BKV, a_cnt - (t % TH) * BKV) : min(BKV, p.Nseq - t * BKV);
   };
-  const int nq = (cnt - q0 > BT) ? 2 : 1;  // query tiles holding rows in this CTA
-  // A lone query tile splits the keys instead: group A takes K/V tiles [0, TA),
-  // group B [TA, T), and the two partial softmax results are merged at the end.
-  const bool split = !UPD && nq == 1 && T >= 2;
+  auto pair_nq = [&](int i) { return (cnt - pair_q0(i) > BT) ? 2 : 1; };  // tiles with rows
+  const int nq = pair_nq(0);
+  // A lone query tile splits the keys instead (one pair per CTA only): group A
+  // takes K/V tiles [0, TA), group B [TA, T), and the two partial softmax
+  // results are merged at the end.
+  const bool split = !UPD && !multi && nq == 1 && T >= 2;
   const int TA = split ? (T + 1) / 2 : T;
   const int TB = split ? T - TA : T;
   const int ngroups = (nq == 2 || split) ? 2 : 1;
   auto ntiles = [&](int x) { return x == 0 ? TA : TB; };         // K/V tiles of group x
   auto kv_first = [&](int x) { return (split && x == 1) ? TA : 0; };
   auto qtile = [&](int x) { return split ? 0 : x; };             // query tile of group x
-  // softmax warps of group x that hold at least one selected row
-  auto live_warps = [&](int x) {
-    const int rows = min(BT, cnt - q0 - qtile(x) * BT);
+  // softmax warps of group x that hold at least one selected row in pair i
+  auto live_warps_in = [&](int i, int x) {
+    const int rows = min(BT, cnt - pair_q0(i) - qtile(x) * BT);
     return rows > 0 ? (rows + 31) / 32 : 1;
   };
+  auto live_warps = [&](int x) { return live_warps_in(0, x); };
   const int g = (h * p.Hkv) / p.Hq;
 
   extern __shared__ uint8_t smem_raw[];
@@ -214,9 +228,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                            ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR_OFF);
   float* stat = reinterpret_cast<float*>(sm + L::STAT_OFF);  // group B's (m, l) per row
-  // s_full[X], p_full[X], pv_done[X], q_full, drain, full[slot], empty[slot]
+  // s_full[X], p_full[X], pv_done[X], q_full, drain, full[slot], empty[slot],
+  // q_empty, o_free[X]
   constexpr int NS = L::SLOTS;
-  static_assert(NS >= 2 && 7 + 2 * NS + 1 <= 32, "barrier area holds 32 words");
+  static_assert(NS >= 2 && 11 + 2 * NS + 1 <= 32, "barrier area holds 32 words");
   auto s_full = [&](int x) { return smem_u32(&bars[0 + x]); };
   auto p_full = [&](int x) { return smem_u32(&bars[2 + x]); };
   auto pv_done = [&](int x) { return smem_u32(&bars[4 + x]); };
@@ -224,7 +239,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t drain_bar = smem_u32(&bars[7]);
   auto full = [&](int i) { return smem_u32(&bars[8 + i]); };
   auto empty = [&](int i) { return smem_u32(&bars[8 + NS + i]); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[8 + 2 * NS]);
+  const uint32_t q_empty = smem_u32(&bars[8 + 2 * NS]);  // Q tiles read (multi-pair)
+  auto o_free = [&](int x) { return smem_u32(&bars[9 + 2 * NS + x]); };  // O_X read out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(&bars[11 + 2 * NS]);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -245,9 +262,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(p_full(i), 32 * live_warps(i));
+      // one pair: the warps with rows; several: every warp of the group, every pair
+      mbar_init(p_full(i), multi ? 128 : 32 * live_warps(i));
       mbar_init(pv_done(i), 1);
+      mbar_init(o_free(i), 128);
     }
+    mbar_init(q_empty, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -294,19 +314,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++n;
         return true;
       };
-      mbar_arrive_expect_tx(q_full, nq * L::Q_TILE);
-      for (int x = 0; x < nq; ++x)
-        for (int c = 0; c < NB; ++c)
-          tma_load_2d(sQ + x * L::Q_TILE + c * BT * 128, &tmQ, q_full, h * HD + c * 64,
-                      off + q0 + x * BT);
-      bool ok;
+      bool ok = true;
+      int q_issued = 0;  // pairs whose Q tiles were requested
       if (!split) {
-        ok = load(false, 0);
-        for (int j = 0; j < T && ok; ++j) {
-          ok = load(true, j);
-          if (ok && j + 1 < T) ok = load(false, j + 1);
+        for (int i = 0; i < npairs && ok; ++i) {
+          // the previous pair's Q tiles stay until its last Q.K^T has run
+          if (i > 0 && !(ok = mbar_wait(q_empty, (i - 1) & 1, abort_flag, p.status))) break;
+          const int nqi = pair_nq(i);
+          mbar_arrive_expect_tx(q_full, nqi * L::Q_TILE);
+          for (int x = 0; x < nqi; ++x)
+            for (int c = 0; c < NB; ++c)
+              tma_load_2d(sQ + x * L::Q_TILE + c * BT * 128, &tmQ, q_full, h * HD + c * 64,
+                          off + pair_q0(i) + x * BT);
+          ++q_issued;
+          ok = load(false, 0);
+          for (int j = 0; j < T && ok; ++j) {
+            ok = load(true, j);
+            if (ok && j + 1 < T) ok = load(false, j + 1);
+          }
         }
       } else {
+        mbar_arrive_expect_tx(q_full, nq * L::Q_TILE);
+        for (int c = 0; c < NB; ++c)
+          tma_load_2d(sQ + c * BT * 128, &tmQ, q_full, h * HD + c * 64, off + q0);
+        q_issued = 1;
         ok = load(false, 0) && load(false, TA);
         for (int j = 0; j < TA && ok; ++j) {
           ok = load(true, j);
@@ -316,7 +347,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (!ok) {
-        wait_drain(q_full, 0);
+        if (q_issued > 0) wait_drain(q_full, (q_issued - 1) & 1);
         for (int sl = 0; sl < NS; ++sl)
           if (issued & (1u << sl)) wait_drain(full(sl), (issue_par >> sl) & 1u);
       }
@@ -326,9 +357,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_qk = umma_idesc_bf16(BT, BKV);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(BT, HD) | (1u << 16);  // B (V) MN-major
-      bool ok = mbar_wait(q_full, 0, abort_flag, p.status);
+      bool ok = true;
       bool any = false;
       int m = 0;  // ring tiles consumed
+      int jx[2] = {0, 0};  // K/V tiles group x has been through (barrier phases)
+      int px[2] = {0, 0};  // pairs group x has finished
       auto take = [&]() -> int {  // slot of the next ring tile, once it has landed
         const int sl = slot_of(m);
         if (!mbar_wait(full(sl), use_par(m), abort_flag, p.status)) return -1;
@@ -350,7 +383,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         any = true;
       };
       auto pv = [&](int x, int j, int sl) -> bool {
-        if (!mbar_wait(p_full(x), j & 1, abort_flag, p.status)) return false;
+        // a later pair's first P.V overwrites O_X: the group must have read it out
+        if (j == 0 && px[x] > 0 &&
+            !mbar_wait(o_free(x), (px[x] - 1) & 1, abort_flag, p.status))
+          return false;
+        if (!mbar_wait(p_full(x), jx[x] & 1, abort_flag, p.status)) return false;
+        ++jx[x];
         tc_fence_after();
         const uint32_t vb = sRing + sl * L::KV_BYTES;
 #pragma unroll
@@ -358,32 +396,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const uint64_t db = umma_desc_mn_sw128(vb + kk * 2048, BKV * 128);
           tc_mma_ts(tO(x), tS(x) + (uint32_t)(kk * 8), db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        if (j == ntiles(x) - 1) tc_commit(pv_done(x));  // single phase: O_X is final
+        if (j == ntiles(x) - 1) {  // O_X of this pair is final
+          tc_commit(pv_done(x));
+          ++px[x];
+        }
         return true;
       };
-      if (ok && !split) {
-        const int sk = take();
-        ok = sk >= 0;
-        if (ok) {
-          for (int x = 0; x < nq; ++x) qk(x, sk);
+      if (!split) {
+        for (int i = 0; i < npairs && ok; ++i) {
+          if (!(ok = mbar_wait(q_full, i & 1, abort_flag, p.status))) break;
+          const int nqi = pair_nq(i);
+          const int sk = take();
+          if (!(ok = sk >= 0)) break;
+          for (int x = 0; x < nqi; ++x) qk(x, sk);
           give(sk);
-        }
-        for (int j = 0; j < T && ok; ++j) {
-          const int sv = take();
-          if (!(ok = sv >= 0 && pv(0, j, sv))) break;
-          int sk1 = -1;
-          if (j + 1 < T) {
-            if (!(ok = (sk1 = take()) >= 0)) break;
-            qk(0, sk1);
+          for (int j = 0; j < T && ok; ++j) {
+            const int sv = take();
+            if (!(ok = sv >= 0 && pv(0, j, sv))) break;
+            int sk1 = -1;
+            if (j + 1 < T) {
+              if (!(ok = (sk1 = take()) >= 0)) break;
+              qk(0, sk1);
+            }
+            if (nqi == 2) {
+              if (!(ok = pv(1, j, sv))) break;
+              if (sk1 >= 0) qk(1, sk1);
+            }
+            give(sv);
+            if (sk1 >= 0) give(sk1);
           }
-          if (nq == 2) {
-            if (!(ok = pv(1, j, sv))) break;
-            if (sk1 >= 0) qk(1, sk1);
-          }
-          give(sv);
-          if (sk1 >= 0) give(sk1);
+          if (ok) tc_commit(q_empty);  // every Q.K^T of the pair is issued
         }
-      } else if (ok) {
+      } else if ((ok = mbar_wait(q_full, 0, abort_flag, p.status))) {
         for (int x = 0; x < 2 && ok; ++x) {
           const int sk = take();
           if ((ok = sk >= 0)) {
@@ -422,18 +466,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;       // query row in the tile (= TMEM lane)
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    // a warp whose 32 rows are all past the sequence's selected rows takes no part
-    if (x < ngroups && quad < live_warps(x)) {
+    int jcnt = 0, pcnt = 0;  // this group's K/V tiles and pairs so far (barrier phases)
+    for (int pi = 0; pi < npairs; ++pi) {
+      if (x >= (multi ? pair_nq(pi) : ngroups)) continue;
+      const bool live = quad < (multi ? live_warps_in(pi, x) : live_warps(x));
+      // one pair: a warp whose 32 rows are all past the sequence's rows takes no part;
+      // several pairs: it keeps the barrier counts (waits for each S tile, arrives)
+      if (!multi && !live) continue;
       const float sc = p.scale_log2;
       float m_ref = -INFINITY, lsum = 0.f;  // reference maximum in the exp2 domain
-      const int row_x = q0 + qtile(x) * BT + r;  // this thread's row in the sequence
+      const int row_x = pair_q0(pi) + qtile(x) * BT + r;  // this thread's row in the sequence
       const size_t st_i = (size_t)(off + row_x) * p.Hq + h;
       if (UPD) m_ref = row_x < cnt ? p.st_m[st_i] * kLog2e : 0.f;  // the cached maximum
       bool ok = true;
       const int nj = ntiles(x);
       for (int j = 0; j < nj; ++j) {
-        ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), j & 1, abort_flag, p.status));
+        ok = __all_sync(0xffffffffu, mbar_wait(s_full(x), jcnt & 1, abort_flag, p.status));
+        ++jcnt;
         if (!ok) break;
+        if (!live) {  // rows past the sequence: keep the count of P arrivals only
+          mbar_arrive(p_full(x));
+          continue;
+        }
         tc_fence_after();
         float s[BKV];
 #pragma unroll
@@ -500,7 +554,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tc_fence_before();
         mbar_arrive(p_full(x));
       }
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(pv_done(x), 0, abort_flag, p.status));
+      if (ok && live)
+        ok = __all_sync(0xffffffffu, mbar_wait(pv_done(x), pcnt & 1, abort_flag, p.status));
+      ++pcnt;
       if (split) {
         // group B hands its (m, l) to group A, which merges O_B into O_A
         if (x == 1) {
@@ -511,7 +567,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         named_bar_sync(1, 2 * 32 * live_warps(0));
         tc_fence_after();
       }
-      if (ok && (x == 0 || !split)) {
+      if (ok && live && (x == 0 || !split)) {
         const int row = row_x;
         float wa = 1.f, wb = 0.f, m_out = m_ref, w_old = 0.f;
         if (split) {
@@ -559,6 +615,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           p.st_l[st_i] = lsum;
         }
       }
+      if (multi) {  // O_X has been read out: the next pair's first P.V may overwrite it
+        tc_fence_before();
+        mbar_arrive(o_free(x));
+      }
+      if (!ok) break;
     }
   }
 
@@ -610,11 +671,21 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
   if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
     return cudaErrorInvalidValue;
   AttnParams p{row_off, o,      Nseq, Hq,      Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
-               status,  st_m,   st_l, nullptr};
+               status,  st_m,   st_l, nullptr, 1};
   dim3 grid((k_cap + NTILE * BT - 1) / (NTILE * BT), Hq, B);
   ProfScope prof("attention", s);
   return hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
                    : launch_hd<64, false>(tq, tk, tv, tk, tv, p, grid, s);
+}
+
+int num_sms_cached() {
+  static int n = [] {
+    int dev = 0, v = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    return v;
+  }();
+  return n;
 }
 
 cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bfloat16* o,
@@ -633,9 +704,14 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
       !tmap_bf16_2d(&tk2, k_old, (uint64_t)A_cap, cols, BKV) ||
       !tmap_bf16_2d(&tv2, v_old, (uint64_t)A_cap, cols, BKV))
     return cudaErrorInvalidValue;
-  AttnParams p{r_off, o,    0,    Hq,   Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
-               status, st_m, st_l, a_off};
-  dim3 grid((r_cap + NTILE * BT - 1) / (NTILE * BT), Hq, B);
+  // few changed keys make short key streams: a CTA takes several pairs of query
+  // tiles of its (sequence, head) in turn, keeping about two CTAs per SM in flight
+  const int pairs = (r_cap + NTILE * BT - 1) / (NTILE * BT);
+  const int min_x = std::max(1, (2 * num_sms_cached() + B * Hq - 1) / (B * Hq));
+  const int ppc = std::max(1, (pairs + min_x - 1) / min_x);
+  AttnParams p{r_off, o,    0,    Hq,   Hkv,   Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
+               status, st_m, st_l, a_off, ppc};
+  dim3 grid((pairs + ppc - 1) / ppc, Hq, B);
   ProfScope prof("attention_update", s);
   return hd == 128 ? launch_hd<128, true>(tq, tk, tv, tk2, tv2, p, grid, s)
                    : launch_hd<64, true>(tq, tk, tv, tk2, tv2, p, grid, s);

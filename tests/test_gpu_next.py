@@ -223,12 +223,9 @@ def _lse(m, l):
     return np.asarray(m, dtype=np.float64) + np.log(np.asarray(l, dtype=np.float64))
 
 
-@pytest.mark.parametrize("Hq,Hkv,hd", [(4, 2, 128), (2, 2, 64)])
-def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
+def _update_case(lib, Hq, Hkv, hd, N, r_count, a_count, r_cap, a_cap):
     g = torch.Generator().manual_seed(31)
-    B, N, r_cap, a_cap = 3, 300, 150, 40
-    r_count = [150, 70, 33]
-    a_count = [40, 7, 0]          # the last sequence has no changed key
+    B = len(r_count)
     kc = SY.normal((B, N, Hkv, hd), 1.0, 41, "cuda", "bf16")
     vc = SY.normal((B, N, Hkv, hd), 1.0, 42, "cuda", "bf16")
     q = SY.normal((B * r_cap, Hq * hd), 1.0, 43, "cuda", "bf16")
@@ -241,6 +238,8 @@ def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
     # statistics of the exact attention: the same log-sum-exp as the oracle's
     off = 0
     for b, c in enumerate(r_count):
+        if c == 0:
+            continue
         qb = f64(q[off:off + c]).reshape(c, Hq, hd)
         om, ol, oo = O.attention_stats(qb, f64(kc[b]), f64(vc[b]))
         assert np.max(np.abs(_lse(m[off:off + c].cpu(), l[off:off + c].cpu()) - _lse(om, ol))) < 2e-2
@@ -268,6 +267,8 @@ def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
     off = 0
     for b, c in enumerate(r_count):
         sl = slice(off, off + c)
+        if c == 0:
+            continue
         if a_count[b] == 0:
             assert torch.equal(o[sl], o_before[sl]) and torch.equal(m[sl], m_before[sl])
             assert torch.equal(l[sl], l_before[sl])
@@ -277,6 +278,19 @@ def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
             assert max_abs_rel(f64(o[sl]), O.store(eo, "bf16").reshape(c, -1)) < TOL["bf16"]
             assert np.max(np.abs(_lse(m[sl].cpu(), l[sl].cpu()) - _lse(em, el))) < 2e-2
         off += c
+
+
+@pytest.mark.parametrize("Hq,Hkv,hd", [(4, 2, 128), (2, 2, 64)])
+def test_attention_stats_and_update_match_oracle(lib, Hq, Hkv, hd):
+    # the last sequence has no changed key
+    _update_case(lib, Hq, Hkv, hd, 300, [150, 70, 33], [40, 7, 0], 150, 40)
+
+
+def test_attention_update_several_pairs_per_cta(lib):
+    """Enough sequences x heads that a CTA walks two pairs of query tiles, the
+    last pair of a sequence holding one tile (or none)."""
+    _update_case(lib, 32, 8, 64, 300, [600, 300, 257, 1, 0, 520, 88, 513],
+                 [40, 7, 0, 13, 3, 128, 129, 1], 600, 129)
 
 
 # ----------------------------------------------------------------- FFN gate
