@@ -775,6 +775,46 @@ __device__ __forceinline__ void rmsnorm_row(const T* __restrict__ x, const T* __
                                             T* __restrict__ o, int d, float eps) {
   const int lane = threadIdx.x & 31;
   float ss = 0.f;
+  if constexpr (sizeof(T) == 2) {
+    if (d <= 256 * 16) {
+      // bf16: the row and the gains stay packed in registers (16 + 16 vectors of 8
+      // per lane); every load of both is issued before the first use, so a row
+      // costs one memory round trip
+      uint4 xr[16], gr[16];
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        const int i = lane * 8 + v * 256;
+        if (i < d) {
+          xr[v] = __ldg(reinterpret_cast<const uint4*>(x + i));
+          gr[v] = __ldg(reinterpret_cast<const uint4*>(g + i));
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        if (lane * 8 + v * 256 < d) {
+          float f[8];
+          unpack8(xr[v], f);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+        }
+      }
+      ss = warp_sum(ss);
+      const float s = rsqrtf(ss / (float)d + eps);
+#pragma unroll
+      for (int v = 0; v < 16; ++v) {
+        const int i = lane * 8 + v * 256;
+        if (i < d) {
+          float f[8], w[8];
+          unpack8(xr[v], f);
+          unpack8(gr[v], w);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = f[j] * s * w[j];
+          *reinterpret_cast<uint4*>(o + i) = pack8(f);
+        }
+      }
+      return;
+    }
+  }
   if (d <= 256 * 16) {
     // whole row in registers (up to 16 vectors of 8 per lane): every load is
     // issued before the first use, then the row is normalised from registers
