@@ -207,6 +207,8 @@ struct LayerWs {
   float* vraw;
   float* graw;
   float* uraw;
+  float* part;  // partial outputs of the key-split attention
+  size_t part_bytes;
 };
 
 // scratch of a layer pass over up to `cap` compact rows
@@ -222,6 +224,12 @@ void layout_layer(Bump& bp, const dllm_model_cfg* c, int B, int N, int cap, Laye
   w.o = bp.take<char>((size_t)cap * q * es);
   w.act = bp.take<char>((size_t)cap * c->ffn * es);
   w.qraw = w.kraw = w.vraw = w.graw = w.uraw = nullptr;
+  w.part = nullptr;
+  w.part_bytes = 0;
+  if (c->dtype == DLLM_BF16) {
+    w.part_bytes = attention_part_bytes_bound(cap, c->n_heads, c->head_dim);
+    w.part = bp.take<float>(w.part_bytes / sizeof(float));
+  }
   if (c->dtype == DLLM_F32) {
     w.qraw = bp.take<float>((size_t)cap * q);
     w.kraw = bp.take<float>((size_t)cap * kv);
@@ -303,7 +311,8 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
                                    static_cast<const bf*>(k_cache),
                                    static_cast<const bf*>(v_cache), static_cast<bf*>(w.o),
                                    w.row_off, B, k_cap, N, c->n_heads, c->n_kv_heads, hd,
-                                   w.status, s) != cudaSuccess) {
+                                   w.status, s, nullptr, nullptr, w.part,
+                                   w.part_bytes) != cudaSuccess) {
       return DLLM_ERR_CUDA;
     }
     GemmSpec go = g;

@@ -74,6 +74,12 @@ struct AttnParams {
   float* st_l;
   const int* a_off;  // update mode: changed keys of sequence b at rows a_off[b]..a_off[b+1]
   int ppc;           // pairs of query tiles per CTA (consecutive; > 1 only without key splits)
+  // keys split over kv_split CTAs per pair (exact mode, few query tiles): each
+  // writes its normalised partial output and (m, l) for a merge kernel
+  int kv_split;
+  int part_rows;     // row capacity of the partial buffers
+  float* part_o;     // [kv_split, part_rows, Hq, HD]
+  float* part_ml;    // [kv_split, part_rows, Hq, 2] (m in the exp2 domain, l)
 };
 
 // 32 columns without the trailing wait: several loads in flight before one wait
@@ -187,7 +193,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // (several pairs per CTA only in the update mode, whose key streams are short)
   constexpr bool multi = UPD;
   const int ppc = UPD ? p.ppc : 1;
-  const int pair0 = blockIdx.x * ppc;
+  const int S_kv = UPD ? 1 : p.kv_split;           // CTAs sharing a pair's keys
+  const int s_kv = UPD ? 0 : (int)blockIdx.x % S_kv;  // this CTA's share
+  const int pair0 = (UPD ? blockIdx.x : blockIdx.x / S_kv) * ppc;
   auto pair_q0 = [&](int i) { return (pair0 + i) * (NTILE * BT); };
   const int npairs = UPD ? min(ppc, (cnt - pair_q0(0) + NTILE * BT - 1) / (NTILE * BT))
                          : (pair_q0(0) < cnt ? 1 : 0);
@@ -197,11 +205,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int a_base = UPD ? p.a_off[b] : 0;
   const int a_cnt = UPD ? p.a_off[b + 1] - a_base : 0;
   const int TH = UPD ? (a_cnt + BKV - 1) / BKV : 0;
-  const int T = UPD ? 2 * TH : (p.Nseq + BKV - 1) / BKV;
+  // exact mode: this CTA's K/V tiles [k_lo, k_lo + T) of the sequence's T_all
+  const int T_all = (p.Nseq + BKV - 1) / BKV;
+  const int TS = (T_all + S_kv - 1) / S_kv;
+  const int k_lo = UPD ? 0 : s_kv * TS;
+  const int T = UPD ? 2 * TH : max(0, min(T_all, k_lo + TS) - k_lo);
   if (T == 0) return;  // no changed key: the cached statistics stand
   // keys of K/V tile t that exist (the rest score -inf)
   auto tile_keys = [&](int t) {
-    return UPD ? min(BKV, a_cnt - (t % TH) * BKV) : min(BKV, p.Nseq - t * BKV);
+    return UPD ? min(BKV, a_cnt - (t % TH) * BKV) : min(BKV, p.Nseq - (k_lo + t) * BKV);
   };
   auto pair_nq = [&](int i) { return (cnt - pair_q0(i) > BT) ? 2 : 1; };  // tiles with rows
   const int nq = pair_nq(0);
@@ -305,7 +317,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_arrive_expect_tx(full(sl), L::KV_BYTES);
         const bool old = UPD && tile >= TH;
         const CUtensorMap* tm = is_v ? (old ? &tmV2 : &tmV) : (old ? &tmK2 : &tmK);
-        const int row = UPD ? a_base + (tile - (old ? TH : 0)) * BKV : krow0 + tile * BKV;
+        const int row = UPD ? a_base + (tile - (old ? TH : 0)) * BKV : krow0 + (k_lo + tile) * BKV;
         for (int c = 0; c < NB; ++c)
           tma_load_2d(sRing + sl * L::KV_BYTES + c * BKV * 128, tm, full(sl), g * HD + c * 64,
                       row);
@@ -587,13 +599,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         wa *= inv;
         wb *= inv;
         w_old *= inv;
+        const bool partial = !UPD && S_kv > 1;  // a share of the keys: fp32 partial out
 #pragma unroll 1
         for (int c = 0; c < HD; c += 32) {
           float o[32], ob[32];
           tmem_ld32_nowait(tO(x) + lane_off + c, o);
           if (split) tmem_ld32_nowait(tO(1) + lane_off + c, ob);
           tmem_wait_ld();
-          if (row < cnt) {
+          if (row < cnt && partial) {
+            float* dst = p.part_o + (((size_t)s_kv * p.part_rows + off + row) * p.Hq + h) * HD + c;
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *reinterpret_cast<float4*>(dst + i) =
+                  split ? make_float4(o[i] * wa + ob[i] * wb, o[i + 1] * wa + ob[i + 1] * wb,
+                                      o[i + 2] * wa + ob[i + 2] * wb, o[i + 3] * wa + ob[i + 3] * wb)
+                        : make_float4(o[i] * wa, o[i + 1] * wa, o[i + 2] * wa, o[i + 3] * wa);
+          } else if (row < cnt) {
             __nv_bfloat16* dst = p.O + (size_t)(off + row) * p.ldo + h * HD + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 8) {
@@ -610,7 +631,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        if (row < cnt && p.st_m) {
+        if (row < cnt && partial) {
+          float* ml = p.part_ml + (((size_t)s_kv * p.part_rows + off + row) * p.Hq + h) * 2;
+          ml[0] = m_out;
+          ml[1] = lsum;
+        } else if (row < cnt && p.st_m) {
           p.st_m[st_i] = m_out / kLog2e;
           p.st_l[st_i] = lsum;
         }
@@ -628,6 +653,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Merge of the key shares of the split exact attention: one warp per (row,
+// head): M = max m_s, w_s = l_s 2^(m_s - M), O = sum w_s o_s / sum w_s (o_s are
+// the shares' normalised outputs), in share order.
+template <int HD>
+__global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict__ part_o,
+                                                         const float* __restrict__ part_ml,
+                                                         int S, int part_rows,
+                                                         const int* __restrict__ M_dev, int Hq,
+                                                         __nv_bfloat16* __restrict__ O, int ldo,
+                                                         float* __restrict__ st_m,
+                                                         float* __restrict__ st_l) {
+  constexpr int PER = HD / 32;  // floats per lane
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int h = blockIdx.y, lane = threadIdx.x & 31;
+  if (r >= min(*M_dev, part_rows)) return;
+  float mx = -INFINITY;
+  for (int sh = 0; sh < S; ++sh)
+    mx = fmaxf(mx, part_ml[(((size_t)sh * part_rows + r) * Hq + h) * 2]);
+  float acc[PER], L = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+  for (int sh = 0; sh < S; ++sh) {
+    const size_t base = ((size_t)sh * part_rows + r) * Hq + h;
+    const float w = part_ml[base * 2 + 1] * ex2_approx(part_ml[base * 2] - mx);
+    L += w;
+    const float* src = part_o + base * HD + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, src[i], acc[i]);
+  }
+  const float inv = 1.0f / L;
+  __nv_bfloat16* dst = O + (size_t)r * ldo + h * HD + lane * PER;
+#pragma unroll
+  for (int i = 0; i < PER; i += 2) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(acc[i] * inv, acc[i + 1] * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dst + i) = t;
+  }
+  if (st_m && lane == 0) {
+    st_m[(size_t)r * Hq + h] = mx / 1.4426950408889634f;
+    st_l[(size_t)r * Hq + h] = L;
   }
 }
 
@@ -658,26 +725,6 @@ cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensor
 
 }  // namespace
 
-cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
-                                const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
-                                int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
-                                cudaStream_t s, float* st_m, float* st_l) {
-  if (B <= 0 || k_cap <= 0 || M_cap <= 0) return cudaSuccess;
-  if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
-  CUtensorMap tq, tk, tv;
-  if (!tmap_bf16_2d(&tq, q, (uint64_t)M_cap, (uint64_t)Hq * hd, BT)) return cudaErrorInvalidValue;
-  if (!tmap_bf16_2d(&tk, kc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
-    return cudaErrorInvalidValue;
-  if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
-    return cudaErrorInvalidValue;
-  AttnParams p{row_off, o,      Nseq, Hq,      Hkv, Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
-               status,  st_m,   st_l, nullptr, 1};
-  dim3 grid((k_cap + NTILE * BT - 1) / (NTILE * BT), Hq, B);
-  ProfScope prof("attention", s);
-  return hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
-                   : launch_hd<64, false>(tq, tk, tv, tk, tv, p, grid, s);
-}
-
 int num_sms_cached() {
   static int n = [] {
     int dev = 0, v = 148;
@@ -686,6 +733,62 @@ int num_sms_cached() {
     return v;
   }();
   return n;
+}
+
+int attention_kv_split(int B, int k_cap, int Nseq, int Hq) {
+  // few (sequence, head, pair) CTAs leave most SMs idle: share each pair's keys
+  // among up to 8 CTAs, at least two K/V tiles each
+  const int T = (Nseq + BKV - 1) / BKV;
+  const int ctas = ((k_cap + NTILE * BT - 1) / (NTILE * BT)) * Hq * B;
+  if (ctas <= 0 || 2 * ctas > num_sms_cached() || T < 4) return 1;
+  int S = std::max(1, std::min(std::min(8, T / 2), num_sms_cached() / ctas));
+  while (S > 1 && (S - 1) * ((T + S - 1) / S) >= T) --S;  // every share holds keys
+  return S;
+}
+
+size_t attention_part_bytes_bound(int cap, int Hq, int hd) {
+  // a split launch has S * rows <= SMs * (rows of a pair) for any batch shape
+  const size_t rows = std::min((size_t)8 * cap * Hq, (size_t)num_sms_cached() * NTILE * BT);
+  return rows * (hd + 2) * sizeof(float);
+}
+
+size_t attention_part_bytes(int S, int M_cap, int Hq, int hd) {
+  return S > 1 ? (size_t)S * M_cap * Hq * (hd + 2) * sizeof(float) : 0;
+}
+
+cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
+                                const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
+                                int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
+                                cudaStream_t s, float* st_m, float* st_l, float* part,
+                                size_t part_bytes) {
+  if (B <= 0 || k_cap <= 0 || M_cap <= 0) return cudaSuccess;
+  if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
+  CUtensorMap tq, tk, tv;
+  if (!tmap_bf16_2d(&tq, q, (uint64_t)M_cap, (uint64_t)Hq * hd, BT)) return cudaErrorInvalidValue;
+  if (!tmap_bf16_2d(&tk, kc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
+    return cudaErrorInvalidValue;
+  if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
+    return cudaErrorInvalidValue;
+  int S = part ? attention_kv_split(B, k_cap, Nseq, Hq) : 1;
+  if (S > 1 && attention_part_bytes(S, M_cap, Hq, hd) > part_bytes) S = 1;
+  float* part_o = S > 1 ? part : nullptr;
+  float* part_ml = S > 1 ? part + (size_t)S * M_cap * Hq * hd : nullptr;
+  AttnParams p{row_off, o,      Nseq, Hq,      Hkv,    Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
+               status,  st_m,   st_l, nullptr, 1,      S,       M_cap,
+               part_o,  part_ml};
+  dim3 grid(((k_cap + NTILE * BT - 1) / (NTILE * BT)) * S, Hq, B);
+  ProfScope prof("attention", s);
+  cudaError_t e = hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
+                            : launch_hd<64, false>(tq, tk, tv, tk, tv, p, grid, s);
+  if (e != cudaSuccess || S == 1) return e;
+  dim3 mgrid((M_cap + 7) / 8, Hq);
+  if (hd == 128)
+    attn_merge_kernel<128><<<mgrid, 256, 0, s>>>(part_o, part_ml, S, M_cap, row_off + B, Hq, o,
+                                                 Hq * hd, st_m, st_l);
+  else
+    attn_merge_kernel<64><<<mgrid, 256, 0, s>>>(part_o, part_ml, S, M_cap, row_off + B, Hq, o,
+                                                Hq * hd, st_m, st_l);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bfloat16* o,
@@ -710,7 +813,8 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
   const int min_x = std::max(1, (2 * num_sms_cached() + B * Hq - 1) / (B * Hq));
   const int ppc = std::max(1, (pairs + min_x - 1) / min_x);
   AttnParams p{r_off, o,    0,    Hq,   Hkv,   Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
-               status, st_m, st_l, a_off, ppc};
+               status, st_m, st_l, a_off, ppc,   1,       0,
+               nullptr, nullptr};
   dim3 grid((pairs + ppc - 1) / ppc, Hq, B);
   ProfScope prof("attention_update", s);
   return hd == 128 ? launch_hd<128, true>(tq, tk, tv, tk2, tv2, p, grid, s)

@@ -124,7 +124,14 @@ void launch_confidence_rows_f32(const float* logits, int V, const int* lm_rows, 
 cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
                                 const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
                                 int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
-                                cudaStream_t s, float* st_m = nullptr, float* st_l = nullptr);
+                                cudaStream_t s, float* st_m = nullptr, float* st_l = nullptr,
+                                float* part = nullptr, size_t part_bytes = 0);
+// key shares per pair of query tiles the attention uses for this shape (1: none), and
+// the partial-output scratch (fp32) that launch_attention_tc then needs in `part`
+int attention_kv_split(int B, int k_cap, int Nseq, int Hq);
+size_t attention_part_bytes(int S, int M_cap, int Hq, int hd);
+// scratch that covers the split of any launch over at most `cap` rows
+size_t attention_part_bytes_bound(int cap, int Hq, int hd);
 // incremental attention of stable rows: q [R_cap, Hq*hd] with cached o, st_m, st_l (in/out),
 // rows of sequence b at r_off[b].. (at most r_cap); changed keys' new and old K/V
 // [A_cap, Hkv*hd] compact, sequence b at rows a_off[b]..a_off[b+1]

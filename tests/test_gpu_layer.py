@@ -106,3 +106,14 @@ def test_layer_bf16_7b_gqa_shape(lib):
     shape = SY.with_(SY.GQA7B_B8_N2048, n_layers=1)
     _run_layer(lib, shape, B=2, N=2048, counts=[103, 250], k_cap=250, weights_on_gpu=True,
                check_seqs=[0, 1])
+
+
+@pytest.mark.parametrize("B,N,counts", [(1, 1000, [77]), (1, 1100, [300]), (1, 4096, [5]),
+                                        (2, 1536, [0, 40])])
+def test_layer_bf16_few_rows_split_keys(lib, B, N, counts):
+    """Few query rows over long sequences: the attention shares each sequence's
+    keys among several CTAs and merges their partial outputs; ragged key tails
+    (1000 and 1100 keys), an empty sequence and up to eight shares."""
+    shape = SY.with_(SY.TINY, dtype="bf16", d=512, n_heads=4, n_kv_heads=2, head_dim=128,
+                     ffn=1024, vocab=2048)
+    _run_layer(lib, shape, B=B, N=N, counts=counts, k_cap=max(counts))
