@@ -73,7 +73,7 @@ __device__ __forceinline__ void decode_unit(int u, int m_tiles, int tiles_n, int
                                             int& n, int& s) {
   s = u % splits;
   const int t = u / splits;
-  constexpr int G = 16;  // m-tiles per raster group: keeps A and B slices resident in L2
+  constexpr int G = 32;  // m-tiles per raster group: keeps A and B slices resident in L2
   const int per_group = G * tiles_n;
   const int g = t / per_group;
   const int first_m = g * G;
