@@ -117,3 +117,16 @@ def test_layer_bf16_few_rows_split_keys(lib, B, N, counts):
     shape = SY.with_(SY.TINY, dtype="bf16", d=512, n_heads=4, n_kv_heads=2, head_dim=128,
                      ffn=1024, vocab=2048)
     _run_layer(lib, shape, B=B, N=N, counts=counts, k_cap=max(counts))
+
+
+@pytest.mark.parametrize("heads,kv,hd", [(8, 8, 64), (8, 4, 128)])
+def test_layer_bf16_many_sequences_mixed_counts(lib, heads, kv, hd):
+    """A grid several waves deep (76 sequences): row counts cover a lone first
+    query tile, a lone remainder after two full tiles, full pairs, one row and
+    an empty sequence, for MHA and GQA."""
+    shape = SY.with_(SY.TINY, dtype="bf16", d=512, n_heads=heads, n_kv_heads=kv, head_dim=hd,
+                     ffn=1024, vocab=2048)
+    pattern = [300, 100, 0, 200, 129, 1, 256, 257]
+    counts = [pattern[i % len(pattern)] for i in range(76)]
+    _run_layer(lib, shape, B=76, N=384, counts=counts, k_cap=300,
+               check_seqs=[0, 1, 2, 3, 4, 5, 6, 7, 75])
