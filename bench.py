@@ -41,8 +41,8 @@ GQA = SY.GQA7B_B8_N2048
 # DRAM bytes (read + write) per launch of the layer-projection GEMM, averaged over
 # its four launches per layer (QKV, O, gate/up, down) at 32 x 308 rows of the 8B
 # layer, from the ncu capture summarised in
-# profiles/gemm_tc_8b_layer_b32_n1536_k308_dram.md; re-take it when gemm_tc changes.
-GEMM_TRAFFIC_PER_LAUNCH = 832.3e6
+# profiles/gemm_projections_8b_layer_b32_n1536_k308_dram.md; re-take it when either GEMM kernel changes.
+GEMM_TRAFFIC_PER_LAUNCH = 889.7e6
 
 
 def parse():
@@ -514,8 +514,9 @@ def run_ours(args):
                    "l2": "inputs larger than L2: ~16 GB weights + ~26 GB K/V caches per step"},
         "steps_per_s": round(1000.0 / ms_step, 3),
         "roofline": {
-            "kernel": "gemm_tc (tcgen05 layer projections: QKV+RoPE+KV scatter, O+residual, "
-                      "gate/up+SwiGLU, down+residual)",
+            "kernel": "gemm_pair_kernel / gemm_tc_kernel (tcgen05 layer projections: "
+                      "QKV+RoPE+KV scatter, O+residual and down+residual on CTA pairs, "
+                      "gate/up+SwiGLU on single CTAs)",
             "bound": "tensor", "achieved": round(achieved, 1) if achieved else None,
             "peak": tc_sus, "unit": "TFLOP/s",
             "frac": round(achieved / tc_sus, 4) if achieved else None,

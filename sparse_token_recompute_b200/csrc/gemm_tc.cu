@@ -17,7 +17,9 @@
 //   * weight-streaming shapes may split K across the CTAs of a thread-block
 //     cluster: each CTA stages its fp32 partial tile in shared memory and the
 //     cluster reduces it over distributed shared memory in split order, so
-//     the result does not depend on timing.
+//     the result does not depend on timing;
+//   * tensor-bound plain, residual and QKV GEMMs run on CTA pairs instead
+//     (gemm_pair_kernel: tcgen05 cta_group::2, 256 x 256 tiles).
 // No TMA multicast is used anywhere.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -66,14 +68,16 @@ struct Params {
   int V;
   int a_tx;  // bytes one A box delivers (fewer than a full 128-row tile when M_cap < 128)
   int prefetch_b;  // issue the first unit's weight tiles before waiting on the previous kernel
+  int raster_g;    // CTA-pair kernel: row-tile pairs per raster group
   int* status;
 };
 
+// G: m-tiles per raster group (the group's A rows stay in L2 while its CTAs sweep
+// every column tile)
 __device__ __forceinline__ void decode_unit(int u, int m_tiles, int tiles_n, int splits, int& m,
-                                            int& n, int& s) {
+                                            int& n, int& s, int G = 32) {
   s = u % splits;
   const int t = u / splits;
-  constexpr int G = 32;  // m-tiles per raster group: keeps A and B slices resident in L2
   const int per_group = G * tiles_n;
   const int g = t / per_group;
   const int first_m = g * G;
@@ -583,6 +587,313 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel
+// Tensor-bound shapes (>= 256 rows, 256-wide tiles, no K split): the two CTAs of
+// a cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2 issued by
+// CTA 0.  CTA r stages rows [128 r, 128 r + 128) of the A tile and columns
+// [128 r, 128 r + 128) of the B tile (32 KB per 64-deep k-block instead of
+// 48 KB, so the ring holds 7 k-blocks), and its TMEM receives its 128 rows of
+// the accumulator over all 256 columns.  Each CTA's TMA loads complete on its
+// own barriers; CTA 1's issuer thread forwards each landed stage to CTA 0
+// (remote mbarrier arrive), CTA 0's commits arrive on both CTAs' barriers
+// (multicast commit), and CTA 1's epilogue warps release accumulators to CTA 0
+// by remote arrive.  No TMA multicast.
+
+constexpr int PAIR_BN = 256;
+constexpr int PAIR_STAGES = 7;
+constexpr size_t PAIR_SMEM = (size_t)PAIR_STAGES * (BM * BK * 2 + (PAIR_BN / 2) * BK * 2) + 1024 + 256;
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+// D (+)= A * B^T over the CTA pair: M = 256 (128 rows per CTA), N = 256
+__device__ __forceinline__ void tc_mma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive on the barrier at this offset in both CTAs of the pair once the pair's
+// earlier tcgen05 ops issued by this thread complete
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+// the same, on this CTA's barrier only
+__device__ __forceinline__ void tc_commit_pair_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// arrive on a barrier of another CTA of the cluster (address from mapa).  The
+// cross-CTA barriers use the default (CTA-scope) semantics of arrive and
+// try_wait: the data they guard is read by the tensor core or by tcgen05.ld
+// after tcgen05 fences, not through the generic proxy.  Cluster-scope acquire in
+// the waits cost the pair ring about half its throughput (QKV shape 684 against
+// 1340 TFLOP/s).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmB1,
+                     const __grid_constant__ CUtensorMap tmB2, const Params p) {
+  constexpr int BN = PAIR_BN, BNH = PAIR_BN / 2, STAGES = PAIR_STAGES;
+  constexpr int A_BYTES = BM * BK * 2;
+  constexpr int B_BYTES = BNH * BK * 2;  // this CTA's half of the B tile
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr int EPI_WARPS = EPI_THREADS / 32;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  // bars: full[S], empty[S], pfull[S], tfull[2], tempty[2], drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 issues the MMAs, 1 is its peer
+  const int pair_id = (int)blockIdx.x >> 1;
+  const int n_pairs = (int)gridDim.x >> 1;
+
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+  auto pfull_bar = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };  // CTA 0: peer landed
+  auto tfull_bar = [&](int a) { return smem_u32(&bars[3 * STAGES + a]); };
+  auto tempty_bar = [&](int a) { return smem_u32(&bars[3 * STAGES + 2 + a]); };
+  const uint32_t drain_bar = smem_u32(&bars[3 * STAGES + 4]);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(pfull_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 2 * EPI_WARPS);  // the epilogue warps of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (EPI == EPI_SWIGLU || EPI == EPI_QKV) tma_prefetch_desc(&tmB1);
+    if (EPI == EPI_QKV) tma_prefetch_desc(&tmB2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  // both CTAs' barriers exist before either CTA signals the other's
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();
+
+  // this CTA's half (columns [n*BN + rank*BNH, +BNH)) of the B tile of k-block kb
+  auto load_b_half = [&](uint32_t b_dst, uint32_t bar, int kb, int n) {
+    if constexpr (EPI == EPI_SWIGLU) {
+      // gate columns come from CTA 0, the matching up columns from CTA 1
+      tma_load_2d(b_dst, rank == 0 ? &tmB0 : &tmB1, bar, kb * BK, n * BNH);
+    } else if constexpr (EPI == EPI_QKV) {
+      const int n0 = n * BN + (int)rank * BNH;  // segments are multiples of BN
+      if (n0 < p.seg0)
+        tma_load_2d(b_dst, &tmB0, bar, kb * BK, n0);
+      else if (n0 < p.seg1)
+        tma_load_2d(b_dst, &tmB1, bar, kb * BK, n0 - p.seg0);
+      else
+        tma_load_2d(b_dst, &tmB2, bar, kb * BK, n0 - p.seg1);
+    } else {
+      tma_load_2d(b_dst, &tmB0, bar, kb * BK, n * BN + (int)rank * BNH);
+    }
+  };
+
+  griddep_wait();
+  int M = p.M_cap;
+  if (p.M_dev) {
+    M = *p.M_dev;
+    if (M > p.M_cap || M < 0) {
+      if (threadIdx.x == 0 && blockIdx.x == 0) raise_status(p.status, DEV_BAD_SHAPE);
+      M = M < 0 ? 0 : p.M_cap;
+    }
+  }
+  const int m_pairs = (M + 2 * BM - 1) / (2 * BM);
+  const int n_units = m_pairs * p.tiles_n;
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issue_phase = 0;
+      bool ok = true;
+      for (int u = pair_id; u < n_units && ok; u += n_pairs) {
+        int mp, n, s;
+        decode_unit(u, m_pairs, p.tiles_n, 1, mp, n, s, p.raster_g);
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(A_BYTES + B_BYTES));
+          tma_load_2d(smem_u32(sA + stage * A_BYTES), &tmA, full_bar(stage), kb * BK,
+                      mp * 2 * BM + (int)rank * BM);
+          load_b_half(smem_u32(sB + stage * B_BYTES), full_bar(stage), kb, n);
+          issued |= 1u << stage;
+          if (phase) issue_phase |= 1u << stage; else issue_phase &= ~(1u << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (ok) {
+        // every stage's last release (a commit of CTA 0 arriving here) has landed
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait_drain(empty_bar(s), (issue_phase >> s) & 1u);
+      } else {
+        // every load this thread issued lands before the block exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (issue_phase >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 1) {
+      // ------------------------------------------------ CTA 1: forward landed stages
+      const uint32_t peer_pfull0 = mapa_rank(pfull_bar(0), 0u);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int u = pair_id; u < n_units && ok; u += n_pairs) {
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_remote(peer_pfull0 + (uint32_t)(stage * 8));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    } else if (lane == 0) {
+      // ------------------------------------------------ CTA 0: MMA issuer for the pair
+      constexpr uint32_t idesc = umma_idesc_bf16(2 * BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int u = pair_id; u < n_units && ok; u += n_pairs) {
+        if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < p.kb_total; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status) ||
+              !mbar_wait(pfull_bar(stage), phase, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_base = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_bf16_pair(d_tmem, umma_desc_k_sw128(a_base + k * 32),
+                             umma_desc_k_sw128(b_base + k * 32), idesc,
+                             (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit_pair_both(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_both(tfull_bar(acc));
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok && issued_any) {
+        tc_commit_pair_local(drain_bar);
+        mbar_wait_drain(drain_bar, 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+    const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad+32)
+    const int r_in_tile = quad * 32 + lane;
+    const uint32_t tempty0 = rank == 0 ? 0u : mapa_rank(tempty_bar(0), 0u);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = pair_id; u < n_units; u += n_pairs) {
+      int mp, n, s;
+      decode_unit(u, m_pairs, p.tiles_n, 1, mp, n, s, p.raster_g);
+      const bool ok = __all_sync(0xffffffffu,
+                                 mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      const int row = mp * 2 * BM + (int)rank * BM + r_in_tile;
+      const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * BN);
+      epilogue_tile<BN, EPI>(p, row, row < M, mp * 2 + (int)rank, n,
+                             [&](int c, float* v) { tmem_ld_32x32b_x32(t_row + c, v); });
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(tempty_bar(acc));
+        else
+          mbar_arrive_remote(tempty0 + (uint32_t)(acc * 8));
+      }
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  // neither CTA leaves (or frees TMEM) while the other may still signal it
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 
 // [rows, cols] bf16 row-major, box (64 cols, box_rows rows), 128-byte swizzle
@@ -630,6 +941,39 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 }
 
 template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                        const CUtensorMap& b2, const Params& p, int grid, cudaStream_t s) {
+  static bool attr_set = false;  // per template instance; device-wide attribute
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PAIR_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PAIR_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned na = 0;
+  attr[na].id = cudaLaunchAttributeClusterDimension;
+  attr[na].val.clusterDim.x = 2;
+  attr[na].val.clusterDim.y = 1;
+  attr[na].val.clusterDim.z = 1;
+  ++na;
+  if (pdl_enabled()) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, gemm_pair_kernel<EPI>, a, b0, b1, b2, p);
+}
+
+template <int EPI>
 cudaError_t launch_bn(int bn, const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                       const CUtensorMap& b2, const Params& p, int grid, cudaStream_t s) {
   switch (bn) {
@@ -645,6 +989,15 @@ cudaError_t launch_bn(int bn, const CUtensorMap& a, const CUtensorMap& b0, const
 bool pdl_enabled() {
   static const bool on = [] {
     const char* e = getenv("DLLM_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// CTA-pair GEMM for tensor-bound shapes; DLLM_GEMM_PAIR=0 keeps single-CTA tiles
+bool pair_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DLLM_GEMM_PAIR");
     return !(e && e[0] == '0');
   }();
   return on;
@@ -749,6 +1102,18 @@ GemmPlan gemm_plan(const GemmSpec& g) {
   pl.units_cap = pl.m_tiles_cap * pl.tiles_n * pl.splits;
   // split K runs one unit per CTA (clusters of `splits`); otherwise persistent CTAs
   pl.grid = splits > 1 ? pl.units_cap : std::max(1, std::min(pl.units_cap, sms));
+  // at least two row tiles, 256-wide tiles, no split: persistent CTA pairs, each
+  // pair one 256-row tile at a time.  Inside the power-capped 8B step (32 x 308
+  // rows) the pairs made the QKV GEMM 2% and the O/down GEMMs 3.5% faster, but
+  // the gate/up (SwiGLU) GEMM 5% and the LM head 9% slower (both read ~30% more
+  // DRAM), so those two keep single-CTA tiles.
+  pl.pair = (pair_enabled() && !weight_bound && splits == 1 && bn == PAIR_BN &&
+             pl.m_tiles_cap >= 2 && sms >= 2 && g.epi != EPI_SWIGLU && g.epi != EPI_LMHEAD)
+                ? 1 : 0;
+  if (pl.pair) {
+    const int units = ((pl.m_tiles_cap + 1) / 2) * pl.tiles_n;
+    pl.grid = 2 * std::max(1, std::min(units, sms / 2));
+  }
   return pl;
 }
 
@@ -788,8 +1153,11 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   const int a_rows = g.M_cap < BM ? ((g.M_cap + 15) / 16) * 16 : BM;
   p.a_tx = a_rows * BK * 2;
   p.prefetch_b = (g.M_cap <= BM && pdl_enabled()) ? 1 : 0;
+  // the A rows of a raster group (256 per pair) stay within ~32 MB of L2
+  p.raster_g = std::max(2, std::min(16, (int)((32u << 20) / ((size_t)2 * BM * g.K * 2))));
   if (!make_map(&ta, g.A, g.M_cap, g.K, a_rows)) return cudaErrorInvalidValue;
-  const int bbox = (g.epi == EPI_SWIGLU) ? pl.bn / 2 : pl.bn;
+  // a CTA pair stages half of each 256-wide B tile per CTA
+  const int bbox = (g.epi == EPI_SWIGLU || pl.pair) ? pl.bn / 2 : pl.bn;
   if (!make_map(&tb0, g.B[0], g.seg_cols[0], g.K, bbox)) return cudaErrorInvalidValue;
   tb1 = tb0;
   tb2 = tb0;
@@ -799,6 +1167,14 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   static const char* names[5] = {"gemm_store", "gemm_resid", "gemm_swiglu", "gemm_qkv",
                                  "gemm_lmhead"};
   ProfScope prof(names[g.epi], s);
+  if (pl.pair) {
+    switch (g.epi) {
+      case EPI_STORE: return launch_pair<EPI_STORE>(ta, tb0, tb1, tb2, p, pl.grid, s);
+      case EPI_RESID: return launch_pair<EPI_RESID>(ta, tb0, tb1, tb2, p, pl.grid, s);
+      case EPI_QKV: return launch_pair<EPI_QKV>(ta, tb0, tb1, tb2, p, pl.grid, s);
+      default: return cudaErrorInvalidValue;  // the planner pairs no other epilogue
+    }
+  }
   switch (g.epi) {
     case EPI_STORE: return launch_bn<EPI_STORE>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);
     case EPI_RESID: return launch_bn<EPI_RESID>(pl.bn, ta, tb0, tb1, tb2, p, pl.grid, s);

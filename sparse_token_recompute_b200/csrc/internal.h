@@ -67,6 +67,7 @@ bool pdl_enabled();
 
 struct GemmPlan {
   int bn, splits, tiles_n, m_tiles_cap, units_cap, grid;
+  int pair;  // CTA pairs (tcgen05 cta_group::2) computing 256-row tiles
 };
 
 int gemm_total_cols(const GemmSpec& g);

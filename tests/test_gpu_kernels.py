@@ -29,6 +29,8 @@ pytestmark = pytest.mark.gpu
     (500, 1024, 4096, 0, False),     # four row tiles, few column tiles
     (400, 4096, 12288, 0, True),     # four row tiles, deep K, residual accumulate
     (257, 8192, 1024, 0, False),     # three row tiles, the last one holding one row
+    (600, 1000, 512, 0, False),      # ragged last column tile
+    (384, 640, 200, 0, True),        # ragged K (a partial last k-block), 1.5 row-tile pairs
 ])
 def test_gemm_bf16(lib, M, N, K, splits, acc):
     A = SY.normal((M, K), 1.0, 11 + M, "cuda", "bf16")
