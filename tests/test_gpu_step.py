@@ -182,3 +182,18 @@ def test_step_full_ratio_equals_dense_step_on_gpu(lib):
                     r2.cache.k + r2.cache.v + [r2.cache.h_ref, r2.cache.conf, r2.cache.pred]):
         assert torch.equal(a, b)
     assert torch.equal(r1.tokens, r2.tokens)
+
+
+def test_step_8b_width_two_layers_forced(lib):
+    """The 8B step's launch configuration at full width (d 4096, 32 heads, FFN
+    12288, vocab 126464, 1536 tokens with 512 prompt, 308 rows and 16 reveals per
+    sequence per step) on 2 of its 32 sequences and 2 of its 32 layers: the
+    dense first step and two partial steps with the oracle's decisions; every
+    cache, the confidences and the predictions compared."""
+    shape = SY.with_(SY.DENSE8B_B32_N1536, n_layers=2, batch=2)
+    r = Run(lib, shape)
+    for t in range(3):
+        out = O.step(r.ocfg, r.ow, r.st, r.opol, dense=(t == 0))
+        r.gpu_step(t == 0, None if t == 0 else out.idx, out.unmasked)
+        r.compare_state(TOL["bf16"], out.final_rows, out.idx)
+        np.testing.assert_array_equal(f64(r.tokens).astype(np.int64), r.st.tokens)
