@@ -183,8 +183,33 @@ def time_steps(S, model, cache, tokens, pol, ws, K, stream):
     return e0.elapsed_time(e1)
 
 
-def bs1_measure(S, W, steps, warmup):
-    """Batch-1 8B step (768 tokens, blocks of 32, 8 revealed/step) at 10/25/50 %."""
+def step_roofline(shape, ms, hbm_gbs, tc_tflops):
+    """Whole-step roofline of a partial step: algorithmic bytes = every layer's
+    weights + the LM head + the K/V caches the attention reads + the K/V rows
+    written; flops = the layer projections and the attention of the selected rows
+    (the LM head's flops are left out: its row count is decided on the device).
+    The bound is the side of the ridge (peak flops / peak bytes) the step's
+    arithmetic intensity falls on."""
+    M = shape.batch * shape.k
+    d, q, kv, f = shape.d, shape.n_heads * shape.head_dim, shape.n_kv_heads * shape.head_dim, shape.ffn
+    p_layer = d * (q + 2 * kv) + q * d + 3 * d * f
+    L, e = shape.n_layers, 2
+    nbytes = (L * p_layer + shape.vocab * d) * e \
+        + L * shape.batch * shape.seq_len * 2 * kv * e + L * M * 2 * kv * e
+    flops = L * (2.0 * M * p_layer + 4.0 * M * shape.seq_len * q)
+    t = ms / 1000.0
+    ridge = tc_tflops * 1e12 / (hbm_gbs * 1e9)
+    return {"bound": "hbm" if flops / nbytes < ridge else "tensor",
+            "bytes": int(nbytes), "flops": flops,
+            "achieved_gbs": round(nbytes / t / 1e9, 1), "hbm_frac": round(nbytes / t / 1e9 / hbm_gbs, 4),
+            "achieved_tflops": round(flops / t / 1e12, 1),
+            "tensor_frac": round(flops / t / 1e12 / tc_tflops, 4),
+            "peaks": {"hbm_gbs": hbm_gbs, "bf16_tflops_burst": tc_tflops}}
+
+
+def bs1_measure(S, W, steps, warmup, hbm_gbs, tc_tflops):
+    """Batch-1 8B step (768 tokens, blocks of 32, 8 revealed/step) at 10/25/50/100 %,
+    each with its whole-step roofline (HBM-bound below the ridge)."""
     import torch
     out = {}
     model = S.Model(S.cfg_from_shape(BS1), W)
@@ -225,6 +250,7 @@ def bs1_measure(S, W, steps, warmup):
                                        "tokens_per_s": round(shape.n_unmask * 1000.0 / ms, 1),
                                        "ms_per_step_eager": round(ms_eager, 4),
                                        "ms_per_step_eager_profiled": round(ms_prof, 4),
+                                       "roofline": step_roofline(shape, ms, hbm_gbs, tc_tflops),
                                        "kernels_ms_per_step": {
                                            n: [v[0] // K, round(v[1] / K, 4)]
                                            for n, v in sorted(prof.items())}}
@@ -563,7 +589,7 @@ def run_ours(args):
     if not args.no_bs1 and not args.layers:
         del cache, ws
         torch.cuda.empty_cache()
-        result["bs1"] = bs1_measure(S, W, args.steps, args.warmup)
+        result["bs1"] = bs1_measure(S, W, args.steps, args.warmup, hbm, tc_burst)
     if not args.no_gqa and not args.layers and world == 1:
         del W, model
         torch.cuda.empty_cache()
