@@ -479,6 +479,22 @@ dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, int M, int N,
                            dllm_stream_t stream);
 
 /*
+ * dllm_selftest_gemm_stall - failure-path check of the CTA-pair GEMM (256-row
+ * tiles, tcgen05 cta_group::2): the same launch as dllm_gemm_bf16 (M >= 256,
+ * N a multiple of 256, accumulate 0, no K split) with one signal withheld:
+ * the second CTA of every pair never reports its first k-block to the first,
+ * so the first CTA's bounded wait runs out after its limit (2 s).  Every CTA
+ * then drains its own loads and returns; the kernel ends with DLLM_DEV_TIMEOUT
+ * in the workspace's device status word (read it with
+ * dllm_get_device_status) and C undefined, and the CUDA context stays usable.
+ * Returns DLLM_ERR_UNSUPPORTED_SHAPE for shapes that do not run on CTA pairs
+ * (or when they are turned off with DLLM_GEMM_PAIR=0).  Arguments as for
+ * dllm_gemm_bf16; ws of dllm_gemm_workspace_size(M, N, K, 1) bytes.
+ */
+dllm_status dllm_selftest_gemm_stall(const void* A, const void* Bm, void* C, int M, int N, int K,
+                                     void* ws, size_t ws_bytes, dllm_stream_t stream);
+
+/*
  * Kernel timing.  dllm_profile_enable(1) brackets every kernel the library
  * launches with CUDA events on the launch stream; dllm_profile_read()
  * synchronises the device, writes a JSON object

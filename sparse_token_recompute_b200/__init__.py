@@ -122,6 +122,7 @@ _attn = _sig("dllm_attention_bf16", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i,
                                          vp])
 _gemm_ws = _sig("dllm_gemm_workspace_size", _sz, [_i, _i, _i, _i])
 _gemm = _sig("dllm_gemm_bf16", _i, [vp, vp, vp, _i, _i, _i, _i, _i, vp, _sz, vp])
+_gemm_stall = _sig("dllm_selftest_gemm_stall", _i, [vp, vp, vp, _i, _i, _i, vp, _sz, vp])
 _prof_enable = _sig("dllm_profile_enable", None, [_i])
 _prof_reset = _sig("dllm_profile_reset", None, [])
 _prof_read = _sig("dllm_profile_read", _sz, [C.c_char_p, _sz])
@@ -270,6 +271,18 @@ def dllm_gemm_bf16(A, Bm, Cm, accumulate=False, splits=0, ws: Workspace = None, 
     st = _gemm(ptr(A), ptr(Bm), ptr(Cm), M, N, K, int(bool(accumulate)), int(splits), ws.ptr,
                ws.nbytes, _stream(stream))
     _check(st, "dllm_gemm_bf16")
+    return ws
+
+
+def dllm_selftest_gemm_stall(A, Bm, Cm, ws: Workspace = None, stream=None):
+    """The CTA-pair GEMM with one stage signal withheld: ends with DLLM_DEV_TIMEOUT
+    in ws's device status (after the 2 s wait limit); C is undefined."""
+    M, K = A.shape
+    N = Bm.shape[0]
+    if ws is None:
+        ws = Workspace(dllm_gemm_workspace_size(M, N, K, 1), A.device)
+    st = _gemm_stall(ptr(A), ptr(Bm), ptr(Cm), M, N, K, ws.ptr, ws.nbytes, _stream(stream))
+    _check(st, "dllm_selftest_gemm_stall")
     return ws
 
 

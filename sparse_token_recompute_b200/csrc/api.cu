@@ -605,6 +605,34 @@ extern "C" dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, in
   return cuda_status(gemm_launch(g, s));
 }
 
+extern "C" dllm_status dllm_selftest_gemm_stall(const void* A, const void* Bm, void* C, int M,
+                                                int N, int K, void* ws, size_t ws_bytes,
+                                                dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M < 256 || N < 256 || N % 256 || K <= 0 || K % 8) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  if (!A || !Bm || !C) return DLLM_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(Bm, 16) || !aligned(C, 16)) return DLLM_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dllm_gemm_workspace_size(M, N, K, 1))
+    return DLLM_ERR_WORKSPACE;
+  GemmSpec g{};
+  g.epi = EPI_STORE;
+  g.A = static_cast<const __nv_bfloat16*>(A);
+  g.M_cap = M;
+  g.K = K;
+  g.B[0] = static_cast<const __nv_bfloat16*>(Bm);
+  g.seg_cols[0] = N;
+  g.n_seg = 1;
+  g.out = static_cast<__nv_bfloat16*>(C);
+  g.ldo = N;
+  g.force_bn = 256;
+  g.force_splits = 1;
+  g.stall_test = 1;
+  if (!gemm_plan(g).pair) return DLLM_ERR_UNSUPPORTED_SHAPE;
+  Bump bp(ws);
+  g.status = bp.take<int>(kHeader / sizeof(int));
+  return cuda_status(gemm_launch(g, s));
+}
+
 // ---------------------------------------------------------------- attention alone
 
 extern "C" size_t dllm_attention_workspace_size(int B) {

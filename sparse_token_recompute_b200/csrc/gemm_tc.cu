@@ -69,6 +69,7 @@ struct Params {
   int a_tx;  // bytes one A box delivers (fewer than a full 128-row tile when M_cap < 128)
   int prefetch_b;  // issue the first unit's weight tiles before waiting on the previous kernel
   int raster_g;    // CTA-pair kernel: row-tile pairs per raster group
+  int stall_test;  // CTA-pair kernel, tests only: CTA 1 withholds its first stage
   int* status;
 };
 
@@ -797,7 +798,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_remote(peer_pfull0 + (uint32_t)(stage * 8));
+          if (!(p.stall_test && kb == 0 && u == pair_id))
+            mbar_arrive_remote(peer_pfull0 + (uint32_t)(stage * 8));
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -1146,6 +1148,8 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   p.lm_part = g.lm_part;
   p.V = N;
   p.status = g.status;
+  p.stall_test = g.stall_test;
+  if (g.stall_test && !pl.pair) return cudaErrorInvalidValue;
 
   CUtensorMap ta, tb0, tb1, tb2;
   // with fewer than 128 rows the A box covers only them (rounded to 16): the MMA still

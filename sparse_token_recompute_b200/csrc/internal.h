@@ -59,6 +59,9 @@ struct GemmSpec {
   int* status;
   int force_bn;      // 0: choose
   int force_splits;  // 0: choose
+  // fault injection for tests (CTA-pair plans only): CTA 1 of every pair never
+  // reports its first stage, so CTA 0's bounded wait runs out (DEV_TIMEOUT)
+  int stall_test;
 };
 
 // launch kernels with programmatic stream serialization (they griddepcontrol.wait

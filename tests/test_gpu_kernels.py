@@ -196,3 +196,21 @@ def test_unmask_random(lib):
         np.testing.assert_array_equal(t_gpu.cpu().numpy(), t_ora)
         if n:
             np.testing.assert_array_equal(pos.cpu().numpy()[:, :n], p_ora)
+
+
+def test_gemm_pair_stall_times_out_and_context_survives(lib):
+    """Failure path of the CTA-pair GEMM: with one stage signal withheld the
+    bounded wait runs out, every CTA drains and returns, the device status
+    reports DLLM_DEV_TIMEOUT, and the same context then computes a correct GEMM."""
+    M, N, K = 512, 1024, 512
+    A = SY.normal((M, K), 1.0, 21, "cuda", "bf16")
+    Bm = SY.normal((N, K), 0.05, 22, "cuda", "bf16")
+    C = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    ws = lib.dllm_selftest_gemm_stall(A, Bm, C)
+    torch.cuda.synchronize()
+    assert ws.device_status() & lib.DLLM_DEV_TIMEOUT
+    C2 = torch.zeros(M, N, dtype=torch.bfloat16, device="cuda")
+    ws2 = lib.dllm_gemm_bf16(A, Bm, C2)
+    torch.cuda.synchronize()
+    assert ws2.device_status() == 0
+    assert max_abs_rel(f64(C2), f64(A) @ f64(Bm).T) < 1e-2
