@@ -54,7 +54,6 @@ def parse():
     ap.add_argument("--no-bs1", action="store_true", help="skip the batch-1 measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gqa", action="store_true", help="skip the 7B GQA ratio sweep")
-    ap.add_argument("--layers", type=int, default=0, help="(debug) override the layer count")
     return ap.parse_args()
 
 
@@ -156,10 +155,8 @@ def barrier(world):
 
 # ----------------------------------------------------------------------------- our path
 
-def setup(S, shape, rank, layers=0):
+def setup(S, shape, rank):
     import torch
-    if layers:
-        shape = SY.with_(shape, n_layers=layers)
     W = SY.model_weights(shape, seed=0, device="cuda")
     model = S.Model(S.cfg_from_shape(shape), W)
     tokens = rank_inputs(shape, rank)
@@ -436,7 +433,7 @@ def run_ours(args):
     import sparse_token_recompute_b200 as S  # raises if the CUDA library is missing
 
     hbm, tc_burst, tc_sus, peak_kind = peaks()
-    shape, W, model, tokens, cache, pol, ws = setup(S, SHAPE, rank, args.layers)
+    shape, W, model, tokens, cache, pol, ws = setup(S, SHAPE, rank)
     stream = torch.cuda.current_stream()
     S.dllm_step(model, cache, tokens, pol, True, ws)           # dense first step (untimed)
     for _ in range(args.warmup):
