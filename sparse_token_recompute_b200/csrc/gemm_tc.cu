@@ -1109,8 +1109,10 @@ GemmPlan gemm_plan(const GemmSpec& g) {
   // rows) the pairs made the QKV GEMM 2% and the O/down GEMMs 3.5% faster, but
   // the gate/up (SwiGLU) GEMM 5% and the LM head 9% slower (both read ~30% more
   // DRAM), so those two keep single-CTA tiles.
-  pl.pair = (pair_enabled() && !weight_bound && splits == 1 && bn == PAIR_BN &&
-             pl.m_tiles_cap >= 2 && sms >= 2 && g.epi != EPI_SWIGLU && g.epi != EPI_LMHEAD)
+  // With two row tiles and no split (129-255 rows, e.g. the QKV GEMM of one
+  // sequence at 192 rows) a pair also halves the weight bytes each SM streams.
+  pl.pair = (pair_enabled() && splits == 1 && bn == PAIR_BN && pl.m_tiles_cap >= 2 && sms >= 2 &&
+             g.epi != EPI_SWIGLU && g.epi != EPI_LMHEAD)
                 ? 1 : 0;
   if (pl.pair) {
     const int units = ((pl.m_tiles_cap + 1) / 2) * pl.tiles_n;
