@@ -578,16 +578,16 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline_sample(W, cache, tokens, shape)
-    if not args.layers and world == 1:
+    if world == 1:
         result["es_two_point"] = es_two_point_measure(S, model, shape, rank, args.steps,
                                                       args.warmup)
         result["dyllm_ffn_gate"] = ffn_gate_measure(S, model, shape, rank, args.steps,
                                                     args.warmup)
-    if not args.no_bs1 and not args.layers:
+    if not args.no_bs1:
         del cache, ws
         torch.cuda.empty_cache()
         result["bs1"] = bs1_measure(S, W, args.steps, args.warmup, hbm, tc_burst)
-    if not args.no_gqa and not args.layers and world == 1:
+    if not args.no_gqa and world == 1:
         del W, model
         torch.cuda.empty_cache()
         result["gqa7b"] = gqa_measure(S, args.steps, args.warmup)
