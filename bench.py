@@ -180,6 +180,32 @@ def time_steps(S, model, cache, tokens, pol, ws, K, stream):
     return e0.elapsed_time(e1)
 
 
+def hbm_kernels(shape, prof, hbm_gbs):
+    """HBM roofline of the step's memory-bound kernels from the event-timed pass
+    (`prof`: name -> [launches, total ms]): algorithmic bytes per launch over the
+    average launch time.  score: the layer-0 input rows (embedding gathers) and
+    the hidden references of every row, confidences and tokens in, scores out;
+    gather: the selected rows read, written compact and written back as
+    references; select: the scores of every row (0.24 MB, one CTA per
+    sequence: bound by latency, not bandwidth)."""
+    B, N, d = shape.batch, shape.seq_len, shape.d
+    M, e = B * shape.k, 2
+    nbytes = {"score": 2 * B * N * d * e + B * N * (4 + 4 + 4),
+              "gather": 3 * M * d * e,
+              "select": B * N * 4 + M * 4}
+    out = {}
+    for name, b in nbytes.items():
+        if name not in prof or prof[name][0] <= 0:
+            continue
+        ms = prof[name][1] / prof[name][0]
+        out[name] = {"bound": "latency" if name == "select" else "hbm",
+                     "bytes_per_launch": int(b), "ms_per_launch": round(ms, 5),
+                     "achieved_gbs": round(b / (ms / 1000.0) / 1e9, 1),
+                     "frac": round(b / (ms / 1000.0) / 1e9 / hbm_gbs, 4)}
+    out["peak_gbs"] = hbm_gbs
+    return out
+
+
 def step_roofline(shape, ms, hbm_gbs, tc_tflops):
     """Whole-step roofline of a partial step: algorithmic bytes = every layer's
     weights + the LM head + the K/V caches the attention reads + the K/V rows
@@ -573,6 +599,7 @@ def run_ours(args):
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "kernels_ms": {k: [v[0], round(v[1], 3)] for k, v in sorted(prof.items())},
+        "hbm_kernels": hbm_kernels(shape, prof, hbm),
         "kernels_ms_note": f"{args.steps} steps with an event pair around every launch "
                            f"({ms_prof / args.steps:.2f} ms/step in that pass)",
     }
