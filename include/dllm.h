@@ -40,6 +40,14 @@
  *   - Storage dtype DLLM_BF16 computes with fp32 accumulation and stores
  *     bf16; DLLM_F32 stores fp32 (small models, exact-arithmetic checks).
  *   - No C++ exception crosses this boundary.
+ *
+ * Environment (read once per process; every setting computes the same
+ * results up to summation order)
+ *   DLLM_PDL=0        launch kernels without programmatic dependent launch
+ *   DLLM_GEMM_PAIR=0  run tensor-bound GEMMs on single CTAs (128-row tiles)
+ *                     instead of CTA pairs (256-row tiles, tcgen05 cta_group::2)
+ *   DLLM_ATTENTION=mma  the warp-level mma.sync attention kernel instead of
+ *                     the tcgen05 one (a cross-check of the two)
  */
 #ifndef DLLM_H
 #define DLLM_H
