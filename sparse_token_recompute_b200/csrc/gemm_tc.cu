@@ -589,8 +589,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ---------------------------------------------------------------- CTA-pair kernel
-// Tensor-bound shapes (>= 256 rows, 256-wide tiles, no K split): the two CTAs of
-// a cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2 issued by
+// Plain, residual and QKV GEMMs with at least two row tiles, 256-wide tiles and
+// no K split (the tensor-bound shapes, and 129-255-row weight streaming): the
+// two CTAs of a cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2
+// issued by
 // CTA 0.  CTA r stages rows [128 r, 128 r + 128) of the A tile and columns
 // [128 r, 128 r + 128) of the B tile (32 KB per 64-deep k-block instead of
 // 48 KB, so the ring holds 7 k-blocks), and its TMEM receives its 128 rows of
@@ -707,8 +709,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB0);
-    if (EPI == EPI_SWIGLU || EPI == EPI_QKV) tma_prefetch_desc(&tmB1);
-    if (EPI == EPI_QKV) tma_prefetch_desc(&tmB2);
+    if (EPI == EPI_QKV) {
+      tma_prefetch_desc(&tmB1);
+      tma_prefetch_desc(&tmB2);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -719,11 +723,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   griddep_launch_dependents();
 
   // this CTA's half (columns [n*BN + rank*BNH, +BNH)) of the B tile of k-block kb
+  // (plain, residual and QKV epilogues; the planner keeps SwiGLU and the LM head
+  // on single CTAs)
+  static_assert(EPI != EPI_SWIGLU && EPI != EPI_LMHEAD, "not run on CTA pairs");
   auto load_b_half = [&](uint32_t b_dst, uint32_t bar, int kb, int n) {
-    if constexpr (EPI == EPI_SWIGLU) {
-      // gate columns come from CTA 0, the matching up columns from CTA 1
-      tma_load_2d(b_dst, rank == 0 ? &tmB0 : &tmB1, bar, kb * BK, n * BNH);
-    } else if constexpr (EPI == EPI_QKV) {
+    if constexpr (EPI == EPI_QKV) {
       const int n0 = n * BN + (int)rank * BNH;  // segments are multiples of BN
       if (n0 < p.seg0)
         tma_load_2d(b_dst, &tmB0, bar, kb * BK, n0);
