@@ -592,11 +592,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 // Plain, residual and QKV GEMMs with at least two row tiles, 256-wide tiles and
 // no K split (the tensor-bound shapes, and 129-255-row weight streaming): the
 // two CTAs of a cluster compute one 256 x 256 tile with tcgen05.mma.cta_group::2
-// issued by
-// CTA 0.  CTA r stages rows [128 r, 128 r + 128) of the A tile and columns
-// [128 r, 128 r + 128) of the B tile (32 KB per 64-deep k-block instead of
-// 48 KB, so the ring holds 7 k-blocks), and its TMEM receives its 128 rows of
-// the accumulator over all 256 columns.  Each CTA's TMA loads complete on its
+// issued by CTA 0.  CTA r stages rows [128 r, 128 r + 128) of the A tile and
+// columns [128 r, 128 r + 128) of the B tile (32 KB per 64-deep k-block instead
+// of 48 KB, so the ring holds 7 k-blocks), and its TMEM receives its 128 rows
+// of the accumulator over all 256 columns.  Each CTA's TMA loads complete on its
 // own barriers; CTA 1's issuer thread forwards each landed stage to CTA 0
 // (remote mbarrier arrive), CTA 0's commits arrive on both CTAs' barriers
 // (multicast commit), and CTA 1's epilogue warps release accumulators to CTA 0
