@@ -487,6 +487,20 @@ dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, int M, int N,
                            dllm_stream_t stream);
 
 /*
+ * dllm_gemm_plan_info - the launch plan the library picks for one projection
+ * GEMM, computed on the host (no GPU work; with no device visible the plan
+ * assumes 148 SMs).  kind: 0 plain, 1 residual, 2 gate/up + SwiGLU (n_seg 2:
+ * seg_cols = {F, F}), 3 QKV + RoPE (n_seg 3: {q, kv, kv} columns), 4 LM head
+ * (n_seg 1, as plain otherwise).  M rows (capacity), K inner size, head_dim
+ * for QKV.  out (HOST, 5 int32): column-tile width, K splits, column tiles,
+ * CTAs launched, 1 when CTA pairs (256-row tiles, tcgen05 cta_group::2) run it.
+ * DLLM_ERR_INVALID_ARG for an unknown kind, a segment count that does not
+ * match it, or non-positive sizes.
+ */
+dllm_status dllm_gemm_plan_info(int kind, int M, int K, const int32_t* seg_cols, int n_seg,
+                                int head_dim, int32_t* out);
+
+/*
  * dllm_selftest_gemm_stall - failure-path check of the CTA-pair GEMM (256-row
  * tiles, tcgen05 cta_group::2): the same launch as dllm_gemm_bf16 (M >= 256,
  * N a multiple of 256, accumulate 0, no K split) with one signal withheld:

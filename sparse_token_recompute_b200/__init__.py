@@ -123,6 +123,7 @@ _attn = _sig("dllm_attention_bf16", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i,
 _gemm_ws = _sig("dllm_gemm_workspace_size", _sz, [_i, _i, _i, _i])
 _gemm = _sig("dllm_gemm_bf16", _i, [vp, vp, vp, _i, _i, _i, _i, _i, vp, _sz, vp])
 _gemm_stall = _sig("dllm_selftest_gemm_stall", _i, [vp, vp, vp, _i, _i, _i, vp, _sz, vp])
+_gemm_plan = _sig("dllm_gemm_plan_info", _i, [_i, _i, _i, vp, _i, _i, vp])
 _prof_enable = _sig("dllm_profile_enable", None, [_i])
 _prof_reset = _sig("dllm_profile_reset", None, [])
 _prof_read = _sig("dllm_profile_read", _sz, [C.c_char_p, _sz])
@@ -272,6 +273,19 @@ def dllm_gemm_bf16(A, Bm, Cm, accumulate=False, splits=0, ws: Workspace = None, 
                ws.nbytes, _stream(stream))
     _check(st, "dllm_gemm_bf16")
     return ws
+
+
+GEMM_KINDS = {"plain": 0, "residual": 1, "swiglu": 2, "qkv": 3, "lmhead": 4}
+
+
+def dllm_gemm_plan_info(kind: str, M: int, K: int, seg_cols, head_dim: int = 0) -> Dict[str, int]:
+    """The host-side launch plan of one projection GEMM (no GPU work)."""
+    segs = (C.c_int32 * len(seg_cols))(*[int(c) for c in seg_cols])
+    out = (C.c_int32 * 5)()
+    st = _gemm_plan(GEMM_KINDS[kind], int(M), int(K), C.cast(segs, C.c_void_p), len(seg_cols),
+                    int(head_dim), C.cast(out, C.c_void_p))
+    _check(st, "dllm_gemm_plan_info")
+    return {"bn": out[0], "splits": out[1], "tiles_n": out[2], "grid": out[3], "pair": out[4]}
 
 
 def dllm_selftest_gemm_stall(A, Bm, Cm, ws: Workspace = None, stream=None):

@@ -605,6 +605,32 @@ extern "C" dllm_status dllm_gemm_bf16(const void* A, const void* Bm, void* C, in
   return cuda_status(gemm_launch(g, s));
 }
 
+extern "C" dllm_status dllm_gemm_plan_info(int kind, int M, int K, const int32_t* seg_cols,
+                                           int n_seg, int head_dim, int32_t* out) {
+  if (kind < EPI_STORE || kind > EPI_LMHEAD || M <= 0 || K <= 0 || !seg_cols || !out ||
+      n_seg < 1 || n_seg > 3)
+    return DLLM_ERR_INVALID_ARG;
+  if ((kind == EPI_QKV) != (n_seg == 3) || (kind == EPI_SWIGLU) != (n_seg == 2))
+    return DLLM_ERR_INVALID_ARG;
+  GemmSpec g{};
+  g.epi = kind;
+  g.M_cap = M;
+  g.K = K;
+  g.n_seg = n_seg;
+  for (int i = 0; i < n_seg; ++i) {
+    if (seg_cols[i] <= 0) return DLLM_ERR_INVALID_ARG;
+    g.seg_cols[i] = seg_cols[i];
+  }
+  g.hd = head_dim;
+  const GemmPlan pl = gemm_plan(g);
+  out[0] = pl.bn;
+  out[1] = pl.splits;
+  out[2] = pl.tiles_n;
+  out[3] = pl.grid;
+  out[4] = pl.pair;
+  return DLLM_OK;
+}
+
 extern "C" dllm_status dllm_selftest_gemm_stall(const void* A, const void* Bm, void* C, int M,
                                                 int N, int K, void* ws, size_t ws_bytes,
                                                 dllm_stream_t stream) {

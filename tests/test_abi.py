@@ -78,3 +78,46 @@ def test_workspace_sizes_are_host_computable(lib):
     assert 0 < a < b
     assert S.dllm_partial_layer_workspace_size(cfg, 1, 128, 32) > 0
     assert S.dllm_select_workspace_size(4, 100) >= 4
+
+
+def test_gemm_plans_of_the_benchmarked_shapes(lib):
+    """The host-side GEMM planner (no GPU: 148 SMs assumed) picks the plans the
+    measurements behind it chose: CTA pairs for the QKV, O and down projections
+    at 32 x 308 rows, single CTAs for gate/up and the LM head; at one sequence,
+    weight-streaming plans that fill one wave (K splits for the narrow O and
+    down projections) and a pair for QKV at 192 rows."""
+    import sparse_token_recompute_b200 as S
+    P = S.dllm_gemm_plan_info
+    qkv, o, gu, down = (["qkv", 4096, [4096, 4096, 4096], 128], ["residual", 4096, [4096]],
+                        ["swiglu", 4096, [12288, 12288]], ["residual", 12288, [4096]])
+
+    def plan(spec, M):
+        kind, K, segs, *hd = spec
+        return P(kind, M, K, segs, *hd)
+
+    M = 32 * 308
+    for spec in (qkv, o, down):
+        assert plan(spec, M) == {**plan(spec, M), "bn": 256, "splits": 1, "grid": 148, "pair": 1}
+    assert plan(gu, M) == {"bn": 256, "splits": 1, "tiles_n": 96, "grid": 148, "pair": 0}
+    assert P("lmhead", 8100, 4096, [126464])["pair"] == 0
+    assert plan(qkv, 77) == {"bn": 128, "splits": 1, "tiles_n": 96, "grid": 96, "pair": 0}
+    for spec in (o, down):
+        assert plan(spec, 77) == {"bn": 128, "splits": 4, "tiles_n": 32, "grid": 128, "pair": 0}
+    assert plan(qkv, 192) == {"bn": 256, "splits": 1, "tiles_n": 48, "grid": 96, "pair": 1}
+    assert plan(o, 192)["pair"] == 0 and plan(o, 192)["splits"] == 4
+    # no plan is wider than the SM count in one wave, except split K (one unit per CTA)
+    for spec in (qkv, o, gu, down):
+        for rows in (1, 77, 192, 384, 1000, 9856):
+            p = plan(spec, rows)
+            assert p["grid"] <= 148 or p["splits"] > 1
+            assert p["pair"] in (0, 1) and (not p["pair"] or p["grid"] % 2 == 0)
+
+
+def test_gemm_plan_rejects_bad_arguments(lib):
+    import sparse_token_recompute_b200 as S
+    segs = (C.c_int32 * 3)(4096, 4096, 4096)
+    out = (C.c_int32 * 5)()
+    assert S._gemm_plan(9, 100, 64, C.cast(segs, C.c_void_p), 1, 0, C.cast(out, C.c_void_p)) == 1
+    assert S._gemm_plan(3, 100, 64, C.cast(segs, C.c_void_p), 1, 128, C.cast(out, C.c_void_p)) == 1
+    assert S._gemm_plan(0, 0, 64, C.cast(segs, C.c_void_p), 1, 0, C.cast(out, C.c_void_p)) == 1
+    assert S._gemm_plan(0, 100, 64, None, 1, 0, C.cast(out, C.c_void_p)) == 1
