@@ -725,30 +725,20 @@ cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensor
 
 }  // namespace
 
-int num_sms_cached() {
-  static int n = [] {
-    int dev = 0, v = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    return v;
-  }();
-  return n;
-}
-
 int attention_kv_split(int B, int k_cap, int Nseq, int Hq) {
   // few (sequence, head, pair) CTAs leave most SMs idle: share each pair's keys
   // among up to 8 CTAs, at least two K/V tiles each
   const int T = (Nseq + BKV - 1) / BKV;
   const int ctas = ((k_cap + NTILE * BT - 1) / (NTILE * BT)) * Hq * B;
-  if (ctas <= 0 || 2 * ctas > num_sms_cached() || T < 4) return 1;
-  int S = std::max(1, std::min(std::min(8, T / 2), num_sms_cached() / ctas));
+  if (ctas <= 0 || 2 * ctas > num_sms() || T < 4) return 1;
+  int S = std::max(1, std::min(std::min(8, T / 2), num_sms() / ctas));
   while (S > 1 && (S - 1) * ((T + S - 1) / S) >= T) --S;  // every share holds keys
   return S;
 }
 
 size_t attention_part_bytes_bound(int cap, int Hq, int hd) {
   // a split launch has S * rows <= SMs * (rows of a pair) for any batch shape
-  const size_t rows = std::min((size_t)8 * cap * Hq, (size_t)num_sms_cached() * NTILE * BT);
+  const size_t rows = std::min((size_t)8 * cap * Hq, (size_t)num_sms() * NTILE * BT);
   return rows * (hd + 2) * sizeof(float);
 }
 
@@ -810,7 +800,7 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
   // few changed keys make short key streams: a CTA takes several pairs of query
   // tiles of its (sequence, head) in turn, keeping about two CTAs per SM in flight
   const int pairs = (r_cap + NTILE * BT - 1) / (NTILE * BT);
-  const int min_x = std::max(1, (2 * num_sms_cached() + B * Hq - 1) / (B * Hq));
+  const int min_x = std::max(1, (2 * num_sms() + B * Hq - 1) / (B * Hq));
   const int ppc = std::max(1, (pairs + min_x - 1) / min_x);
   AttnParams p{r_off, o,    0,    Hq,   Hkv,   Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
                status, st_m, st_l, a_off, ppc,   1,       0,
