@@ -40,14 +40,8 @@
  *   - Storage dtype DLLM_BF16 computes with fp32 accumulation and stores
  *     bf16; DLLM_F32 stores fp32 (small models, exact-arithmetic checks).
  *   - No C++ exception crosses this boundary.
- *
- * Environment (read once per process; every setting computes the same
- * results up to summation order)
- *   DLLM_PDL=0        launch kernels without programmatic dependent launch
- *   DLLM_GEMM_PAIR=0  run tensor-bound GEMMs on single CTAs (128-row tiles)
- *                     instead of CTA pairs (256-row tiles, tcgen05 cta_group::2)
- *   DLLM_ATTENTION=mma  the warp-level mma.sync attention kernel instead of
- *                     the tcgen05 one (a cross-check of the two)
+ *   - One kernel path per operation: no environment variable or run-time
+ *     switch selects another implementation.
  */
 #ifndef DLLM_H
 #define DLLM_H
@@ -333,6 +327,10 @@ typedef struct {
   float* scores2_out;
   int32_t* ffn_rows_out;  /* [n_layers] device: rows that ran each layer's FFN under the
                            * FFN gate (layers the step did not run are left untouched) */
+  const uint8_t* forced_ffn; /* [n_layers, B*k_cap] device: replaces the FFN gate's rule in a
+                              * partial step; entry l*B*k_cap + r != 0 makes compact row r
+                              * (rows packed by sequence in ascending position, after a
+                              * second skip point the kept rows) salient in layer l */
 } dllm_step_io;
 
 /*
@@ -381,6 +379,24 @@ dllm_status dllm_generate(const dllm_model_cfg* cfg, const dllm_model_w* w,
                           const dllm_cache* cache, int32_t* tokens, int B, int N,
                           const dllm_policy* policy, int n_steps, int32_t* pos_log,
                           uint8_t* dense_log, void* ws, size_t ws_bytes, dllm_stream_t stream);
+
+/*
+ * dllm_step_host - one dllm_step whose token state lives in HOST memory, for
+ * callers that keep tokens on the host between steps: copies tokens_host
+ * [B, N] int32 (HOST, in/out) into the workspace, runs the step there, and
+ * copies the updated tokens back into tokens_host and, when pos_host is not
+ * NULL, the revealed positions into pos_host [B, dllm_unmask_capacity(policy)]
+ * (HOST, -1 padded).  Everything is enqueued on `stream`; the host buffers are
+ * read and written by the copies in stream order, so they hold the results
+ * once the stream has been synchronised (page-locked host memory keeps the
+ * copies asynchronous).  ws: dllm_step_host_workspace_size() bytes.
+ */
+size_t dllm_step_host_workspace_size(const dllm_model_cfg* cfg, int B, int N,
+                                     const dllm_policy* policy);
+dllm_status dllm_step_host(const dllm_model_cfg* cfg, const dllm_model_w* w,
+                           const dllm_cache* cache, int32_t* tokens_host, int B, int N,
+                           const dllm_policy* policy, int dense, int32_t* pos_host, void* ws,
+                           size_t ws_bytes, dllm_stream_t stream);
 
 /*
  * dllm_attention_bf16 - the partial attention of one layer on its own
@@ -442,22 +458,26 @@ dllm_status dllm_attention_update_bf16(const void* q, void* o, float* m, float* 
 
 /*
  * dllm_attention_bf16_noalloc - dllm_attention_bf16 without a workspace, for
- * callers that cannot allocate device memory: code running while a CUDA
- * graph is captured (cudaMalloc cannot be captured and may synchronise the
- * device), servers whose memory is split into fixed pools before serving,
- * plugins that only receive the tensors they compute on.  The pages have no
+ * callers that cannot allocate device memory: servers that split all device
+ * memory into fixed pools before serving (nothing may allocate on the request
+ * path, and cudaMalloc can synchronise the device), and plugins or operators
+ * that are handed only the tensors they compute on.  The pages have no
  * counterpart; this is an integration convenience.
  * Same arguments and result as dllm_attention_bf16 minus ws/ws_bytes.  Its
  * scratch (a status word and B + 1 row offsets) is a fixed array in the
  * library's device memory, sized for at most DLLM_NOALLOC_MAX_SEQS sequences
  * (larger B returns DLLM_ERR_CAPACITY before anything is launched); every GPU
- * that loads the library holds it until the process exits.  The first call on
- * a device looks up the array's device address: make it before any stream
- * capture.  All calls share the array: calls that may overlap on the GPU
- * (other streams, other host threads on the same device) race and must be
- * ordered by the caller.  Device-side faults are recorded in the shared
- * status word, which this entry point clears at the start of each call and
- * does not report.
+ * that loads the library holds it until the process exits.  The first call in
+ * each device context (per device, and again after the context changes, e.g.
+ * after cudaDeviceReset) looks up the array's device address: make it before
+ * any stream capture.  All calls share the array: calls that may overlap on
+ * the GPU (other streams, other host threads on the same device) race and
+ * must be ordered by the caller.  Device-side faults are recorded in the
+ * shared status word, which this entry point clears at the start of each call
+ * and does not report.  It never splits one sequence's keys among several
+ * CTAs (that needs a partial-output scratch far larger than the fixed array),
+ * so with few query tiles (one or two sequences of a few hundred selected
+ * rows) it runs fewer CTAs than dllm_attention_bf16 and can be slower.
  */
 #define DLLM_NOALLOC_MAX_SEQS 4096
 dllm_status dllm_attention_bf16_noalloc(const void* q, const void* k_cache, const void* v_cache,
@@ -509,8 +529,7 @@ dllm_status dllm_gemm_plan_info(int kind, int M, int K, const int32_t* seg_cols,
  * then drains its own loads and returns; the kernel ends with DLLM_DEV_TIMEOUT
  * in the workspace's device status word (read it with
  * dllm_get_device_status) and C undefined, and the CUDA context stays usable.
- * Returns DLLM_ERR_UNSUPPORTED_SHAPE for shapes that do not run on CTA pairs
- * (or when they are turned off with DLLM_GEMM_PAIR=0).  Arguments as for
+ * Returns DLLM_ERR_UNSUPPORTED_SHAPE for shapes that do not run on CTA pairs.  Arguments as for
  * dllm_gemm_bf16; ws of dllm_gemm_workspace_size(M, N, K, 1) bytes.
  */
 dllm_status dllm_selftest_gemm_stall(const void* A, const void* Bm, void* C, int M, int N, int K,

@@ -614,6 +614,9 @@ class StepOut:
     idx2: Optional[List[np.ndarray]] = None   # rows kept at the second skip point
     scores2: Optional[List[np.ndarray]] = None  # their scores, per sequence in idx order
     ffn_rows: Optional[List[int]] = None  # FFN gating: salient rows per recomputed layer
+    # FFN gating: per recomputed layer, the salient flag of each compact row (rows packed
+    # by sequence, ascending positions; after a second skip point, the kept rows)
+    ffn_salient: Optional[List[np.ndarray]] = None
 
 
 def embed(W: ModelW, tokens: np.ndarray) -> np.ndarray:
@@ -691,6 +694,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
     l2 = pol.score_layer2 if pol.score_layer2 > ls else -1
     idx2 = sc2 = None
     ffn_rows = [] if pol.ffn_gate else None
+    ffn_sal = [] if pol.ffn_gate else None
     for l in range(ls, cfg.n_layers):
         if l == l2:
             if not dense:
@@ -702,6 +706,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
             x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l], gate)
             if gate is not None:
                 ffn_rows.append(int(np.sum(gate.salient)))
+                ffn_sal.append(gate.salient.copy())
     sel_masked = masked[b_of, p_of]
     if np.any(sel_masked):
         n = store(rms_norm(x[sel_masked], W.final_norm, cfg.rms_eps), cfg.dtype)
@@ -719,7 +724,7 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
     for a in (idx2 if idx2 is not None else idx):
         rows.append(x[off:off + len(a)].copy())
         off += len(a)
-    return StepOut(idx, scores, pos, rows, idx2, sc2, ffn_rows)
+    return StepOut(idx, scores, pos, rows, idx2, sc2, ffn_rows, ffn_sal)
 
 
 def block_starts(cfg: ModelCfg, pol: Policy, tokens: np.ndarray) -> List[int]:

@@ -71,7 +71,8 @@ class StepIO(C.Structure):
     _fields_ = [("forced_idx", vp), ("forced_count", vp), ("forced_unmask_pos", vp),
                 ("idx_out", vp), ("count_out", vp), ("pos_out", vp), ("scores_out", vp),
                 ("forced_idx2", vp), ("forced_count2", vp), ("idx2_out", vp),
-                ("count2_out", vp), ("scores2_out", vp), ("ffn_rows_out", vp)]
+                ("count2_out", vp), ("scores2_out", vp), ("ffn_rows_out", vp),
+                ("forced_ffn", vp)]
 
 
 def _sig(name, res, args):
@@ -109,6 +110,11 @@ _gen_ws = _sig("dllm_generate_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i
 _gen = _sig("dllm_generate", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW), C.POINTER(CacheS), vp,
                                   _i, _i, C.POINTER(Policy), _i, vp, C.POINTER(C.c_uint8), vp,
                                   _sz, vp])
+_step_host_ws = _sig("dllm_step_host_workspace_size", _sz, [C.POINTER(ModelCfg), _i, _i,
+                                                            C.POINTER(Policy)])
+_step_host = _sig("dllm_step_host", _i, [C.POINTER(ModelCfg), C.POINTER(ModelW),
+                                         C.POINTER(CacheS), vp, _i, _i, C.POINTER(Policy), _i,
+                                         vp, vp, _sz, vp])
 _devstat = _sig("dllm_get_device_status", _i, [vp, vp, C.POINTER(C.c_int32)])
 _attn_noalloc = _sig("dllm_attention_bf16_noalloc", _i, [vp, vp, vp, vp, vp, _i, _i, _i, _i, _i,
                                                          _i, vp])
@@ -351,8 +357,8 @@ DLLM_NOALLOC_MAX_SEQS = 4096
 
 def dllm_attention_bf16_noalloc(q, k_cache, v_cache, o, count, k_cap: int, stream=None):
     """Partial attention without a workspace, for callers that cannot allocate
-    device memory (e.g. inside CUDA-graph capture, after the first call on the
-    device); its scratch is a fixed array inside the library shared by all calls."""
+    device memory (memory carved into fixed pools, operators handed only their
+    tensors); its scratch is a fixed array inside the library shared by all calls."""
     B, N, Hkv, hd = k_cache.shape
     Hq = q.shape[1] // hd
     st = _attn_noalloc(ptr(q), ptr(k_cache), ptr(v_cache), ptr(o), ptr(count), B, int(k_cap), N,
@@ -501,7 +507,8 @@ def dllm_step_ex(model: Model, cache: Cache, tokens, pol: Policy, dense: bool, w
                  stream=None, **io):
     """dllm_step with the second skip point; keyword tensors fill dllm_step_io
     (forced_idx, forced_count, forced_unmask_pos, idx_out, count_out, pos_out,
-    scores_out, forced_idx2, forced_count2, idx2_out, count2_out, scores2_out)."""
+    scores_out, forced_idx2, forced_count2, idx2_out, count2_out, scores2_out,
+    ffn_rows_out, forced_ffn)."""
     B, N = tokens.shape
     s = StepIO(*[ptr(io.get(name)) for name, _ in StepIO._fields_])
     unknown = set(io) - {name for name, _ in StepIO._fields_}
@@ -513,14 +520,22 @@ def dllm_step_ex(model: Model, cache: Cache, tokens, pol: Policy, dense: bool, w
     _check(st, "dllm_step_ex")
 
 
+def dllm_step_host_workspace_size(cfg: ModelCfg, B: int, N: int, pol: Policy) -> int:
+    return int(_step_host_ws(C.byref(cfg), B, N, C.byref(pol)))
+
+
 def dllm_step_host(model: Model, cache: Cache, tokens_host, pol: Policy, dense: bool,
-                   ws: Workspace, dev_tokens, dev_pos, pos_host, stream=None):
-    """One step from HOST token buffers: copies tokens in (pinned host -> device),
-    runs dllm_step, copies the updated tokens and revealed positions back."""
-    dev_tokens.copy_(tokens_host, non_blocking=True)
-    dllm_step(model, cache, dev_tokens, pol, dense, ws, pos_out=dev_pos, stream=stream)
-    tokens_host.copy_(dev_tokens, non_blocking=True)
-    pos_host.copy_(dev_pos, non_blocking=True)
+                   ws: Workspace, pos_host=None, stream=None):
+    """One step whose tokens live in HOST memory (the C entry point copies them
+    in, runs the step and copies tokens and revealed positions back, all on the
+    stream; the host tensors hold the results after the stream synchronises).
+    tokens_host [B, N] int32 and pos_host [B, capacity] int32: CPU tensors,
+    preferably pinned."""
+    B, N = tokens_host.shape
+    st = _step_host(C.byref(model.cfg), C.byref(model.s), C.byref(cache.s), ptr(tokens_host), B,
+                    N, C.byref(pol), int(bool(dense)), ptr(pos_host), ws.ptr, ws.nbytes,
+                    _stream(stream))
+    _check(st, "dllm_step_host")
 
 
 class StepGraph:

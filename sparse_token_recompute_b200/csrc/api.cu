@@ -239,17 +239,6 @@ void layout_layer(Bump& bp, const dllm_model_cfg* c, int B, int N, int cap, Laye
   }
 }
 
-// DLLM_ATTENTION=mma selects the warp-level MMA attention kernel instead of
-// the tcgen05 one (used to compare the two on the same inputs).
-bool attention_legacy() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("DLLM_ATTENTION");
-    v = (e && strcmp(e, "mma") == 0) ? 1 : 0;
-  }
-  return v == 1;
-}
-
 // One transformer layer over the compact rows in x (in place).
 // DyLLM FFN gate of one layer (see launch_ffn_gate)
 struct LayerGate {
@@ -257,6 +246,7 @@ struct LayerGate {
   void* ffn;          // [B, N, d] FFN outputs at each row's last salient pass
   float tau;          // salient when 1 - cos > tau
   int all_rows;       // every row salient (dense steps)
+  const uint8_t* forced;  // [cap] decisions replacing the rule, or null
   int* flag;          // [cap] scratch
   int* list;          // [cap] salient rows
   int* inv;           // [cap] row -> place in the list, or -1
@@ -303,11 +293,7 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     g.hd = hd;
     g.rope = rope;
     if (gemm_launch(g, s) != cudaSuccess) return DLLM_ERR_CUDA;
-    if (attention_legacy()) {
-      launch_attention_bf16(static_cast<const bf*>(w.q), static_cast<const bf*>(k_cache),
-                            static_cast<const bf*>(v_cache), static_cast<bf*>(w.o), w.row_off, B,
-                            k_cap, N, c->n_heads, c->n_kv_heads, hd, s);
-    } else if (launch_attention_tc(static_cast<const bf*>(w.q), M_cap,
+    if (launch_attention_tc(static_cast<const bf*>(w.q), M_cap,
                                    static_cast<const bf*>(k_cache),
                                    static_cast<const bf*>(v_cache), static_cast<bf*>(w.o),
                                    w.row_off, B, k_cap, N, c->n_heads, c->n_kv_heads, hd,
@@ -328,8 +314,8 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     if (gate) {
       // DyLLM: the FFN only on rows whose attention output moved, the rest reuse it
       launch_ffn_gate<bf>(static_cast<const bf*>(w.o), static_cast<bf*>(gate->ctx), w.row_pos,
-                          w.row_seq, M_dev, M_cap, N, q, gate->tau, gate->all_rows, gate->flag,
-                          gate->list, gate->inv, gate->n_sal, s);
+                          w.row_seq, M_dev, M_cap, N, q, gate->tau, gate->all_rows,
+                          gate->forced, gate->flag, gate->list, gate->inv, gate->n_sal, s);
       launch_rmsnorm_rows<bf>(xb, static_cast<const bf*>(lw->ffn_norm), nb, gate->list,
                               gate->n_sal, M_cap, d, c->rms_eps, s);
       GemmSpec gu = g;
@@ -407,7 +393,7 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     if (gate) {
       launch_ffn_gate<float>(static_cast<const float*>(w.o), static_cast<float*>(gate->ctx),
                              w.row_pos, w.row_seq, M_dev, M_cap, N, q, gate->tau, gate->all_rows,
-                             gate->flag, gate->list, gate->inv, gate->n_sal, s);
+                             gate->forced, gate->flag, gate->list, gate->inv, gate->n_sal, s);
       launch_rmsnorm_rows<float>(xf, static_cast<const float*>(lw->ffn_norm), nf, gate->list,
                                  gate->n_sal, M_cap, d, c->rms_eps, s);
       launch_gemm_f32(nf, static_cast<const float*>(lw->w_gate), w.graw, nullptr, gate->n_sal,
@@ -1003,8 +989,10 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
   const int* M_dev = L.row_off + B;
   auto gate_of = [&](int l, bool all_rows, LayerGate& gt) -> const LayerGate* {
     if (!pol->ffn_gate) return nullptr;
-    gt = LayerGate{cache->ctx[l], cache->ffn[l], pol->ffn_tau, all_rows ? 1 : 0, w.g_flag,
-                   w.g_list, w.g_inv, w.g_n, w.g_f,
+    const uint8_t* forced =
+        (!all_rows && io.forced_ffn) ? io.forced_ffn + (size_t)l * B * k_cap : nullptr;
+    gt = LayerGate{cache->ctx[l], cache->ffn[l], pol->ffn_tau, all_rows ? 1 : 0, forced,
+                   w.g_flag, w.g_list, w.g_inv, w.g_n, w.g_f,
                    io.ffn_rows_out ? io.ffn_rows_out + l : nullptr};
     return &gt;
   };
@@ -1243,5 +1231,47 @@ extern "C" dllm_status dllm_generate(const dllm_model_cfg* c, const dllm_model_w
     if (st != DLLM_OK) return st;
     if (dense_log) dense_log[t] = dense ? 1 : 0;
   }
+  return DLLM_OK;
+}
+
+// ---------------------------------------------------------------- host token buffers
+
+extern "C" size_t dllm_step_host_workspace_size(const dllm_model_cfg* c, int B, int N,
+                                                const dllm_policy* pol) {
+  const size_t step = dllm_step_workspace_size(c, B, N, pol);
+  if (step == 0) return 0;
+  const size_t cap = (size_t)std::max(dllm_unmask_capacity(pol), 1);
+  return round_up(step, 256) + round_up((size_t)B * N * sizeof(int32_t), 256) +
+         round_up((size_t)B * cap * sizeof(int32_t), 256);
+}
+
+extern "C" dllm_status dllm_step_host(const dllm_model_cfg* c, const dllm_model_w* mw,
+                                      const dllm_cache* cache, int32_t* tokens_host, int B, int N,
+                                      const dllm_policy* pol, int dense, int32_t* pos_host,
+                                      void* ws, size_t ws_bytes, dllm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!c || !pol || !tokens_host || B < 0 || N < 0) return DLLM_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return DLLM_OK;
+  const size_t step_ws = dllm_step_workspace_size(c, B, N, pol);
+  if (step_ws == 0) return check_cfg(c) != DLLM_OK ? check_cfg(c) : DLLM_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dllm_step_host_workspace_size(c, B, N, pol))
+    return DLLM_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  int32_t* d_tok = reinterpret_cast<int32_t*>(base + round_up(step_ws, 256));
+  int32_t* d_pos = reinterpret_cast<int32_t*>(base + round_up(step_ws, 256) +
+                                              round_up((size_t)B * N * sizeof(int32_t), 256));
+  const size_t tok_bytes = (size_t)B * N * sizeof(int32_t);
+  const size_t pos_bytes = (size_t)B * std::max(dllm_unmask_capacity(pol), 1) * sizeof(int32_t);
+  if (cudaMemcpyAsync(d_tok, tokens_host, tok_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  const dllm_status st = dllm_step(c, mw, cache, d_tok, B, N, pol, dense, nullptr, nullptr,
+                                   nullptr, nullptr, nullptr, pos_host ? d_pos : nullptr, nullptr,
+                                   ws, step_ws, stream);
+  if (st != DLLM_OK) return st;
+  if (cudaMemcpyAsync(tokens_host, d_tok, tok_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DLLM_ERR_CUDA;
+  if (pos_host &&
+      cudaMemcpyAsync(pos_host, d_pos, pos_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return DLLM_ERR_CUDA;
   return DLLM_OK;
 }

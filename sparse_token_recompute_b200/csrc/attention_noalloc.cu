@@ -3,22 +3,29 @@
 // dllm_attention_bf16 takes a caller workspace for its scratch: one status word
 // and the per-sequence offsets of the compact query rows.  Some callers have no
 // way to provide one:
-//   * code that runs while a CUDA graph is being captured -- cudaMalloc is not
-//     a stream operation, cannot be captured, and may synchronise the device;
 //   * serving processes that carve all device memory into fixed pools before
-//     they start, so nothing may allocate on the request path;
-//   * plugins handed only the tensors they compute on.
+//     they start, so nothing may allocate on the request path (cudaMalloc can
+//     also synchronise the device, which stalls every stream in flight);
+//   * plugins and operators handed only the tensors they compute on, with no
+//     allocator of their own.
 // dllm_attention_bf16_noalloc keeps that scratch in a fixed array in the
 // library's own device memory instead (about 16 KB for DLLM_NOALLOC_MAX_SEQS
 // sequences, held by every GPU that loads the library until the process exits).
 //
 // Host code cannot use the array's name as a device address: on the host it
-// names a host-side stand-in.  The device address is looked up once per
-// device with cudaGetSymbolAddress, with that device current, on the first
-// call made on it; make that first call before any stream capture.  Every call
+// names a host-side stand-in.  The device address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call made in
+// each device context (and again if the context changes, e.g. after a
+// cudaDeviceReset); make that first call before any stream capture.  Every call
 // shares the array, so calls that may overlap on the GPU (different streams,
 // or different host threads on one device) race on it and must be ordered by
-// the caller.
+// the caller.  This entry point never splits a sequence's keys among CTAs (the
+// split needs a partial-output scratch far larger than the fixed array), so
+// with few query tiles -- one or two sequences of a few hundred selected rows --
+// it runs fewer CTAs than dllm_attention_bf16 and can be slower.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "../../include/dllm.h"
@@ -34,22 +41,49 @@ constexpr int kOffsetBase = 64;  // status word at [0]; offsets start 256 bytes 
 static __device__ __align__(256) int g_noalloc_scratch[kOffsetBase + kMaxSeqs + 1];
 
 std::mutex g_mu;
-int* g_addr[64] = {};
+struct Slot {
+  CUcontext ctx;  // the context the address was looked up in
+  int* addr;
+};
+Slot g_slot[64] = {};
 
-// device address of g_noalloc_scratch on the current device (set up once per device)
+// the driver's cuCtxGetCurrent, reached through the runtime (no link-time libcuda)
+PFN_cuCtxGetCurrent_v4000 ctx_current_fn() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  });
+  return fn;
+}
+
+// device address of g_noalloc_scratch in the current device context (looked up once
+// per device and context)
 cudaError_t scratch_address(int** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  auto get_ctx = ctx_current_fn();
+  if (!get_ctx) return cudaErrorUnknown;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return cudaErrorUnknown;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
+  Slot& sl = g_slot[dev];
+  if (!sl.addr || !ctx || sl.ctx != ctx) {
+    // the lookup also makes the device's primary context current when none was
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    g_addr[dev] = static_cast<int*>(p);
+    if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorUnknown;
+    sl.addr = static_cast<int*>(p);
+    sl.ctx = ctx;
   }
-  *out = g_addr[dev];
+  *out = sl.addr;
   return cudaSuccess;
 }
 

@@ -140,12 +140,6 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&t);
 }
 
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-}
-
 // B operand stored MN-major (hd contiguous, one 128-byte row per key) with the
 // 128-byte swizzle: 8-key groups 1024 B apart (SBO), 64-column halves LBO apart.
 __device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t lbo_bytes) {
@@ -359,9 +353,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
       if (!ok) {
-        if (q_issued > 0) wait_drain(q_full, (q_issued - 1) & 1);
+        if (q_issued > 0) mbar_wait_drain(q_full, (q_issued - 1) & 1, p.status);
         for (int sl = 0; sl < NS; ++sl)
-          if (issued & (1u << sl)) wait_drain(full(sl), (issue_par >> sl) & 1u);
+          if (issued & (1u << sl)) mbar_wait_drain(full(sl), (issue_par >> sl) & 1u, p.status);
       }
     }
   } else if (warp == 1) {
@@ -469,7 +463,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (!ok && any) {
         tc_commit(drain_bar);
-        wait_drain(drain_bar, 0);
+        mbar_wait_drain(drain_bar, 0, p.status);
       }
     }
   } else {
@@ -703,13 +697,8 @@ cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensor
                       const CUtensorMap& k2, const CUtensorMap& v2, const AttnParams& p, dim3 grid,
                       cudaStream_t s) {
   constexpr int smem = Smem<HD>::TOTAL;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<HD, UPD>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  const cudaError_t ea = ensure_smem_attr<attn_tc_kernel<HD, UPD>>(smem);
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(NTHREADS);

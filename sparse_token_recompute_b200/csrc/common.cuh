@@ -155,6 +155,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
+// Bounded wait used while draining after an abort (it ignores the abort flag):
+// when the phase does not complete within the limit, DEV_TIMEOUT is raised so
+// that a drain which runs out is always reported.
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      raise_status(status, DEV_TIMEOUT);
+      return;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {

@@ -92,14 +92,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// bounded wait that ignores the abort flag (used while draining after an abort)
-__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
-  }
-}
-
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
 // ---------------------------------------------------------------- cluster / DSMEM
@@ -395,7 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         issued |= 1u << i;
       }
       if (npre > 0 && (int)blockIdx.x >= n_units) {
-        for (int i = 0; i < npre; ++i) mbar_wait_drain(full_bar(i), 0);
+        for (int i = 0; i < npre; ++i) mbar_wait_drain(full_bar(i), 0, p.status);
         npre = 0;
       }
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -424,7 +416,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) {
         // drain: every load this thread issued must land before the block exits
         for (int s = 0; s < STAGES; ++s)
-          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (issue_phase >> s) & 1u);
+          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (issue_phase >> s) & 1u, p.status);
       }
     }
   } else if (warp == 1) {
@@ -475,7 +467,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok && issued_any) {
         tc_commit(drain_bar);
-        mbar_wait_drain(drain_bar, 0);
+        mbar_wait_drain(drain_bar, 0, p.status);
       }
     }
   } else {
@@ -781,11 +773,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (ok) {
         // every stage's last release (a commit of CTA 0 arriving here) has landed
         for (int s = 0; s < STAGES; ++s)
-          if (issued & (1u << s)) mbar_wait_drain(empty_bar(s), (issue_phase >> s) & 1u);
+          if (issued & (1u << s)) mbar_wait_drain(empty_bar(s), (issue_phase >> s) & 1u, p.status);
       } else {
         // every load this thread issued lands before the block exits
         for (int s = 0; s < STAGES; ++s)
-          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (issue_phase >> s) & 1u);
+          if (issued & (1u << s)) mbar_wait_drain(full_bar(s), (issue_phase >> s) & 1u, p.status);
       }
     }
   } else if (warp == 1) {
@@ -853,7 +845,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (!ok && issued_any) {
         tc_commit_pair_local(drain_bar);
-        mbar_wait_drain(drain_bar, 0);
+        mbar_wait_drain(drain_bar, 0, p.status);
       }
     }
   } else {
@@ -911,13 +903,8 @@ template <int BN, int EPI>
 cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                      const CUtensorMap& b2, const Params& p, int grid, cudaStream_t s) {
   constexpr size_t smem = smem_bytes_for(BN);
-  static bool attr_set = false;  // per template instance; device-wide attribute
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t ea = ensure_smem_attr<gemm_tc_kernel<BN, EPI>>((int)smem);
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -948,14 +935,8 @@ cudaError_t launch_t(const CUtensorMap& a, const CUtensorMap& b0, const CUtensor
 template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                         const CUtensorMap& b2, const Params& p, int grid, cudaStream_t s) {
-  static bool attr_set = false;  // per template instance; device-wide attribute
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_pair_kernel<EPI>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)PAIR_SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t ea = ensure_smem_attr<gemm_pair_kernel<EPI>>((int)PAIR_SMEM);
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -990,23 +971,13 @@ cudaError_t launch_bn(int bn, const CUtensorMap& a, const CUtensorMap& b0, const
 
 }  // namespace
 
-// programmatic dependent launch (GEMMs, norms, attention); DLLM_PDL=0 turns it off
-bool pdl_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("DLLM_PDL");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
-
-// CTA-pair GEMM for tensor-bound shapes; DLLM_GEMM_PAIR=0 keeps single-CTA tiles
-bool pair_enabled() {
-  static const bool on = [] {
-    const char* e = getenv("DLLM_GEMM_PAIR");
-    return !(e && e[0] == '0');
-  }();
-  return on;
-}
+// CTA-pair GEMM for tensor-bound shapes; a build with -DDLLM_BUILD_NO_PAIR keeps
+// single-CTA tiles (an experiment switch of the build, not a run-time one)
+#ifdef DLLM_BUILD_NO_PAIR
+constexpr bool pair_enabled() { return false; }
+#else
+constexpr bool pair_enabled() { return true; }
+#endif
 
 int gemm_total_cols(const GemmSpec& g) {
   int n = 0;

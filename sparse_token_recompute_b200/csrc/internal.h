@@ -7,10 +7,28 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace dllm {
 
 int num_sms();
 cudaError_t last_error();
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) is a per-device setting of a
+// kernel: set it once for each device the kernel is launched on (one bit per
+// device ordinal below 64; higher ordinals set it on every launch).
+template <auto Kernel>
+cudaError_t ensure_smem_attr(int bytes) {
+  static std::atomic<unsigned long long> done{0ull};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // ----- kernel timing (dllm_profile_*) -----
 void prof_begin(const char* name, cudaStream_t s);
@@ -64,9 +82,15 @@ struct GemmSpec {
   int stall_test;
 };
 
-// launch kernels with programmatic stream serialization (they griddepcontrol.wait
-// before reading what earlier kernels wrote); DLLM_PDL=0 turns it off
-bool pdl_enabled();
+// Kernels launch with programmatic stream serialization (they griddepcontrol.wait
+// before reading what earlier kernels wrote).  A build with -DDLLM_BUILD_NO_PDL
+// launches them plainly (an experiment switch of the build, not a run-time one).
+#ifdef DLLM_BUILD_NO_PDL
+constexpr bool kPdl = false;
+#else
+constexpr bool kPdl = true;
+#endif
+inline bool pdl_enabled() { return kPdl; }
 
 struct GemmPlan {
   int bn, splits, tiles_n, m_tiles_cap, units_cap, grid;
@@ -145,11 +169,6 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
                                     const __nv_bfloat16* k_old, const __nv_bfloat16* v_old,
                                     const int* a_off, int A_cap, int B, int Hq, int Hkv, int hd,
                                     int* status, cudaStream_t s);
-// warp-level MMA flash attention (mma.sync), kept for comparison
-void launch_attention_bf16(const __nv_bfloat16* q, const __nv_bfloat16* kc,
-                           const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
-                           int B, int k_cap, int Nseq, int Hq, int Hkv, int hd,
-                           cudaStream_t s);
 
 // ----- score / select / unmask -----
 template <typename T>
@@ -186,12 +205,14 @@ void launch_unmask(const float* conf, const int32_t* pred, int32_t* tokens, int 
                    int pos_cap, int32_t* pos_out, const int32_t* forced, cudaStream_t s);
 void launch_block_start(const int32_t* tokens, int B, int N, int mask_id, int gen_start,
                         int block_len, int32_t* out, cudaStream_t s);
-// DyLLM FFN gate: flag rows whose attention output moved (1 - cos > tau, or all rows),
-// refresh the context cache, compact the salient rows (list, inverse map, count)
+// DyLLM FFN gate: flag rows whose attention output moved (1 - cos > tau, or all rows,
+// or forced[r] != 0 when forced is given), refresh the context cache, compact the
+// salient rows (list, inverse map, count)
 template <typename T>
 void launch_ffn_gate(const T* o, T* ctx, const int* row_pos, const int* row_seq,
                      const int* M_dev, int M_cap, int N, int q, float tau, int all_rows,
-                     int* flag, int* list, int* inv, int* n_sal, cudaStream_t s);
+                     const uint8_t* forced, int* flag, int* list, int* inv, int* n_sal,
+                     cudaStream_t s);
 // x[r] += FFN output: the new one of a salient row (cached too) or the cached one
 template <typename T>
 void launch_ffn_combine(T* x, const T* f_new, T* f_cache, const int* inv, const int* row_pos,

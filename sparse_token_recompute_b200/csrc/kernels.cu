@@ -950,6 +950,7 @@ __global__ void __launch_bounds__(256) ffn_gate_kernel(const T* __restrict__ o, 
                                                        const int* __restrict__ row_seq,
                                                        const int* __restrict__ M_dev, int M_cap,
                                                        int N, int q, float tau, int all_rows,
+                                                       const uint8_t* __restrict__ forced,
                                                        int* __restrict__ flag) {
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -960,7 +961,7 @@ __global__ void __launch_bounds__(256) ffn_gate_kernel(const T* __restrict__ o, 
   const float v = row_variation<T>(a, c, q, DLLM_SCORE_COS, lane);
   __syncwarp();
   for (int i = lane; i < q; i += 32) c[i] = a[i];
-  if (lane == 0) flag[r] = (all_rows || v > tau) ? 1 : 0;
+  if (lane == 0) flag[r] = (all_rows || (forced ? forced[r] != 0 : v > tau)) ? 1 : 0;
 }
 
 // rows r < M with flag[r] -> list (ascending) and count; inv[r] = position in the
@@ -1320,18 +1321,21 @@ void launch_row_map_dense(int B, int N, int* row_off, int* row_pos, int* row_seq
 template <typename T>
 void launch_ffn_gate(const T* o, T* ctx, const int* row_pos, const int* row_seq,
                      const int* M_dev, int M_cap, int N, int q, float tau, int all_rows,
-                     int* flag, int* list, int* inv, int* n_sal, cudaStream_t s) {
+                     const uint8_t* forced, int* flag, int* list, int* inv, int* n_sal,
+                     cudaStream_t s) {
   if (M_cap <= 0) return;
   ProfScope prof("ffn_gate", s);
   ffn_gate_kernel<T><<<(M_cap + 7) / 8, 256, 0, s>>>(o, ctx, row_pos, row_seq, M_dev, M_cap, N, q,
-                                                     tau, all_rows, flag);
+                                                     tau, all_rows, forced, flag);
   flag_compact_kernel<<<1, 1024, 0, s>>>(flag, M_dev, M_cap, list, inv, n_sal);
 }
 template void launch_ffn_gate<float>(const float*, float*, const int*, const int*, const int*, int,
-                                     int, int, float, int, int*, int*, int*, int*, cudaStream_t);
+                                     int, int, float, int, const uint8_t*, int*, int*, int*, int*,
+                                     cudaStream_t);
 template void launch_ffn_gate<__nv_bfloat16>(const __nv_bfloat16*, __nv_bfloat16*, const int*,
                                              const int*, const int*, int, int, int, float, int,
-                                             int*, int*, int*, int*, cudaStream_t);
+                                             const uint8_t*, int*, int*, int*, int*,
+                                             cudaStream_t);
 
 template <typename T>
 void launch_ffn_combine(T* x, const T* f_new, T* f_cache, const int* inv, const int* row_pos,
@@ -1463,12 +1467,7 @@ void launch_attention_f32(const float* q, const float* kc, const float* vc, floa
   if (M_cap <= 0) return;
   ProfScope prof("attention_f32", s);
   const size_t smem = (size_t)Nseq * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(attention_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         64 * 1024);
-    attr = true;
-  }
+  if (ensure_smem_attr<attention_f32_kernel>(64 * 1024) != cudaSuccess) return;
   dim3 grid(M_cap, Hq);
   attention_f32_kernel<<<grid, 128, smem, s>>>(q, kc, vc, o, row_seq, M_dev, M_cap, Nseq, Hq, Hkv,
                                                hd);

@@ -121,3 +121,27 @@ def test_gemm_plan_rejects_bad_arguments(lib):
     assert S._gemm_plan(3, 100, 64, C.cast(segs, C.c_void_p), 1, 128, C.cast(out, C.c_void_p)) == 1
     assert S._gemm_plan(0, 0, 64, C.cast(segs, C.c_void_p), 1, 0, C.cast(out, C.c_void_p)) == 1
     assert S._gemm_plan(0, 100, 64, None, 1, 0, C.cast(out, C.c_void_p)) == 1
+
+
+def test_host_buffer_step_validates_before_any_copy(lib):
+    """dllm_step_host rejects a missing token buffer, a bad shape and a small
+    workspace before it enqueues a copy; its workspace adds the token and
+    revealed-position buffers to the step's."""
+    import sparse_token_recompute_b200 as S
+    cfg = S.make_cfg(1, 256, 4, 4, 64, 688, 1024, 5e5, 1e-5, 1023, "f32")
+    pol = S.make_policy(k=32, n_unmask=8, gen_start=64, block_len=64)
+    step = S.dllm_step_workspace_size(cfg, 2, 128, pol)
+    host = S.dllm_step_host_workspace_size(cfg, 2, 128, pol)
+    assert host >= step + 2 * 128 * 4 + 2 * 8 * 4
+    m = S.ModelW()
+    c = S.CacheS()
+    tok = (C.c_int32 * 256)()
+    assert S._step_host(C.byref(cfg), C.byref(m), C.byref(c), None, 2, 128, C.byref(pol), 0,
+                        None, None, 0, None) == 1
+    assert S._step_host(C.byref(cfg), C.byref(m), C.byref(c), C.cast(tok, C.c_void_p), -1, 128,
+                        C.byref(pol), 0, None, None, 0, None) == 1
+    assert S._step_host(C.byref(cfg), C.byref(m), C.byref(c), C.cast(tok, C.c_void_p), 2, 128,
+                        C.byref(pol), 0, None, None, 0, None) == 3
+    bad = S.make_cfg(1, 256, 4, 3, 64, 688, 1024, 5e5, 1e-5, 1023, "f32")
+    assert S._step_host(C.byref(bad), C.byref(m), C.byref(c), C.cast(tok, C.c_void_p), 2, 128,
+                        C.byref(pol), 0, None, None, 0, None) == 2

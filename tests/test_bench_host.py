@@ -82,3 +82,32 @@ def test_hbm_kernels_by_hand():
     assert r["select"]["bound"] == "latency"
     assert "attention" not in r
     assert bench.hbm_kernels(s, {}, 6550.0) == {"peak_gbs": 6550.0}
+
+
+def test_generation_from_sample_by_hand():
+    """Whole generation = dense step + 63 partial steps, each 32 sequences x 32 layers
+    of the one-sequence one-layer sample plus the sequence's LM head."""
+    s = bench.SHAPE
+    gen, dense, partial = bench.generation_from_sample(s, 0.5, 0.25, 2.0, 1.5)
+    assert dense == 32 * (32 * 2.0 + 1.5)
+    assert partial == 32 * (32 * 0.5 + 0.25)
+    assert gen == dense + 63 * partial
+
+
+def test_clock_summaries_merge(tmp_path):
+    """Samples of several windows summarise as one: median SM clock of the loaded
+    samples, every throttle reason seen."""
+    rows = [
+        ["0, u, 1400, 1965, 900, 0x4, Not Active, Not Active, Not Active, Active",
+         "0, u, 1500, 1965, 950, 0x0, Not Active, Not Active, Not Active, Not Active"],
+        ["0, u, 1300, 1965, 990, 0x4, Not Active, Not Active, Not Active, Active",
+         "0, u, 210, 1965, 90, 0x0, Not Active, Not Active, Not Active, Not Active"]]
+    cl = []
+    for i, rr in enumerate(rows):
+        c = bench.Clocks("u")
+        c.path = str(tmp_path / f"c{i}.csv")
+        open(c.path, "w").write("\n".join(rr) + "\n")
+        cl.append(c)
+    m = bench.Clocks.merge(cl)
+    assert m["samples"] == 4 and m["sm_mhz"] == 1400.0 and m["reasons"] == ["sw_power_cap"]
+    assert cl[1].summary()["sm_mhz"] == 1300.0    # the idle 210 MHz sample is not under load

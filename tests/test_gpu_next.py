@@ -351,3 +351,102 @@ def test_ffn_gate_fixed_point_bf16(lib):
     assert rows.cpu().tolist() == [0] * r.ocfg.n_layers
     for a, b in zip(kv0, r.cache.k + r.cache.v):
         assert max_abs_rel(f64(b), f64(a)) < TOL["bf16"]
+
+
+def _gated_mixed_forced(lib, shape, tau, tol, steps):
+    """The gate at a threshold that splits the recomputed rows (DyLLM, French
+    summary §2.A): the oracle decides every row of every layer, the GPU takes
+    those decisions (forced_ffn, as forced_idx does for the selection), and the
+    caches -- K/V, contexts, FFN outputs -- are compared after each step."""
+    r = _gated_run(lib, shape, tau)
+    L = r.ocfg.n_layers
+    mixed = 0
+    for t in range(steps):
+        out = O.step(r.ocfg, r.ow, r.st, r.opol, dense=(t == 0))
+        rows = torch.full((L,), -1, dtype=torch.int32, device="cuda")
+        io = {"forced_unmask_pos": _pad(out.unmasked, out.unmasked.shape[1]), "ffn_rows_out": rows}
+        if t > 0:
+            io.update(forced_idx=_pad(out.idx, r.k_cap),
+                      forced_count=torch.tensor([len(a) for a in out.idx], dtype=torch.int32,
+                                                device="cuda"))
+            fz = np.zeros((L, r.B * r.k_cap), dtype=np.uint8)
+            first = L - len(out.ffn_salient)
+            for j, sal in enumerate(out.ffn_salient):
+                fz[first + j, :len(sal)] = sal
+                mixed += int(0 < int(sal.sum()) < len(sal))
+            io["forced_ffn"] = torch.from_numpy(fz).cuda()
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, t == 0, r.ws, **io)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        assert rows.cpu().tolist() == out.ffn_rows
+        r.compare_state(tol, out.final_rows, out.idx)
+        for l in range(L):
+            assert max_abs_rel(f64(r.cache.ctx[l]), r.st.ctx[l]) < tol, ("ctx", l)
+            assert max_abs_rel(f64(r.cache.ffn[l]), r.st.ffn[l]) < tol, ("ffn", l)
+        r.tokens.copy_(torch.from_numpy(r.st.tokens.astype(np.int32)))
+    assert mixed > 0   # some layer-step ran the FFN on part of its rows only
+
+
+def test_ffn_gate_mixed_threshold_bf16_forced(lib):
+    _gated_mixed_forced(lib, _small_bf16(), 1e-3, TOL["bf16"], 4)
+
+
+def test_ffn_gate_mixed_threshold_tiny_f32_forced(lib):
+    _gated_mixed_forced(lib, SY.with_(SY.TINY, n_layers=2), 1e-2, TOL["f32"], 4)
+
+
+def test_ffn_gate_own_decisions_follow_the_rule(lib):
+    """The GPU's own gate at a mixed threshold: in every layer of every partial
+    step, a recomputed row ran the FFN (its cached FFN output changed) exactly
+    when 1 - cos(its new context, its previous context) > tau, evaluated here in
+    float64 on the contexts the GPU stored; rows within 1e-5 of tau (where the
+    kernel's fp32 cosine may fall on either side) are only counted."""
+    tau, band = 1e-3, 1e-5
+    shape = _small_bf16()
+    r = _gated_run(lib, shape, tau)
+    L, B = r.ocfg.n_layers, r.B
+    lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, True, r.ws)
+    mixed = 0
+    for t in range(1, 4):
+        ctx0 = [f64(c) for c in r.cache.ctx]
+        ffn0 = [c.clone() for c in r.cache.ffn]
+        idx = torch.full((B, r.k_cap), -1, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+        rows = torch.full((L,), -1, dtype=torch.int32, device="cuda")
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, False, r.ws, idx_out=idx,
+                         count_out=cnt, ffn_rows_out=rows)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        sel = [(b, int(p)) for b in range(B) for p in idx[b, :int(cnt[b])].cpu().numpy()]
+        bs = np.array([b for b, _ in sel])
+        ps = np.array([p for _, p in sel])
+        for l in range(L):
+            ran = torch.any(r.cache.ffn[l] != ffn0[l], dim=-1).cpu().numpy()[bs, ps]
+            assert int(ran.sum()) == int(rows[l])
+            v = O.variation(f64(r.cache.ctx[l])[bs, ps], ctx0[l][bs, ps], O.SCORE_COS)
+            clear = np.abs(v - tau) > band
+            np.testing.assert_array_equal(ran[clear], (v > tau)[clear])
+            mixed += int(0 < ran.sum() < len(ran))
+    assert mixed > 0
+
+
+def test_step_host_equals_device_step(lib):
+    """dllm_step_host (token state in pinned host memory, copied in and out by the
+    library on the stream) reproduces dllm_step on device tokens bit for bit."""
+    shape = _small_bf16()
+    r1, r2 = Run(lib, shape), Run(lib, shape)
+    cap = max(lib.dllm_unmask_capacity(r1.pol), 1)
+    ws_h = lib.Workspace(lib.dllm_step_host_workspace_size(r2.model.cfg, r2.B, r2.N, r2.pol))
+    tok_h = r2.tokens.cpu().pin_memory()
+    pos_h = torch.full((r2.B, cap), -9, dtype=torch.int32).pin_memory()
+    for t in range(4):
+        pos = torch.full((r1.B, cap), -9, dtype=torch.int32, device="cuda")
+        lib.dllm_step(r1.model, r1.cache, r1.tokens, r1.pol, t == 0, r1.ws, pos_out=pos)
+        lib.dllm_step_host(r2.model, r2.cache, tok_h, r2.pol, t == 0, ws_h, pos_h)
+        torch.cuda.synchronize()
+        assert torch.equal(r1.tokens.cpu(), tok_h)
+        assert torch.equal(pos.cpu(), pos_h)
+    assert ws_h.device_status() == 0
+    for a, b in zip(r1.cache.k + r1.cache.v + [r1.cache.h_ref, r1.cache.conf, r1.cache.pred],
+                    r2.cache.k + r2.cache.v + [r2.cache.h_ref, r2.cache.conf, r2.cache.pred]):
+        assert torch.equal(a, b)

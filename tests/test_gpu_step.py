@@ -14,7 +14,7 @@ import torch
 
 import oracle as O
 import dllm_synth as SY
-from _util import f64, max_abs_rel, TOL, oracle_policy
+from _util import f64, max_abs_rel, TOL, oracle_cfg, oracle_policy
 from _gpu import build, oracle_w_from, argmax_ok
 
 pytestmark = pytest.mark.gpu
@@ -22,10 +22,17 @@ GOLD = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 class Run:
-    def __init__(self, lib, shape, seed=0, **pol_kw):
+    def __init__(self, lib, shape, seed=0, prebuilt=None, **pol_kw):
+        """prebuilt: (host weights, oracle weights, device weights) of this shape, to
+        share one draw of the weights among several runs."""
         self.lib, self.s = lib, shape
-        self.model, self.ocfg, Wd, Wh = build(shape, seed=seed)
-        self.ow = oracle_w_from(Wh)
+        if prebuilt is None:
+            self.model, self.ocfg, Wd, Wh = build(shape, seed=seed)
+            self.ow = oracle_w_from(Wh)
+        else:
+            Wh, self.ow, Wd = prebuilt
+            self.model = lib.Model(lib.cfg_from_shape(shape), Wd)
+            self.ocfg = oracle_cfg(shape)
         B, N = shape.batch, shape.seq_len
         tok = SY.prompt_tokens(shape, seed=1)
         self.tokens = tok.cuda()
