@@ -84,6 +84,15 @@ in the design notes):
     out of the softmax sums and their new terms put in (reference max raised
     to cover the new scores).  Exact when the query is current; DyLLM's
     approximation when the query is stale.
+  * Approximate attention inside a step [DyLLM §2.B], with the FFN gate on:
+    in every layer a partial step recomputes, the rows it does not recompute
+    (stable rows) keep the query, softmax statistics and attention output of
+    their last pass (per-layer caches q, m, l and the context cache) and
+    receive the incremental update from the keys the step changed in that
+    layer (the recomputed rows' old and new K/V).  The updated output is
+    their context C_{t,l} (the FFN gate's reference for later steps); their
+    hidden states and K/V stay cached.  Recomputed rows write their query and
+    exact statistics into the caches; a dense step writes them for every row.
   * Periodic refresh [ES-nl Methodologie 3]: in a generation, a step is
     dense (every row recomputed, every cache rewritten) at step 0, every
     refresh_every steps, and, with refresh_on_block, at the first step at
@@ -216,6 +225,7 @@ class Policy:
     select_from: int = 0          # positions below it are never selected (partial steps)
     ffn_gate: bool = False        # DyLLM FFN gating on the attention context
     ffn_tau: float = 0.0          # salient when 1 - cos(context, cached context) > ffn_tau
+    attn_update: bool = False     # DyLLM approximate attention of stable rows (needs ffn_gate)
     unmask_tau: float = 0.0       # > 0: over-threshold unmasking with top-n fallback
     refresh_every: int = 0        # generation: dense step every R steps (0: never)
     refresh_on_block: bool = False  # generation: dense step when a block changes
@@ -233,6 +243,11 @@ class State:
     h_ref2: Optional[np.ndarray] = None  # [B, N, d] hidden at the second skip point
     ctx: Optional[List[np.ndarray]] = None  # per layer [B, N, Hq*hd] attention output
     ffn: Optional[List[np.ndarray]] = None  # per layer [B, N, d] FFN output
+    # approximate attention: per layer the query [B, N, Hq*hd] of each row's last exact
+    # pass and its softmax statistics m, l [B, N, Hq] (natural log), kept up to date
+    q: Optional[List[np.ndarray]] = None
+    att_m: Optional[List[np.ndarray]] = None
+    att_l: Optional[List[np.ndarray]] = None
 
     def copy(self) -> "State":
         cp = lambda a: None if a is None else [x.copy() for x in a]
@@ -240,7 +255,7 @@ class State:
                      [a.copy() for a in self.v], self.h_ref.copy(),
                      self.conf.copy(), self.pred.copy(),
                      None if self.h_ref2 is None else self.h_ref2.copy(), cp(self.ctx),
-                     cp(self.ffn))
+                     cp(self.ffn), cp(self.q), cp(self.att_m), cp(self.att_l))
 
 
 def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
@@ -252,7 +267,10 @@ def empty_state(cfg: ModelCfg, tokens: np.ndarray) -> State:
                  np.zeros((B, N, cfg.d)), np.zeros((B, N)),
                  np.zeros((B, N), dtype=np.int64), np.zeros((B, N, cfg.d)),
                  [np.zeros((B, N, cfg.n_heads * cfg.head_dim)) for _ in range(cfg.n_layers)],
-                 [np.zeros((B, N, cfg.d)) for _ in range(cfg.n_layers)])
+                 [np.zeros((B, N, cfg.d)) for _ in range(cfg.n_layers)],
+                 [np.zeros((B, N, cfg.n_heads * cfg.head_dim)) for _ in range(cfg.n_layers)],
+                 [np.zeros((B, N, cfg.n_heads)) for _ in range(cfg.n_layers)],
+                 [np.zeros((B, N, cfg.n_heads)) for _ in range(cfg.n_layers)])
 
 
 # ---------------------------------------------------------------------------
@@ -385,6 +403,11 @@ class FfnGate:
     tau: float
     all_rows: bool = False
     salient: Optional[np.ndarray] = None
+    # approximate attention of the layer's stable rows (None: off): the query and
+    # softmax statistics caches [B, N, .] of the layer
+    q: Optional[np.ndarray] = None
+    att_m: Optional[np.ndarray] = None
+    att_l: Optional[np.ndarray] = None
 
 
 def layer_rows(cfg: ModelCfg, w: LayerW, x: np.ndarray, b_of_row: np.ndarray,
@@ -406,12 +429,32 @@ def layer_rows(cfg: ModelCfg, w: LayerW, x: np.ndarray, b_of_row: np.ndarray,
     k = rope((n @ w.wk.T).reshape(R, Hkv, hd), pos_of_row, cfg.rope_theta)
     v = (n @ w.wv.T).reshape(R, Hkv, hd)
     q, k, v = store(q, dt), store(k, dt), store(v, dt)
+    upd = gate is not None and gate.q is not None
+    if upd:
+        k_old, v_old = k_cache[b_of_row, pos_of_row], v_cache[b_of_row, pos_of_row]
     k_cache[b_of_row, pos_of_row] = k
     v_cache[b_of_row, pos_of_row] = v
     o = np.empty((R, Hq, hd))
     for b in np.unique(b_of_row):
         rows = np.nonzero(b_of_row == b)[0]
-        o[rows] = attention(q[rows], k_cache[b], v_cache[b])
+        if not upd:
+            o[rows] = attention(q[rows], k_cache[b], v_cache[b])
+            continue
+        m_b, l_b, o[rows] = attention_stats(q[rows], k_cache[b], v_cache[b])
+        # DyLLM §2.B: the sequence's stable rows reuse their attention and take in
+        # only the changed keys (their old terms out, their new terms in)
+        N = k_cache.shape[1]
+        stable = np.setdiff1d(np.arange(N), pos_of_row[rows])
+        if len(stable):
+            m2, l2, o2 = attention_update(gate.q[b, stable].reshape(-1, Hq, hd),
+                                          gate.att_m[b, stable], gate.att_l[b, stable],
+                                          gate.ctx[b, stable].reshape(-1, Hq, hd),
+                                          k_old[rows], v_old[rows], k[rows], v[rows])
+            gate.att_m[b, stable], gate.att_l[b, stable] = m2, l2
+            gate.ctx[b, stable] = store(o2.reshape(len(stable), Hq * hd), dt)
+        # the recomputed rows' query and exact statistics, for later updates
+        gate.q[b, pos_of_row[rows]] = q[rows].reshape(len(rows), Hq * hd)
+        gate.att_m[b, pos_of_row[rows]], gate.att_l[b, pos_of_row[rows]] = m_b, l_b
     o = store(o.reshape(R, Hq * hd), dt)
     x = store(x + o @ w.wo.T, dt)
     n2 = store(rms_norm(x, w.ffn_norm, cfg.rms_eps), dt)
@@ -703,6 +746,8 @@ def step(cfg: ModelCfg, W: ModelW, st: State, pol: Policy, dense: bool,
             st.h_ref2[b_of, p_of] = x
         if len(b_of):
             gate = FfnGate(st.ctx[l], st.ffn[l], pol.ffn_tau, dense) if pol.ffn_gate else None
+            if gate is not None and pol.attn_update:
+                gate.q, gate.att_m, gate.att_l = st.q[l], st.att_m[l], st.att_l[l]
             x = layer_rows(cfg, W.layers[l], x, b_of, p_of, st.k[l], st.v[l], gate)
             if gate is not None:
                 ffn_rows.append(int(np.sum(gate.salient)))

@@ -18,6 +18,11 @@
   old and new terms equals the attention over the updated keys computed
   directly; no change, every key changed and a key replaced by itself are
   the limits.
+* Approximate attention inside a step (DyLLM, French summary §2.B): after
+  any run of dense and partial steps, every row's cached context equals the
+  attention of its cached query over the current K/V caches computed afresh,
+  and its cached (m, l) are that attention's max and sum; with every row
+  salient for the FFN the update changes nothing but the stable rows' caches.
 * FFN gating on the attention context (DyLLM, French summary §2.A): every
   row salient is the plain layer; no row salient adds the cached FFN output
   to the post-attention residual (taken from the same model with its FFN
@@ -31,7 +36,7 @@ import pytest
 
 import oracle as O
 from dllm_synth import TINY, with_, model_weights, prompt_tokens
-from _util import oracle_cfg, oracle_weights, oracle_policy, f64
+from _util import oracle_cfg, oracle_weights, oracle_policy, f64, max_abs_rel
 
 RT = 1e-10
 
@@ -409,3 +414,62 @@ def test_ffn_gate_threshold_splits_rows_by_context_change():
     # with tau 0 exactly the rows whose context moved at all run the FFN: in the first
     # recomputed layer every selected row sees the four changed keys
     assert 0 < out.ffn_rows[0] <= 32
+
+
+
+# ----------------------------------------------------------------- approximate attention step
+
+
+def _cached_attention_holds(cfg, st, tol):
+    """Every row's cached context / statistics against a fresh attention of its
+    cached query over the layer's K/V caches."""
+    Hq, hd = cfg.n_heads, cfg.head_dim
+    B, N = st.tokens.shape
+    for l in range(cfg.n_layers):
+        for b in range(B):
+            q = st.q[l][b].reshape(N, Hq, hd)
+            m, lsum, o = O.attention_stats(q, st.k[l][b], st.v[l][b])
+            assert np.max(np.abs(st.ctx[l][b] - o.reshape(N, -1))) < tol * np.abs(o).max()
+            lse = st.att_m[l][b] + np.log(st.att_l[l][b])
+            assert np.max(np.abs(lse - (m + np.log(lsum)))) < tol * np.abs(m).max()
+
+
+@pytest.mark.parametrize("tau", [-1.0, 1e-2])
+def test_approximate_attention_tracks_the_caches(tau):
+    """Stable rows keep their query, so their exactly updated statistics must be
+    those of the attention over the updated keys: the invariant holds after the
+    dense step and after every partial step (f32: no rounding anywhere)."""
+    s, cfg, W, tok = _setup(n_layers=2)
+    st = O.empty_state(cfg, tok)
+    pol = oracle_policy(s, ffn_gate=True, ffn_tau=tau, attn_update=True)
+    for t in range(5):
+        out = O.step(cfg, W, st, pol, dense=(t == 0))
+        _cached_attention_holds(cfg, st, 1e-9)
+    assert sum(len(a) for a in out.idx) < tok.size    # stable rows existed
+
+
+def test_approximate_attention_touches_only_the_stable_rows_caches():
+    """With every row salient for the FFN, decisions never read the contexts, so
+    a run with the update and one without agree on tokens, K/V, references,
+    confidences, predictions and FFN outputs, and on the recomputed rows'
+    contexts (up to the summation order of the two attention routines, 1e-10);
+    only stable rows' contexts differ."""
+    s, cfg, W, tok = _setup(n_layers=2)
+    st1, st2 = O.empty_state(cfg, tok), O.empty_state(cfg, tok)
+    p1 = oracle_policy(s, ffn_gate=True, ffn_tau=-1.0, attn_update=True)
+    p2 = oracle_policy(s, ffn_gate=True, ffn_tau=-1.0)
+    moved = 0
+    for t in range(4):
+        o1 = O.step(cfg, W, st1, p1, dense=(t == 0))
+        o2 = O.step(cfg, W, st2, p2, dense=(t == 0))
+        np.testing.assert_array_equal(st1.tokens, st2.tokens)
+        np.testing.assert_array_equal(st1.pred, st2.pred)
+        for a, b in zip(st1.k + st1.v + st1.ffn + [st1.h_ref, st1.conf],
+                        st2.k + st2.v + st2.ffn + [st2.h_ref, st2.conf]):
+            assert max_abs_rel(a, b) < RT
+        for l in range(cfg.n_layers):
+            for b, idx in enumerate(o1.idx):
+                assert max_abs_rel(st1.ctx[l][b, idx], st2.ctx[l][b, idx]) < RT
+                rest = np.setdiff1d(np.arange(tok.shape[1]), idx)
+                moved += int(max_abs_rel(st1.ctx[l][b, rest], st2.ctx[l][b, rest]) > 1e-6)
+    assert moved > 0
