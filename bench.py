@@ -425,6 +425,43 @@ def ffn_gate_measure(S, model, shape, rank, steps, warmup):
     return out
 
 
+def dyllm_measure(S, model, shape, rank, steps, warmup, tau=1e-3):
+    """DyLLM's mechanisms on a workload: partial steps with the FFN gate at tau
+    (French summary §2.A), and with the gate plus the approximate attention of
+    the stable rows (§2.B: every row not recomputed takes in the changed keys)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, upd in (("ffn_gate", False), ("ffn_gate_and_approx_attention", True)):
+        tokens = SY.prompt_tokens(shape, seed=1 + rank, device="cuda")
+        cache = S.Cache(model.cfg, shape.batch, shape.seq_len, ffn_gate=True, attn_update=upd)
+        pol = S.make_policy(score_layer=0, alpha=shape.alpha, k=shape.k, n_unmask=shape.n_unmask,
+                            gen_start=shape.prompt_len, block_len=shape.block_len,
+                            ffn_gate=True, ffn_tau=tau, attn_update=upd)
+        ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+        S.dllm_step_ex(model, cache, tokens, pol, True, ws)
+        for _ in range(warmup):
+            S.dllm_step_ex(model, cache, tokens, pol, False, ws)
+        torch.cuda.synchronize()
+        K = min(steps, 10)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            S.dllm_step_ex(model, cache, tokens, pol, False, ws, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / K
+        out[name] = {"ms_per_step": round(ms, 4),
+                     "tokens_per_s": round(shape.batch * shape.n_unmask * 1000.0 / ms, 2),
+                     "device_status": ws.device_status()}
+        del cache, ws
+        torch.cuda.empty_cache()
+    out["how"] = (f"{shape.batch} x {shape.seq_len} tokens, {shape.k} rows/seq recomputed, FFN "
+                  f"gate at tau {tau:g}; with the approximate attention every other row of "
+                  f"every layer takes in the recomputed rows' K/V changes")
+    return out
+
+
 def _oracle_cfg(shape):
     import oracle as O
     return O.ModelCfg(shape.n_layers, shape.d, shape.n_heads, shape.n_kv_heads, shape.head_dim,
@@ -784,10 +821,16 @@ def run_ours(args):
                                                       args.warmup)
         result["dyllm_ffn_gate"] = ffn_gate_measure(S, model, shape, rank, args.steps,
                                                     args.warmup)
+        result["dyllm_approx_attention"] = {"b32": dyllm_measure(S, model, shape, rank,
+                                                                 args.steps, args.warmup)}
     if not args.no_bs1:
         del cache, ws
         torch.cuda.empty_cache()
         result["bs1"] = bs1_measure(S, W, args.steps, args.warmup, hbm, tc_burst)
+        if world == 1:
+            m1 = S.Model(S.cfg_from_shape(BS1), W)
+            result.setdefault("dyllm_approx_attention", {})["b1"] = dyllm_measure(
+                S, m1, SY.with_(BS1, ratio=0.10), rank, args.steps, args.warmup)
     if not args.no_gqa and world == 1:
         del W, model
         torch.cuda.empty_cache()

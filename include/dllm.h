@@ -133,6 +133,13 @@ typedef struct {
   void* const* ctx;  /* [B, N, n_heads*head_dim] each row's attention output at its
                       * last pass through the layer */
   void* const* ffn;  /* [B, N, d] each row's FFN output at its last salient pass */
+  /* DyLLM approximate attention (policy.attn_update); HOST arrays of n_layers device
+   * pointers, NULL when off: */
+  void* const* q;       /* [B, N, n_heads*head_dim] each row's query (after RoPE) at its
+                         * last exact pass through the layer */
+  float* const* att_m;  /* [B, N, n_heads] f32: softmax statistics of each row's attention */
+  float* const* att_l;  /* [B, N, n_heads] f32: (reference max and sum, natural log units,
+                         * as dllm_attention_stats_bf16), kept up to date by the updates */
 } dllm_cache;
 
 typedef struct {
@@ -164,6 +171,16 @@ typedef struct {
   /* Dense steps run every FFN and fill both caches.                         */
   int ffn_gate;      /* 0: off                                           */
   float ffn_tau;
+  /* Approximate attention of stable rows [DyLLM 2.B] (needs ffn_gate and      */
+  /* DLLM_BF16): in every layer a partial step recomputes, each row it does    */
+  /* not recompute keeps the query and softmax statistics of its last exact    */
+  /* attention (cache.q/att_m/att_l) and its output (cache.ctx) and takes in   */
+  /* only the keys the step changed in that layer: their old terms leave the   */
+  /* sums, their new terms enter (dllm_attention_update_bf16).  The result is  */
+  /* the row's attention context, the FFN gate's reference at its next pass.   */
+  /* Recomputed rows store their query and exact statistics; a dense step     */
+  /* stores them for every row.  Layers below score_layer keep no such state.  */
+  int attn_update;   /* 0: off                                           */
 } dllm_policy;
 
 /* Supported shapes for DLLM_BF16 layer work: d, n_heads*head_dim,

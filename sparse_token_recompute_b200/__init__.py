@@ -55,7 +55,8 @@ class ModelW(C.Structure):
 
 class CacheS(C.Structure):
     _fields_ = [("k", C.POINTER(vp)), ("v", C.POINTER(vp)), ("h_ref", vp), ("conf", vp),
-                ("pred", vp), ("h_ref2", vp), ("ctx", C.POINTER(vp)), ("ffn", C.POINTER(vp))]
+                ("pred", vp), ("h_ref2", vp), ("ctx", C.POINTER(vp)), ("ffn", C.POINTER(vp)),
+                ("q", C.POINTER(vp)), ("att_m", C.POINTER(vp)), ("att_l", C.POINTER(vp))]
 
 
 class Policy(C.Structure):
@@ -64,7 +65,7 @@ class Policy(C.Structure):
                 ("gen_start", C.c_int), ("block_len", C.c_int), ("select_from", C.c_int),
                 ("unmask_tau", C.c_float), ("refresh_every", C.c_int),
                 ("refresh_on_block", C.c_int), ("score_layer2", C.c_int), ("k2", C.c_int),
-                ("ffn_gate", C.c_int), ("ffn_tau", C.c_float)]
+                ("ffn_gate", C.c_int), ("ffn_tau", C.c_float), ("attn_update", C.c_int)]
 
 
 class StepIO(C.Structure):
@@ -418,7 +419,7 @@ class Cache:
     """Per-layer K/V caches, hidden reference, cached confidence and argmax (torch memory)."""
 
     def __init__(self, cfg: ModelCfg, B: int, N: int, device="cuda", second_ref: bool = False,
-                 ffn_gate: bool = False):
+                 ffn_gate: bool = False, attn_update: bool = False):
         import torch
         dt = torch.bfloat16 if cfg.dtype == DLLM_BF16 else torch.float32
         kv = (B, N, cfg.n_kv_heads, cfg.head_dim)
@@ -433,6 +434,13 @@ class Cache:
                     for _ in range(cfg.n_layers)] if ffn_gate else None
         self.ffn = [torch.zeros(B, N, cfg.d, dtype=dt, device=device)
                     for _ in range(cfg.n_layers)] if ffn_gate else None
+        # approximate attention: per layer each row's query and softmax statistics
+        self.q = [torch.zeros(B, N, q, dtype=dt, device=device)
+                  for _ in range(cfg.n_layers)] if attn_update else None
+        self.att_m = [torch.zeros(B, N, cfg.n_heads, dtype=torch.float32, device=device)
+                      for _ in range(cfg.n_layers)] if attn_update else None
+        self.att_l = [torch.zeros(B, N, cfg.n_heads, dtype=torch.float32, device=device)
+                      for _ in range(cfg.n_layers)] if attn_update else None
         self.conf = torch.zeros(B, N, dtype=torch.float32, device=device)
         self.pred = torch.zeros(B, N, dtype=torch.int32, device=device)
         self._refresh()
@@ -443,18 +451,21 @@ class Cache:
         self._vp = (vp * L)(*[ptr(t) for t in self.v])
         self._cp = (vp * L)(*[ptr(t) for t in self.ctx]) if self.ctx else None
         self._fp = (vp * L)(*[ptr(t) for t in self.ffn]) if self.ffn else None
+        self._qp = (vp * L)(*[ptr(t) for t in self.q]) if self.q else None
+        self._mp = (vp * L)(*[ptr(t) for t in self.att_m]) if self.att_m else None
+        self._lp = (vp * L)(*[ptr(t) for t in self.att_l]) if self.att_l else None
         self.s = CacheS(self._kp, self._vp, ptr(self.h_ref), ptr(self.conf), ptr(self.pred),
-                        ptr(self.h_ref2), self._cp, self._fp)
+                        ptr(self.h_ref2), self._cp, self._fp, self._qp, self._mp, self._lp)
 
 
 def make_policy(score_layer=0, alpha=0.5, kind=DLLM_SCORE_COS, mode=DLLM_SELECT_TOPK, k=1,
                 tau=0.0, n_unmask=1, gen_start=0, block_len=32, select_from=0, unmask_tau=0.0,
                 refresh_every=0, refresh_on_block=False, score_layer2=0, k2=0, ffn_gate=False,
-                ffn_tau=0.0) -> Policy:
+                ffn_tau=0.0, attn_update=False) -> Policy:
     return Policy(score_layer, float(alpha), kind, mode, k, float(tau), n_unmask, gen_start,
                   block_len, int(select_from), float(unmask_tau), int(refresh_every),
                   int(bool(refresh_on_block)), int(score_layer2), int(k2), int(bool(ffn_gate)),
-                  float(ffn_tau))
+                  float(ffn_tau), int(bool(attn_update)))
 
 
 def dllm_partial_layer_workspace_size(cfg: ModelCfg, B: int, N: int, k_cap: int) -> int:

@@ -255,10 +255,27 @@ struct LayerGate {
   int32_t* rows_out;  // this layer's salient-row count (device), or null
 };
 
+// DyLLM approximate attention of one layer (dllm_policy.attn_update): caches of the
+// rows' queries and softmax statistics, and the scratch of the stable-row update
+struct LayerUpd {
+  void* q_cache;   // [B, N, q] query of each row's last exact pass
+  float* m_cache;  // [B, N, Hq] softmax statistics (natural log units)
+  float* l_cache;
+  bool partial;    // partial step: stable rows take in the changed keys
+  float* m_c;      // [cap, Hq] exact statistics of the recomputed rows
+  float* l_c;
+  void* k_old;     // [cap, kv] the recomputed rows' K/V before and after the layer
+  void* v_old;
+  void* k_new;
+  void* v_new;
+  uint8_t* skip;   // [B, N] 1 at the recomputed rows
+  int* seq_off;    // [B + 1] b * N
+};
+
 dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void* x, int M_cap,
                           const int* M_dev, const LayerWs& w, int B, int N, int k_cap,
                           void* k_cache, void* v_cache, bool use_rope, cudaStream_t s,
-                          const LayerGate* gate = nullptr) {
+                          const LayerGate* gate = nullptr, const LayerUpd* upd = nullptr) {
   const int d = c->d, q = c->n_heads * c->head_dim, kv = c->n_kv_heads * c->head_dim;
   const int F = c->ffn, hd = c->head_dim;
   const float2* rope = use_rope ? w.rope : nullptr;
@@ -267,6 +284,12 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
     using bf = __nv_bfloat16;
     bf* xb = static_cast<bf*>(x);
     bf* nb = static_cast<bf*>(w.n);
+    if (upd && upd->partial) {  // the recomputed rows' K/V before this layer rewrites them
+      launch_row_words(k_cache, upd->k_old, w.row_pos, w.row_seq, M_dev, M_cap, N, kv * 2, false,
+                       s);
+      launch_row_words(v_cache, upd->v_old, w.row_pos, w.row_seq, M_dev, M_cap, N, kv * 2, false,
+                       s);
+    }
     launch_rmsnorm<bf>(xb, static_cast<const bf*>(lw->attn_norm), nb, M_dev, M_cap, d,
                        c->rms_eps, s);
     GemmSpec g{};
@@ -297,9 +320,37 @@ dllm_status layer_forward(const dllm_model_cfg* c, const dllm_layer_w* lw, void*
                                    static_cast<const bf*>(k_cache),
                                    static_cast<const bf*>(v_cache), static_cast<bf*>(w.o),
                                    w.row_off, B, k_cap, N, c->n_heads, c->n_kv_heads, hd,
-                                   w.status, s, nullptr, nullptr, w.part,
+                                   w.status, s, upd ? upd->m_c : nullptr,
+                                   upd ? upd->l_c : nullptr, w.part,
                                    w.part_bytes) != cudaSuccess) {
       return DLLM_ERR_CUDA;
+    }
+    if (upd) {
+      // DyLLM 2.B: the recomputed rows' query and exact statistics are cached; in a
+      // partial step every other row of a sequence with changed keys takes in only
+      // those keys (old terms out, new terms in) and its context is updated in place
+      const int Hq = c->n_heads;
+      launch_row_words(upd->q_cache, w.q, w.row_pos, w.row_seq, M_dev, M_cap, N, q * 2, true, s);
+      launch_row_words(upd->m_cache, upd->m_c, w.row_pos, w.row_seq, M_dev, M_cap, N, Hq * 4,
+                       true, s);
+      launch_row_words(upd->l_cache, upd->l_c, w.row_pos, w.row_seq, M_dev, M_cap, N, Hq * 4,
+                       true, s);
+      if (upd->partial) {
+        launch_row_words(k_cache, upd->k_new, w.row_pos, w.row_seq, M_dev, M_cap, N, kv * 2,
+                         false, s);
+        launch_row_words(v_cache, upd->v_new, w.row_pos, w.row_seq, M_dev, M_cap, N, kv * 2,
+                         false, s);
+        launch_mark_rows(w.row_pos, w.row_seq, M_dev, M_cap, B, N, upd->skip, s);
+        launch_seq_offsets(B, N, upd->seq_off, s);
+        if (launch_attention_update(static_cast<const bf*>(upd->q_cache), B * N,
+                                    static_cast<bf*>(gate->ctx), upd->m_cache, upd->l_cache,
+                                    upd->seq_off, N, static_cast<const bf*>(upd->k_new),
+                                    static_cast<const bf*>(upd->v_new),
+                                    static_cast<const bf*>(upd->k_old),
+                                    static_cast<const bf*>(upd->v_old), w.row_off, M_cap, B, Hq,
+                                    c->n_kv_heads, hd, w.status, s, upd->skip) != cudaSuccess)
+          return DLLM_ERR_CUDA;
+      }
     }
     GemmSpec go = g;
     go.epi = EPI_RESID;
@@ -837,6 +888,15 @@ struct StepWs {
   int* g_inv;       // [cap]
   int* g_n;         // [1]
   void* g_f;        // [cap, d]
+  // DyLLM approximate attention (policy.attn_update)
+  float* u_m;       // [cap, Hq]
+  float* u_l;
+  void* u_kold;     // [cap, kv] x 4
+  void* u_vold;
+  void* u_knew;
+  void* u_vnew;
+  uint8_t* u_skip;  // [B * N]
+  int* u_off;       // [B + 1]
 };
 
 int k2_cap_of(const dllm_policy* pol, int N) {
@@ -848,7 +908,7 @@ int k2_cap_of(const dllm_policy* pol, int N) {
 int lm_tiles_for(const dllm_model_cfg* c) { return (c->vocab + 127) / 128; }
 
 void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, int k2_cap,
-                 bool gate, StepWs& w) {
+                 bool gate, bool upd, StepWs& w) {
   const size_t es = esize(c->dtype);
   const int cap = B * N;  // covers the dense step
   w.status = bp.take<int>(kHeader / sizeof(int));
@@ -887,6 +947,17 @@ void layout_step(Bump& bp, const dllm_model_cfg* c, int B, int N, int k_cap, int
     w.g_n = bp.take<int>(1);
     w.g_f = bp.take<char>((size_t)cap * c->d * es);
   }
+  if (upd) {
+    const size_t kvb = (size_t)cap * c->n_kv_heads * c->head_dim * es;
+    w.u_m = bp.take<float>((size_t)cap * c->n_heads);
+    w.u_l = bp.take<float>((size_t)cap * c->n_heads);
+    w.u_kold = bp.take<char>(kvb);
+    w.u_vold = bp.take<char>(kvb);
+    w.u_knew = bp.take<char>(kvb);
+    w.u_vnew = bp.take<char>(kvb);
+    w.u_skip = bp.take<uint8_t>((size_t)B * N);
+    w.u_off = bp.take<int>((size_t)B + 1);
+  }
 }
 
 }  // namespace
@@ -897,7 +968,8 @@ extern "C" size_t dllm_step_workspace_size(const dllm_model_cfg* c, int B, int N
   const int k_cap = std::max(1, std::min(pol->k, N));
   Bump bp(nullptr);
   StepWs w{};
-  layout_step(bp, c, B, N, k_cap, k2_cap_of(pol, N), pol->ffn_gate != 0, w);
+  layout_step(bp, c, B, N, k_cap, k2_cap_of(pol, N), pol->ffn_gate != 0, pol->attn_update != 0,
+              w);
   return bp.off;
 }
 
@@ -967,6 +1039,15 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
           !aligned(cache->ffn[l], 16))
         return DLLM_ERR_INVALID_ARG;
   }
+  if (pol->attn_update) {
+    if (!pol->ffn_gate) return DLLM_ERR_INVALID_ARG;
+    if (c->dtype != DLLM_BF16) return DLLM_ERR_UNSUPPORTED_SHAPE;
+    if (!cache->q || !cache->att_m || !cache->att_l) return DLLM_ERR_INVALID_ARG;
+    for (int l = 0; l < c->n_layers; ++l)
+      if (!cache->q[l] || !cache->att_m[l] || !cache->att_l[l] || !aligned(cache->q[l], 16) ||
+          !aligned(cache->att_m[l], 16) || !aligned(cache->att_l[l], 16))
+        return DLLM_ERR_INVALID_ARG;
+  }
   const int l2 = pol->score_layer2;
   if (l2 != 0) {
     if (l2 <= pol->score_layer || l2 >= c->n_layers || pol->k2 < 0) return DLLM_ERR_INVALID_ARG;
@@ -980,7 +1061,7 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
   const int d = c->d;
   Bump bp(ws);
   StepWs w{};
-  layout_step(bp, c, B, N, k_cap, k2_cap, pol->ffn_gate != 0, w);
+  layout_step(bp, c, B, N, k_cap, k2_cap, pol->ffn_gate != 0, pol->attn_update != 0, w);
   LayerWs& L = w.L;
   const bool use_rope = c->rope_theta > 0.f;
   if (use_rope) launch_rope_table(L.rope, N, c->head_dim, c->rope_theta, s);
@@ -1118,8 +1199,15 @@ extern "C" dllm_status dllm_step_ex(const dllm_model_cfg* c, const dllm_model_w*
       }
     }
     LayerGate gt;
+    LayerUpd ut;
+    const LayerUpd* upd = nullptr;
+    if (pol->attn_update) {
+      ut = LayerUpd{cache->q[l], cache->att_m[l], cache->att_l[l], dense == 0, w.u_m, w.u_l,
+                    w.u_kold, w.u_vold, w.u_knew, w.u_vnew, w.u_skip, w.u_off};
+      upd = &ut;
+    }
     st = layer_forward(c, &mw->layers[l], xc, cap_c, M_c, L, B, N, rps, cache->k[l],
-                       cache->v[l], use_rope, s, gate_of(l, dense != 0, gt));
+                       cache->v[l], use_rope, s, gate_of(l, dense != 0, gt), upd);
     if (st != DLLM_OK) return st;
   }
 

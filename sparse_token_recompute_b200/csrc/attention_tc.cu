@@ -80,6 +80,8 @@ struct AttnParams {
   int part_rows;     // row capacity of the partial buffers
   float* part_o;     // [kv_split, part_rows, Hq, HD]
   float* part_ml;    // [kv_split, part_rows, Hq, 2] (m in the exp2 domain, l)
+  // update mode: rows r with skip[r] != 0 (r = row_off[b] + row) keep o, m, l untouched
+  const uint8_t* skip;
 };
 
 // 32 columns without the trailing wait: several loads in flight before one wait
@@ -575,6 +577,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (ok && live && (x == 0 || !split)) {
         const int row = row_x;
+        // update mode: rows the caller recomputes exactly keep their cached values (the
+        // TMEM loads below stay warp-wide; only this lane's stores are skipped)
+        const bool keep = UPD && p.skip && row < cnt && p.skip[off + row] != 0;
         float wa = 1.f, wb = 0.f, m_out = m_ref, w_old = 0.f;
         if (split) {
           const float mb = stat[r], lb = stat[BT + r];
@@ -600,7 +605,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_ld32_nowait(tO(x) + lane_off + c, o);
           if (split) tmem_ld32_nowait(tO(1) + lane_off + c, ob);
           tmem_wait_ld();
-          if (row < cnt && partial) {
+          if (keep) {
+          } else if (row < cnt && partial) {
             float* dst = p.part_o + (((size_t)s_kv * p.part_rows + off + row) * p.Hq + h) * HD + c;
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -625,7 +631,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
         }
-        if (row < cnt && partial) {
+        if (keep) {
+        } else if (row < cnt && partial) {
           float* ml = p.part_ml + (((size_t)s_kv * p.part_rows + off + row) * p.Hq + h) * 2;
           ml[0] = m_out;
           ml[1] = lsum;
@@ -754,7 +761,7 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
   float* part_ml = S > 1 ? part + (size_t)S * M_cap * Hq * hd : nullptr;
   AttnParams p{row_off, o,      Nseq, Hq,      Hkv,    Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
                status,  st_m,   st_l, nullptr, 1,      S,       M_cap,
-               part_o,  part_ml};
+               part_o,  part_ml, nullptr};
   dim3 grid(((k_cap + NTILE * BT - 1) / (NTILE * BT)) * S, Hq, B);
   ProfScope prof("attention", s);
   cudaError_t e = hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
@@ -775,7 +782,7 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
                                     const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                                     const __nv_bfloat16* k_old, const __nv_bfloat16* v_old,
                                     const int* a_off, int A_cap, int B, int Hq, int Hkv, int hd,
-                                    int* status, cudaStream_t s) {
+                                    int* status, cudaStream_t s, const uint8_t* skip) {
   if (B <= 0 || r_cap <= 0 || R_cap <= 0 || A_cap <= 0) return cudaSuccess;
   if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
   CUtensorMap tq, tk, tv, tk2, tv2;
@@ -793,7 +800,7 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
   const int ppc = std::max(1, (pairs + min_x - 1) / min_x);
   AttnParams p{r_off, o,    0,    Hq,   Hkv,   Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
                status, st_m, st_l, a_off, ppc,   1,       0,
-               nullptr, nullptr};
+               nullptr, nullptr, skip};
   dim3 grid((pairs + ppc - 1) / ppc, Hq, B);
   ProfScope prof("attention_update", s);
   return hd == 128 ? launch_hd<128, true>(tq, tk, tv, tk2, tv2, p, grid, s)

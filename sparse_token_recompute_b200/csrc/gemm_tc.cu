@@ -36,6 +36,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;
+
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_THREADS = 128;
 
@@ -70,6 +71,7 @@ struct Params {
   int prefetch_b;  // issue the first unit's weight tiles before waiting on the previous kernel
   int raster_g;    // CTA-pair kernel: row-tile pairs per raster group
   int stall_test;  // CTA-pair kernel, tests only: CTA 1 withholds its first stage
+  int krot;        // walk each tile's k-blocks from a tile-dependent start (weight streaming)
   int* status;
 };
 
@@ -86,6 +88,18 @@ __device__ __forceinline__ void decode_unit(int u, int m_tiles, int tiles_n, int
   const int r = t - g * per_group;
   m = first_m + r % gsz;
   n = r / gsz;
+}
+
+// The i-th k-block of a unit whose K range is [kb0, kb0 + nkb), for output tile n.
+// With krot the walk starts at a tile-dependent block and wraps around, so that
+// CTAs streaming different weight tiles at the same time read different column
+// ranges of their rows (the same accumulation, in another order); measured ~3%
+// faster on weight-streaming GEMMs and slower on tensor-bound ones.
+__device__ __forceinline__ int kb_at(int i, int kb0, int nkb, int n, int krot) {
+  if (!krot) return kb0 + i;
+  int j = i + (n * 5) % nkb;
+  if (j >= nkb) j -= nkb;
+  return kb0 + j;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -348,15 +362,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Weights never depend on earlier kernels: with a single row tile by
   // capacity, the producer starts streaming this CTA's first weight tiles
   // before it waits for the kernel that writes A (and the row count).
-  int npre = 0, pre_n = 0, pre_kb0 = 0;
+  int npre = 0, pre_n = 0, pre_kb0 = 0, pre_nkb = 1;
   if (p.prefetch_b && warp == 0 && lane == 0 && (int)blockIdx.x < p.tiles_n * p.splits) {
     int m, s;
     decode_unit(blockIdx.x, 1, p.tiles_n, p.splits, m, pre_n, s);
     pre_kb0 = s * p.kb_per_split;
+    pre_nkb = max(1, min(pre_kb0 + p.kb_per_split, p.kb_total) - pre_kb0);
     npre = max(0, min(STAGES, min(pre_kb0 + p.kb_per_split, p.kb_total) - pre_kb0));
     for (int i = 0; i < npre; ++i) {  // fresh stages: no empty wait
       mbar_arrive_expect_tx(full_bar(i), (uint32_t)p.a_tx + B_BYTES);
-      load_b(smem_u32(sB + i * B_BYTES), full_bar(i), pre_kb0 + i, pre_n);
+      load_b(smem_u32(sB + i * B_BYTES), full_bar(i), kb_at(i, pre_kb0, pre_nkb, pre_n, p.krot), pre_n);
     }
   }
   griddep_wait();
@@ -383,7 +398,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // the A halves of the pre-issued stages (row tile 0); when this CTA has no
       // unit after all (no rows), they only complete the stages before exit
       for (int i = 0; i < npre; ++i) {
-        tma_load_2d(smem_u32(sA + i * A_BYTES), &tmA, full_bar(i), (pre_kb0 + i) * BK, 0);
+        tma_load_2d(smem_u32(sA + i * A_BYTES), &tmA, full_bar(i),
+                    kb_at(i, pre_kb0, pre_nkb, pre_n, p.krot) * BK, 0);
         issued |= 1u << i;
       }
       if (npre > 0 && (int)blockIdx.x >= n_units) {
@@ -393,9 +409,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int m, n, s;
         decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
-        const int kb0 = s * p.kb_per_split + (u == (int)blockIdx.x ? npre : 0);
-        const int kb1 = min(s * p.kb_per_split + p.kb_per_split, p.kb_total);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        const int kb0 = s * p.kb_per_split;
+        const int nkb = min(kb0 + p.kb_per_split, p.kb_total) - kb0;
+        for (int i = (u == (int)blockIdx.x ? npre : 0); i < nkb; ++i) {
+          const int kb = kb_at(i, kb0, nkb, n, p.krot);
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
@@ -437,7 +454,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {  // stages arrive in the producer's k order
           if (!mbar_wait(full_bar(stage), phase, abort_flag, p.status)) {
             ok = false;
             break;
@@ -753,7 +770,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int u = pair_id; u < n_units && ok; u += n_pairs) {
         int mp, n, s;
         decode_unit(u, m_pairs, p.tiles_n, 1, mp, n, s, p.raster_g);
-        for (int kb = 0; kb < p.kb_total; ++kb) {
+        for (int i = 0; i < p.kb_total; ++i) {
+          const int kb = kb_at(i, 0, p.kb_total, n, p.krot);
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) {
             ok = false;
             break;
@@ -1126,6 +1144,8 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   p.status = g.status;
   p.stall_test = g.stall_test;
   if (g.stall_test && !pl.pair) return cudaErrorInvalidValue;
+  // weight-streaming shapes (fewer than 256 rows): rotated k walks
+  p.krot = g.M_cap < 256 ? 1 : 0;
 
   CUtensorMap ta, tb0, tb1, tb2;
   // with fewer than 128 rows the A box covers only them (rounded to 16): the MMA still

@@ -168,7 +168,7 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
                                     const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                                     const __nv_bfloat16* k_old, const __nv_bfloat16* v_old,
                                     const int* a_off, int A_cap, int B, int Hq, int Hkv, int hd,
-                                    int* status, cudaStream_t s);
+                                    int* status, cudaStream_t s, const uint8_t* skip = nullptr);
 
 // ----- score / select / unmask -----
 template <typename T>
@@ -218,6 +218,16 @@ template <typename T>
 void launch_ffn_combine(T* x, const T* f_new, T* f_cache, const int* inv, const int* row_pos,
                         const int* row_seq, const int* M_dev, int M_cap, int N, int d,
                         cudaStream_t s);
+// DyLLM approximate attention bookkeeping.  Compact rows r < M (row_bytes per row, a
+// multiple of 4) to / from a per-row cache [B, N, row_bytes]:
+void launch_row_words(void* cache, void* compact, const int* row_pos, const int* row_seq,
+                      const int* M_dev, int M_cap, int N, int row_bytes, bool to_cache,
+                      cudaStream_t s);
+// flags [B, N] uint8: 1 at the compact rows' positions, 0 elsewhere
+void launch_mark_rows(const int* row_pos, const int* row_seq, const int* M_dev, int M_cap, int B,
+                      int N, uint8_t* flags, cudaStream_t s);
+// off[b] = b * N, b = 0..B (every row of every sequence in cache order)
+void launch_seq_offsets(int B, int N, int* off, cudaStream_t s);
 void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
                      int32_t* dst_count, int B, int k_cap, cudaStream_t s);
 

@@ -1021,6 +1021,51 @@ __global__ void __launch_bounds__(128) ffn_combine_kernel(T* __restrict__ x,
   }
 }
 
+// ---------------------------------------------------------------- DyLLM approximate attention
+
+// Rows r < M of a per-row cache [B, N, words] (32-bit words) <-> compact rows
+// [cap, words]: to_cache = 1 scatters compact -> cache, 0 gathers cache -> compact.
+// One block per compact row.
+__global__ void __launch_bounds__(128) row_words_kernel(uint32_t* __restrict__ cache,
+                                                        uint32_t* __restrict__ compact,
+                                                        const int* __restrict__ row_pos,
+                                                        const int* __restrict__ row_seq,
+                                                        const int* __restrict__ M_dev, int M_cap,
+                                                        int N, int words, int to_cache) {
+  const int r = blockIdx.x;
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  if (r >= M) return;
+  uint32_t* c = cache + ((size_t)row_seq[r] * N + row_pos[r]) * words;
+  uint32_t* x = compact + (size_t)r * words;
+  if ((words & 3) == 0) {
+    uint4* c4 = reinterpret_cast<uint4*>(c);
+    uint4* x4 = reinterpret_cast<uint4*>(x);
+    for (int i = threadIdx.x; i < (words >> 2); i += blockDim.x) {
+      if (to_cache) c4[i] = x4[i]; else x4[i] = c4[i];
+    }
+  } else {
+    for (int i = threadIdx.x; i < words; i += blockDim.x) {
+      if (to_cache) c[i] = x[i]; else x[i] = c[i];
+    }
+  }
+}
+
+// flags[seq * N + pos] = 1 for the compact rows r < M (the buffer is cleared first)
+__global__ void __launch_bounds__(256) mark_rows_kernel(const int* __restrict__ row_pos,
+                                                        const int* __restrict__ row_seq,
+                                                        const int* __restrict__ M_dev, int M_cap,
+                                                        int N, uint8_t* __restrict__ flags) {
+  const int M = M_dev ? min(*M_dev, M_cap) : M_cap;
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < M; r += gridDim.x * blockDim.x)
+    flags[(size_t)row_seq[r] * N + row_pos[r]] = 1;
+}
+
+// off[b] = b * N for b <= B: every row of every sequence, in cache order
+__global__ void seq_offsets_kernel(int B, int N, int* off) {
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b <= B; b += gridDim.x * blockDim.x)
+    off[b] = b * N;
+}
+
 __global__ void copy_idx_kernel(const int32_t* src_idx, const int32_t* src_count,
                                 int32_t* dst_idx, int32_t* dst_count, int B, int k_cap) {
   const size_t total = (size_t)B * k_cap;
@@ -1352,6 +1397,29 @@ template void launch_ffn_combine<__nv_bfloat16>(__nv_bfloat16*, const __nv_bfloa
                                                 __nv_bfloat16*, const int*, const int*,
                                                 const int*, const int*, int, int, int,
                                                 cudaStream_t);
+
+void launch_row_words(void* cache, void* compact, const int* row_pos, const int* row_seq,
+                      const int* M_dev, int M_cap, int N, int row_bytes, bool to_cache,
+                      cudaStream_t s) {
+  if (M_cap <= 0 || row_bytes <= 0) return;
+  ProfScope prof(to_cache ? "scatter_rows" : "gather_rows_cache", s);
+  row_words_kernel<<<M_cap, 128, 0, s>>>(static_cast<uint32_t*>(cache),
+                                         static_cast<uint32_t*>(compact), row_pos, row_seq,
+                                         M_dev, M_cap, N, row_bytes / 4, to_cache ? 1 : 0);
+}
+
+void launch_mark_rows(const int* row_pos, const int* row_seq, const int* M_dev, int M_cap, int B,
+                      int N, uint8_t* flags, cudaStream_t s) {
+  ProfScope prof("mark_rows", s);
+  cudaMemsetAsync(flags, 0, (size_t)B * N, s);
+  if (M_cap > 0)
+    mark_rows_kernel<<<grid_for((size_t)M_cap, 256), 256, 0, s>>>(row_pos, row_seq, M_dev, M_cap,
+                                                                  N, flags);
+}
+
+void launch_seq_offsets(int B, int N, int* off, cudaStream_t s) {
+  seq_offsets_kernel<<<grid_for((size_t)B + 1, 256), 256, 0, s>>>(B, N, off);
+}
 
 void launch_copy_idx(const int32_t* src_idx, const int32_t* src_count, int32_t* dst_idx,
                      int32_t* dst_count, int B, int k_cap, cudaStream_t s) {

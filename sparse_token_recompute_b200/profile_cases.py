@@ -9,6 +9,7 @@ but a few GB at most, runs the kernel `--warmup` times untimed and then
   python -m sparse_token_recompute_b200.profile_cases layer --B 32 --N 1536 --k 308
   python -m sparse_token_recompute_b200.profile_cases attention --B 32 --N 1536 --k 308
   python -m sparse_token_recompute_b200.profile_cases step --B 1 --ratio 0.10
+  python -m sparse_token_recompute_b200.profile_cases step_graph --B 1 --ratio 0.10
 """
 from __future__ import annotations
 
@@ -126,6 +127,25 @@ def case_step(a):
     return {"case": "step", "B": shape.batch, "N": shape.seq_len, "k": shape.k, "ms": ms}
 
 
+def case_step_graph(a):
+    """case_step, with the timed partial steps replayed from a CUDA graph (no
+    per-launch host cost), as the benchmark's batch-1 figures are."""
+    base = SY.DENSE8B_B1_N768 if a.B == 1 else SY.DENSE8B_B32_N1536
+    shape = SY.with_(base, ratio=a.ratio)
+    W = SY.model_weights(shape, seed=0, device="cuda")
+    model = S.Model(S.cfg_from_shape(shape), W)
+    tokens = SY.prompt_tokens(shape, seed=1, device="cuda")
+    cache = S.Cache(model.cfg, shape.batch, shape.seq_len)
+    pol = S.make_policy(0, shape.alpha, 0, 0, shape.k, 0.0, shape.n_unmask, shape.prompt_len,
+                        shape.block_len)
+    ws = S.Workspace(S.dllm_step_workspace_size(model.cfg, shape.batch, shape.seq_len, pol))
+    S.dllm_step(model, cache, tokens, pol, True, ws)
+    S.dllm_step(model, cache, tokens, pol, False, ws)
+    graph = S.StepGraph(model, cache, tokens, pol, ws)
+    ms = _time(graph.replay, a.warmup, a.iters)
+    return {"case": "step_graph", "B": shape.batch, "N": shape.seq_len, "k": shape.k, "ms": ms}
+
+
 def case_layer(a):
     shape = SY.with_(SY.DENSE8B_B32_N1536, n_layers=1)
     W = SY.model_weights(shape, seed=0, device="cuda")
@@ -150,7 +170,7 @@ def case_layer(a):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["gemm", "score", "layer", "attention", "attention_update",
-                                     "step"])
+                                     "step", "step_graph"])
     ap.add_argument("--ratio", type=float, default=0.10)
     ap.add_argument("--heads", type=int, default=32)
     ap.add_argument("--kv-heads", dest="kv_heads", type=int, default=32)
@@ -174,7 +194,7 @@ def main():
         a.N = 1536 if a.N == 12288 else a.N
     out = {"gemm": case_gemm, "score": case_score, "layer": case_layer,
            "attention": case_attention, "attention_update": case_attention_update,
-           "step": case_step}[a.case](a)
+           "step": case_step, "step_graph": case_step_graph}[a.case](a)
     print(json.dumps(out))
 
 

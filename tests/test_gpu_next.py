@@ -450,3 +450,87 @@ def test_step_host_equals_device_step(lib):
     for a, b in zip(r1.cache.k + r1.cache.v + [r1.cache.h_ref, r1.cache.conf, r1.cache.pred],
                     r2.cache.k + r2.cache.v + [r2.cache.h_ref, r2.cache.conf, r2.cache.pred]):
         assert torch.equal(a, b)
+
+
+# ----------------------------------------------------------------- approximate attention step
+
+
+def _upd_run(lib, shape, tau, prebuilt=None):
+    r = Run(lib, shape, prebuilt=prebuilt, ffn_gate=True, ffn_tau=tau, attn_update=True)
+    r.pol.ffn_gate, r.pol.ffn_tau, r.pol.attn_update = 1, tau, 1
+    r.cache = lib.Cache(r.model.cfg, r.B, r.N, ffn_gate=True, attn_update=True)
+    r.ws = lib.Workspace(lib.dllm_step_workspace_size(r.model.cfg, r.B, r.N, r.pol))
+    return r
+
+
+def _lse(m, l):
+    return np.asarray(m, dtype=np.float64) + np.log(np.asarray(l, dtype=np.float64))
+
+
+def _compare_upd_caches(r, tol):
+    Hq = r.ocfg.n_heads
+    for l in range(r.ocfg.n_layers):
+        assert max_abs_rel(f64(r.cache.ctx[l]), r.st.ctx[l]) < tol, ("ctx", l)
+        assert max_abs_rel(f64(r.cache.ffn[l]), r.st.ffn[l]) < tol, ("ffn", l)
+        assert max_abs_rel(f64(r.cache.q[l]), r.st.q[l]) < tol, ("q", l)
+        lse_g = _lse(f64(r.cache.att_m[l]), f64(r.cache.att_l[l]))
+        lse_o = _lse(r.st.att_m[l], r.st.att_l[l])
+        assert np.max(np.abs(lse_g - lse_o)) < tol * max(np.abs(lse_o).max(), 1.0), ("lse", l)
+
+
+def _upd_forced(lib, shape, tau, tol, steps, prebuilt=None):
+    """DyLLM's approximate attention inside partial steps (French summary §2.B):
+    the GPU follows the oracle's selections, reveals and FFN-gate decisions; every
+    cache -- K/V, contexts (the stable rows' ones updated incrementally), FFN
+    outputs, queries and softmax statistics -- is compared after each step."""
+    r = _upd_run(lib, shape, tau, prebuilt)
+    L = r.ocfg.n_layers
+    for t in range(steps):
+        out = O.step(r.ocfg, r.ow, r.st, r.opol, dense=(t == 0))
+        io = {"forced_unmask_pos": _pad(out.unmasked, out.unmasked.shape[1])}
+        if t > 0:
+            io.update(forced_idx=_pad(out.idx, r.k_cap),
+                      forced_count=torch.tensor([len(a) for a in out.idx], dtype=torch.int32,
+                                                device="cuda"))
+            fz = np.zeros((L, r.B * r.k_cap), dtype=np.uint8)
+            first = L - len(out.ffn_salient)
+            for j, sal in enumerate(out.ffn_salient):
+                fz[first + j, :len(sal)] = sal
+            io["forced_ffn"] = torch.from_numpy(fz).cuda()
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, t == 0, r.ws, **io)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        r.compare_tokens(r.compare_state(tol, out.final_rows, out.idx))
+        _compare_upd_caches(r, tol)
+    return r
+
+
+def test_approximate_attention_step_bf16_forced(lib):
+    _upd_forced(lib, _small_bf16(), 1e-3, TOL["bf16"], 4)
+
+
+def test_approximate_attention_step_gqa_forced(lib):
+    _upd_forced(lib, _small_bf16(n_heads=4, n_kv_heads=2, head_dim=64, batch=3), 1e-3,
+                TOL["bf16"], 4)
+
+
+def test_approximate_attention_step_own_run_tracks_its_caches(lib):
+    """On its own decisions, after every step each row's cached context on the GPU
+    equals the attention of its cached query over the GPU's current K/V caches
+    (oracle attention in float64 on the GPU's caches; the invariant the oracle's
+    step mode is pinned by), and its (m, l) give that attention's log-sum-exp."""
+    shape = _small_bf16()
+    r = _upd_run(lib, shape, 1e-3)
+    Hq, hd = r.ocfg.n_heads, r.ocfg.head_dim
+    for t in range(4):
+        lib.dllm_step_ex(r.model, r.cache, r.tokens, r.pol, t == 0, r.ws)
+        torch.cuda.synchronize()
+        assert r.ws.device_status() == 0
+        for l in range(r.ocfg.n_layers):
+            for b in range(r.B):
+                q = f64(r.cache.q[l][b]).reshape(r.N, Hq, hd)
+                m, lsum, o = O.attention_stats(q, f64(r.cache.k[l][b]), f64(r.cache.v[l][b]))
+                got = f64(r.cache.ctx[l][b])
+                assert max_abs_rel(got, o.reshape(r.N, -1)) < TOL["bf16"], (t, l, b)
+                lse = _lse(f64(r.cache.att_m[l][b]), f64(r.cache.att_l[l][b]))
+                assert np.max(np.abs(lse - (m + np.log(lsum)))) < 2e-2 * max(np.abs(m).max(), 1), (t, l, b)
