@@ -37,6 +37,7 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 
+
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_THREADS = 128;
 
@@ -69,13 +70,13 @@ struct Params {
   int V;
   int a_tx;  // bytes one A box delivers (fewer than a full 128-row tile when M_cap < 128)
   int prefetch_b;  // issue the first unit's weight tiles before waiting on the previous kernel
-  int raster_g;    // CTA-pair kernel: row-tile pairs per raster group
+  int raster_g;    // row tiles (pairs, in the CTA-pair kernel) per raster group
   int stall_test;  // CTA-pair kernel, tests only: CTA 1 withholds its first stage
   int krot;        // walk each tile's k-blocks from a tile-dependent start (weight streaming)
   int* status;
 };
 
-// G: m-tiles per raster group (the group's A rows stay in L2 while its CTAs sweep
+// G: row tiles per raster group (the group's A rows stay in L2 while its CTAs sweep
 // every column tile)
 __device__ __forceinline__ void decode_unit(int u, int m_tiles, int tiles_n, int splits, int& m,
                                             int& n, int& s, int G = 32) {
@@ -365,7 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   int npre = 0, pre_n = 0, pre_kb0 = 0, pre_nkb = 1;
   if (p.prefetch_b && warp == 0 && lane == 0 && (int)blockIdx.x < p.tiles_n * p.splits) {
     int m, s;
-    decode_unit(blockIdx.x, 1, p.tiles_n, p.splits, m, pre_n, s);
+    decode_unit(blockIdx.x, 1, p.tiles_n, p.splits, m, pre_n, s, p.raster_g);
     pre_kb0 = s * p.kb_per_split;
     pre_nkb = max(1, min(pre_kb0 + p.kb_per_split, p.kb_total) - pre_kb0);
     npre = max(0, min(STAGES, min(pre_kb0 + p.kb_per_split, p.kb_total) - pre_kb0));
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int m, n, s;
-        decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
+        decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s, p.raster_g);
         const int kb0 = s * p.kb_per_split;
         const int nkb = min(kb0 + p.kb_per_split, p.kb_total) - kb0;
         for (int i = (u == (int)blockIdx.x ? npre : 0); i < nkb; ++i) {
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool issued_any = false;
       for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
         int m, n, s;
-        decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
+        decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s, p.raster_g);
         const int kb0 = s * p.kb_per_split;
         const int kb1 = min(kb0 + p.kb_per_split, p.kb_total);
         if (!mbar_wait(tempty_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
@@ -495,7 +496,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
       int m, n, s;
-      decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s);
+      decode_unit(u, m_tiles, p.tiles_n, p.splits, m, n, s, p.raster_g);
       // warp-uniform outcome: TMEM loads below are warp-collective
       const bool ok = __all_sync(0xffffffffu,
                                  mbar_wait(tfull_bar(acc), acc_phase, abort_flag, p.status));
@@ -542,7 +543,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     cluster_sync_all();
     if (warp >= 2 && (int)blockIdx.x < n_units) {
       int m, n, s;
-      decode_unit(blockIdx.x, m_tiles, p.tiles_n, p.splits, m, n, s);
+      decode_unit(blockIdx.x, m_tiles, p.tiles_n, p.splits, m, n, s, p.raster_g);
       const int S = p.splits;
       const int rank = (int)cluster_ctarank();
       const int SR = (BM + S - 1) / S;
@@ -1153,8 +1154,11 @@ cudaError_t gemm_launch(GemmSpec g, cudaStream_t s) {
   const int a_rows = g.M_cap < BM ? ((g.M_cap + 15) / 16) * 16 : BM;
   p.a_tx = a_rows * BK * 2;
   p.prefetch_b = (g.M_cap <= BM && pdl_enabled()) ? 1 : 0;
-  // the A rows of a raster group (256 per pair) stay within ~32 MB of L2
-  p.raster_g = std::max(2, std::min(16, (int)((32u << 20) / ((size_t)2 * BM * g.K * 2))));
+  // m-major raster groups; the A rows of a group (256 per pair) stay within ~32 MB of
+  // L2 (groups of 48, 64 and 96 MB, and column-tile groups chosen by a traffic model,
+  // were measured: no faster, and the larger ones read far more DRAM)
+  p.raster_g = pl.pair ? std::max(2, std::min(16, (int)((32u << 20) / ((size_t)2 * BM * g.K * 2))))
+                       : 32;
   if (!make_map(&ta, g.A, g.M_cap, g.K, a_rows)) return cudaErrorInvalidValue;
   // a CTA pair stages half of each 256-wide B tile per CTA
   const int bbox = (g.epi == EPI_SWIGLU || pl.pair) ? pl.bn / 2 : pl.bn;

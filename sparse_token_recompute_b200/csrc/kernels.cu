@@ -319,6 +319,121 @@ __device__ SoftStat row_softstat(const T* z, int V, SoftStat* red) {
   return r;
 }
 
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Statistics of one logits row, block-wide, in few instructions per logit: each
+// thread keeps a running (max, sum) over chunks of 4 vectors of 8 (three-input
+// maxima; the exponent argument and the sum two lanes per instruction); the first
+// index of the maximum is not tracked in the loop: once the block knows the row's
+// maximum, the threads whose own maximum equals it read the chunk where they first
+// met it again (from cache) and report its first position.  Measured against a
+// variant that tracked the argmax per chunk: 139 -> 129 us for 8192 rows of 32768
+// bf16 logits; staging rows through shared memory with bulk copies (164 us) and
+// computing half the exponentials with a polynomial on the FMA pipe (184 us) were
+// slower: the kernel is bound by instruction issue and the special-function unit.
+template <typename T>
+__device__ SoftStat row_softstat_lean(const T* z, int V, SoftStat* red) {
+  constexpr int U = 4;
+  constexpr float LOG2E = 1.4426950408889634f;
+  float m = -INFINITY;
+  int m_base = 0;  // first element of the chunk that last raised m
+  float2 s2 = make_float2(0.f, 0.f);
+  const int stride = blockDim.x * 8;
+  for (int base = threadIdx.x * 8; base < V; base += stride * U) {
+    float f[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = base + u * stride;
+      if (i < V) {
+        load_vec8<T>(z + i, f[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[u][j] = -INFINITY;
+      }
+    }
+    float cm = m;
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) cm = fmax3f(cm, f[u][j], f[u][j + 1]);
+    if (cm == -INFINITY) continue;
+    if (cm > m) {  // rescale the running sum to the new maximum
+      const float sc = m == -INFINITY ? 0.f : ex2_approx((m - cm) * LOG2E);
+      s2.x *= sc;
+      s2.y *= sc;
+      m = cm;
+      m_base = base;
+    }
+    const float2 l2 = make_float2(LOG2E, LOG2E);
+    const float2 nm = make_float2(-m * LOG2E, -m * LOG2E);
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        const float2 x = fma_f32x2(make_float2(f[u][j], f[u][j + 1]), l2, nm);
+        s2 = add_f32x2(s2, make_float2(ex2_approx(x.x), ex2_approx(x.y)));
+      }
+  }
+  SoftStat st{m, s2.x + s2.y, 0x7fffffff};
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    SoftStat y;
+    y.m = __shfl_xor_sync(0xffffffffu, st.m, o);
+    y.s = __shfl_xor_sync(0xffffffffu, st.s, o);
+    y.a = 0x7fffffff;
+    st = soft_merge(st, y);
+  }
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = st;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    SoftStat t = red[0];
+    for (int i = 1; i < nw; ++i) t = soft_merge(t, red[i]);
+    red[32] = t;
+  }
+  __syncthreads();
+  SoftStat r = red[32];
+  // first position of the maximum: threads whose own maximum is the row's scan the
+  // chunk where they first met it (earlier chunks held only smaller values)
+  int a = 0x7fffffff;
+  if (m == r.m && m != -INFINITY) {
+    float f[U][8];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = m_base + u * stride;
+      if (i < V) {
+        load_vec8<T>(z + i, f[u]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[u][j] = -INFINITY;
+      }
+    }
+#pragma unroll
+    for (int u = U - 1; u >= 0; --u)
+#pragma unroll
+      for (int j = 7; j >= 0; --j)
+        if (f[u][j] == m) a = m_base + u * stride + j;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = min(a, __shfl_xor_sync(0xffffffffu, a, o));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w].a = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = red[0].a;
+    for (int i = 1; i < nw; ++i) t = min(t, red[i].a);
+    red[32].a = t;
+  }
+  __syncthreads();
+  r.a = red[32].a;
+  __syncthreads();
+  return r;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) confidence_kernel(const T* __restrict__ logits,
                                                          const int32_t* __restrict__ logit_pos,
@@ -328,7 +443,7 @@ __global__ void __launch_bounds__(256) confidence_kernel(const T* __restrict__ l
   __shared__ SoftStat red[33];
   const int r = blockIdx.x;  // b * Mm + j
   const int b = r / Mm;
-  const SoftStat st = row_softstat<T>(logits + (size_t)r * V, V, red);
+  const SoftStat st = row_softstat_lean<T>(logits + (size_t)r * V, V, red);
   if (threadIdx.x == 0) {
     const int p = logit_pos[r];
     if (p >= 0 && p < N) {
