@@ -42,7 +42,7 @@ GQA = SY.GQA7B_B8_N2048
 # its four launches per layer (QKV, O, gate/up, down) at 32 x 308 rows of the 8B
 # layer, from the ncu capture summarised in
 # profiles/gemm_projections_8b_layer_b32_n1536_k308_dram.md; re-take it when either GEMM kernel changes.
-GEMM_TRAFFIC_PER_LAUNCH = 889.7e6
+GEMM_TRAFFIC_PER_LAUNCH = 851.4e6
 
 
 def parse():
