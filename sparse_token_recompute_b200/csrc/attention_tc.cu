@@ -326,7 +326,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int q_issued = 0;  // pairs whose Q tiles were requested
       if (!split) {
         for (int i = 0; i < npairs && ok; ++i) {
-          // the previous pair's Q tiles stay until its last Q.K^T has run
+          // a later pair's first K tile enters the ring before its Q tiles wait for the
+          // previous pair's last Q.K^T to run
+          if (i > 0 && !(ok = load(false, 0))) break;
           if (i > 0 && !(ok = mbar_wait(q_empty, (i - 1) & 1, abort_flag, p.status))) break;
           const int nqi = pair_nq(i);
           mbar_arrive_expect_tx(q_full, nqi * L::Q_TILE);
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               tma_load_2d(sQ + x * L::Q_TILE + c * BT * 128, &tmQ, q_full, h * HD + c * 64,
                           off + pair_q0(i) + x * BT);
           ++q_issued;
-          ok = load(false, 0);
+          if (i == 0) ok = load(false, 0);
           for (int j = 0; j < T && ok; ++j) {
             ok = load(true, j);
             if (ok && j + 1 < T) ok = load(false, j + 1);
@@ -418,6 +420,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!(ok = sk >= 0)) break;
           for (int x = 0; x < nqi; ++x) qk(x, sk);
           give(sk);
+          // once the pair's last Q.K^T has run, the next pair's Q tiles may load
+          if (T == 1) tc_commit(q_empty);
           for (int j = 0; j < T && ok; ++j) {
             const int sv = take();
             if (!(ok = sv >= 0 && pv(0, j, sv))) break;
@@ -430,10 +434,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               if (!(ok = pv(1, j, sv))) break;
               if (sk1 >= 0) qk(1, sk1);
             }
+            if (j + 2 == T) tc_commit(q_empty);
             give(sv);
             if (sk1 >= 0) give(sk1);
           }
-          if (ok) tc_commit(q_empty);  // every Q.K^T of the pair is issued
         }
       } else if ((ok = mbar_wait(q_full, 0, abort_flag, p.status))) {
         for (int x = 0; x < 2 && ok; ++x) {
@@ -524,19 +528,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           m_ref = mx;
         }
         lsum *= first ? 0.f : alpha;
-        if (rescale_o) {
-          // S_X(j) complete implies PV_X(j-1) complete: O_X is stable until P_X(j) is ready
-#pragma unroll 1
-          for (int c = 0; c < HD; c += 32) {
-            float o[32];
-            tmem_ld32_nowait(tO(x) + lane_off + c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(tO(x) + lane_off + c, reinterpret_cast<const uint32_t*>(o));
-          }
-          tmem_wait_st();
-        }
         const float neg_m = -m_ref;
         float rsv[8];
 #pragma unroll
@@ -558,6 +549,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // P_X over the first 64 columns of S_X (S_X has been read into registers)
         tmem_st32(tS(x) + lane_off, pk);
         tmem_st32(tS(x) + lane_off + 32, pk + 32);
+        if (rescale_o) {
+          // S_X(j) complete implies PV_X(j-1) complete: O_X is stable until P_X(j) is
+          // ready (rescaled once the scores are out of the registers)
+#pragma unroll 1
+          for (int c = 0; c < HD; c += 32) {
+            float o[32];
+            tmem_ld32_nowait(tO(x) + lane_off + c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(tO(x) + lane_off + c, reinterpret_cast<const uint32_t*>(o));
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full(x));
