@@ -516,9 +516,10 @@ def generation_from_sample(shape, t_pl, t_plm, t_dl, t_dlm):
 def oracle_direct(reps_big=1):
     """The oracle timed end to end, without extrapolation, on the workloads it
     finishes in seconds: the tiny model's whole 8-step generation (dense step 0,
-    then 25 % partial steps), and one dense plus one 10 % partial step of the 8B
+    then 25 % partial steps), one dense plus one 10 % partial step of the 8B
     shape reduced to 2 of its 32 layers (full width, full vocabulary, one
-    sequence of 768 tokens)."""
+    sequence of 768 tokens), and the full standalone score + select workload
+    (32 x 1024 rows of d 4096, 256 x 32768 logits per sequence, top 256)."""
     import numpy as np
     import torch
     import oracle as O
@@ -562,6 +563,20 @@ def oracle_direct(reps_big=1):
         "dense_step_s": round(t1 - t0, 3), "partial_step_10pct_s": round(t2 - t1, 3),
         "workload": "8B shape with 2 of 32 layers (d 4096, FFN 12288, vocab 126464), one "
                     "sequence of 512 prompt + 256 generated tokens; partial step: 77 rows"}
+    si = SY.score_inputs(device="cpu")
+    args = [f64(t) for t in (si.h_cur, si.h_ref, si.conf)] + [
+        si.pred.numpy().astype(np.int64), si.masked.numpy()]
+    lg, lp = f64(si.logits), si.logit_pos.numpy().astype(np.int64)
+    del si
+    t0 = time.perf_counter()
+    scores, _, _ = O.score_call(*args, 0.5, O.SCORE_COS, logits=lg, logit_pos=lp)
+    O.select(scores, O.SELECT_TOPK, 256, 0.0, 256)
+    t = time.perf_counter() - t0
+    out["score_select_32x1024"] = {
+        "s": round(t, 3), "GB_per_s": round(1.073741824 / t, 3),
+        "workload": "dllm_score + dllm_select inputs at full size: h_cur, h_ref bf16 "
+                    "[32, 1024, 4096], logits bf16 [32, 256, 32768], top 256 of 1024 per "
+                    "sequence (1.074 GB of algorithmic input)"}
     return out
 
 
