@@ -31,6 +31,13 @@ pytestmark = pytest.mark.gpu
     (257, 8192, 1024, 0, False),     # three row tiles, the last one holding one row
     (600, 1000, 512, 0, False),      # ragged last column tile
     (384, 640, 200, 0, True),        # ragged K (a partial last k-block), 1.5 row-tile pairs
+    # one row tile, weight streaming (the planner's split-K clusters or wide tiles)
+    (77, 4096, 4096, 0, True),       # O-shaped, residual accumulate
+    (77, 12288, 4096, 0, False),     # QKV-shaped
+    (1, 4096, 12288, 0, True),       # one row, down-shaped K
+    (128, 2048, 4096, 0, False),     # a full row tile
+    (100, 3000, 4096, 0, False),     # ragged last column tile
+    (60, 2048, 4040, 0, True),       # ragged K (a partial last k-block)
 ])
 def test_gemm_bf16(lib, M, N, K, splits, acc):
     A = SY.normal((M, K), 1.0, 11 + M, "cuda", "bf16")
