@@ -486,8 +486,8 @@ dllm_status dllm_attention_update_bf16(const void* q, void* o, float* m, float* 
  * (larger B returns DLLM_ERR_CAPACITY before anything is launched); every GPU
  * that loads the library holds it until the process exits.  The first call in
  * each device context (per device, and again after the context changes, e.g.
- * after cudaDeviceReset) looks up the array's device address: make it before
- * any stream capture.  All calls share the array: calls that may overlap on
+ * after cudaDeviceReset) looks up the array's device address with a runtime
+ * call on the host (cudaGetSymbolAddress).  All calls share the array: calls that may overlap on
  * the GPU (other streams, other host threads on the same device) race and
  * must be ordered by the caller.  Device-side faults are recorded in the
  * shared status word, which this entry point clears at the start of each call

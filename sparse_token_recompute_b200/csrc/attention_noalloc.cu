@@ -16,7 +16,7 @@
 // names a host-side stand-in.  The device address is looked up with
 // cudaGetSymbolAddress, with the device current, on the first call made in
 // each device context (and again if the context changes, e.g. after a
-// cudaDeviceReset); make that first call before any stream capture.  Every call
+// cudaDeviceReset); later calls in the context reuse it.  Every call
 // shares the array, so calls that may overlap on the GPU (different streams,
 // or different host threads on one device) race on it and must be ordered by
 // the caller.  This entry point never splits a sequence's keys among CTAs (the
