@@ -673,6 +673,8 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
                                                          float* __restrict__ st_m,
                                                          float* __restrict__ st_l) {
   constexpr int PER = HD / 32;  // floats per lane
+  griddep_wait();               // the shares are written by the attention launch before
+  griddep_launch_dependents();  // the O projection may start streaming its weights
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int h = blockIdx.y, lane = threadIdx.x & 31;
   if (r >= min(*M_dev, part_rows)) return;
@@ -771,14 +773,21 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
   cudaError_t e = hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
                             : launch_hd<64, false>(tq, tk, tv, tk, tv, p, grid, s);
   if (e != cudaSuccess || S == 1) return e;
-  dim3 mgrid((M_cap + 7) / 8, Hq);
-  if (hd == 128)
-    attn_merge_kernel<128><<<mgrid, 256, 0, s>>>(part_o, part_ml, S, M_cap, row_off + B, Hq, o,
-                                                 Hq * hd, st_m, st_l);
-  else
-    attn_merge_kernel<64><<<mgrid, 256, 0, s>>>(part_o, part_ml, S, M_cap, row_off + B, Hq, o,
-                                                Hq * hd, st_m, st_l);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((M_cap + 7) / 8, Hq);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute la[1];
+  la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  la[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = la;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return hd == 128 ? cudaLaunchKernelEx(&cfg, attn_merge_kernel<128>, (const float*)part_o,
+                                        (const float*)part_ml, S, M_cap, row_off + B, Hq, o,
+                                        Hq * hd, st_m, st_l)
+                   : cudaLaunchKernelEx(&cfg, attn_merge_kernel<64>, (const float*)part_o,
+                                        (const float*)part_ml, S, M_cap, row_off + B, Hq, o,
+                                        Hq * hd, st_m, st_l);
 }
 
 cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bfloat16* o,
