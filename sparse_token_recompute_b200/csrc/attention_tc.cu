@@ -3,7 +3,7 @@
 // The selected query rows of each sequence attend to all N cached keys of
 // that sequence, bidirectionally: O = softmax(Q K^T / sqrt(hd)) V.
 //
-// One CTA = one (sequence, query head) and up to two tiles of 128 compact
+// One CTA = one (sequence, query head) and up to NT = 2 tiles of 128 compact
 // query rows (A and B) that share every K/V tile.  Warp roles (320 threads):
 //   warp 0     TMA producer: both Q tiles once, then K and V tiles of 128 keys
 //              through one ring of shared-memory slots (128-byte-swizzled
@@ -11,6 +11,10 @@
 //   warp 1     TMEM owner and tcgen05.mma issuer;
 //   warps 2-5  softmax of tile A, warps 6-9 softmax of tile B: one query row
 //              per thread (its TMEM lane).
+// With NT = 1 a CTA holds one tile (192 threads, 256 TMEM columns, under half
+// the shared memory) and two CTAs share each SM: their MMAs and softmax
+// interleave as the two groups of a pair do, and one CTA's start-up and
+// epilogue overlap the other's main loop.
 // TMEM holds S_A, S_B (fp32, 128 columns each) and O_A, O_B.  Each softmax
 // group reads S_X, exponentiates against a per-row reference maximum and
 // writes P_X back over the first 64 columns of S_X as packed bf16 pairs; the
@@ -37,29 +41,36 @@ namespace dllm {
 namespace {
 
 constexpr int BT = 128;       // query rows per tile (= TMEM lanes)
-constexpr int NTILE = 2;      // query tiles per CTA
 constexpr int BKV = 128;      // keys per K/V tile
-constexpr int NTHREADS = 64 + NTILE * 128;
-constexpr uint32_t TMEM_COLS = 512;  // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSmemMax = 227 * 1024;  // dynamic shared memory a block may opt in to
 
-template <int HD>
+// NT query tiles per CTA: 2 (a pair sharing every K/V tile, one CTA per SM
+// holding all 512 TMEM columns) or 1 (one tile, 256 TMEM columns and under
+// half the shared memory, two CTAs per SM)
+template <int NT>
+constexpr int nthreads() { return 64 + NT * 128; }
+template <int NT>
+constexpr uint32_t tmem_cols() { return NT * 256u; }  // S_X at 128 x, O_X at 128 (NT + x)
+
+template <int HD, int NT>
 struct Smem {
   static constexpr int Q_TILE = BT * HD * 2;     // HD/64 boxes of 128 rows x 128 B
   static constexpr int KV_BYTES = BKV * HD * 2;
   // K and V tiles share one ring of slots in consumption order K0 V0 K1 V1 ...,
-  // as many as fit next to the two Q tiles (at most 8)
-  static constexpr int SLOTS_FIT = (kSmemMax - 2304 - NTILE * Q_TILE) / KV_BYTES;
+  // as many as fit next to the Q tiles (at most 8) in this CTA's share of the SM
+  static constexpr int BUDGET = NT == 2 ? kSmemMax : 112 * 1024;
+  static constexpr int SLOTS_FIT = (BUDGET - 2304 - 1024 - NT * Q_TILE) / KV_BYTES;
   static constexpr int SLOTS = SLOTS_FIT < 8 ? SLOTS_FIT : 8;
   static constexpr int Q_OFF = 0;
-  static constexpr int RING_OFF = Q_OFF + NTILE * Q_TILE;
+  static constexpr int RING_OFF = Q_OFF + NT * Q_TILE;
   static constexpr int BAR_OFF = RING_OFF + SLOTS * KV_BYTES;
   static constexpr int STAT_OFF = BAR_OFF + 256;  // 2 x 128 floats for the key-split merge
-  // + barriers + alignment slack; at least 116 KB so that one CTA (which holds
-  // all 512 TMEM columns) is resident per SM
-  static constexpr int TOTAL = (STAT_OFF + 1024 + 1024) > 116 * 1024 ? (STAT_OFF + 1024 + 1024)
-                                                                     : 116 * 1024;
+  // + barriers + alignment slack; a pair CTA takes at least 116 KB so that one
+  // CTA (which holds all 512 TMEM columns) is resident per SM
+  static constexpr int NEED = STAT_OFF + 1024 + 1024;
+  static constexpr int TOTAL = (NT == 1 || NEED > 116 * 1024) ? NEED : 116 * 1024;
+  static_assert(NT == 2 || 2 * (TOTAL + 1024) <= 228 * 1024, "two one-tile CTAs per SM");
 };
 
 struct AttnParams {
@@ -172,12 +183,12 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 // with their old values (tmK2, tmV2) entering the sums with a negative sign; the
 // reference maximum starts at the row's cached m, and the epilogue merges the
 // sums into the cached (m, l, o).
-template <int HD, bool UPD>
-__global__ void __launch_bounds__(NTHREADS, 1)
+template <int HD, bool UPD, int NT>
+__global__ void __launch_bounds__(nthreads<NT>(), NT == 1 ? 2 : 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
                    const __grid_constant__ CUtensorMap tmV2, const AttnParams p) {
-  using L = Smem<HD>;
+  using L = Smem<HD, NT>;
   constexpr int NB = HD / 64;  // 64-column boxes per row of Q/K/V
   constexpr float kLog2e = 1.4426950408889634f;
   griddep_wait();  // everything below reads what earlier kernels wrote
@@ -192,8 +203,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int S_kv = UPD ? 1 : p.kv_split;           // CTAs sharing a pair's keys
   const int s_kv = UPD ? 0 : (int)blockIdx.x % S_kv;  // this CTA's share
   const int pair0 = (UPD ? blockIdx.x : blockIdx.x / S_kv) * ppc;
-  auto pair_q0 = [&](int i) { return (pair0 + i) * (NTILE * BT); };
-  const int npairs = UPD ? min(ppc, (cnt - pair_q0(0) + NTILE * BT - 1) / (NTILE * BT))
+  auto pair_q0 = [&](int i) { return (pair0 + i) * (NT * BT); };
+  const int npairs = UPD ? min(ppc, (cnt - pair_q0(0) + NT * BT - 1) / (NT * BT))
                          : (pair_q0(0) < cnt ? 1 : 0);
   if (npairs <= 0) return;
   const int q0 = pair_q0(0);
@@ -211,12 +222,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   auto tile_keys = [&](int t) {
     return UPD ? min(BKV, a_cnt - (t % TH) * BKV) : min(BKV, p.Nseq - (k_lo + t) * BKV);
   };
-  auto pair_nq = [&](int i) { return (cnt - pair_q0(i) > BT) ? 2 : 1; };  // tiles with rows
+  auto pair_nq = [&](int i) { return (NT == 2 && cnt - pair_q0(i) > BT) ? 2 : 1; };
   const int nq = pair_nq(0);
   // A lone query tile splits the keys instead (one pair per CTA only): group A
   // takes K/V tiles [0, TA), group B [TA, T), and the two partial softmax
   // results are merged at the end.
-  const bool split = !UPD && !multi && nq == 1 && T >= 2;
+  const bool split = NT == 2 && !UPD && !multi && nq == 1 && T >= 2;
   const int TA = split ? (T + 1) / 2 : T;
   const int TB = split ? T - TA : T;
   const int ngroups = (nq == 2 || split) ? 2 : 1;
@@ -281,7 +292,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), tmem_cols<NT>());
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -298,7 +309,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   auto tS = [&](int x) { return tmem + (uint32_t)(x * 128); };
-  auto tO = [&](int x) { return tmem + 256u + (uint32_t)(x * 128); };
+  auto tO = [&](int x) { return tmem + (uint32_t)(NT * 128 + x * 128); };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -657,7 +668,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, tmem_cols<NT>());
   }
 }
 
@@ -705,16 +716,16 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
   }
 }
 
-template <int HD, bool UPD>
+template <int HD, bool UPD, int NT>
 cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                       const CUtensorMap& k2, const CUtensorMap& v2, const AttnParams& p, dim3 grid,
                       cudaStream_t s) {
-  constexpr int smem = Smem<HD>::TOTAL;
-  const cudaError_t ea = ensure_smem_attr<attn_tc_kernel<HD, UPD>>(smem);
+  constexpr int smem = Smem<HD, NT>::TOTAL;
+  const cudaError_t ea = ensure_smem_attr<attn_tc_kernel<HD, UPD, NT>>(smem);
   if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(NTHREADS);
+  cfg.blockDim = dim3(nthreads<NT>());
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute la[1];
@@ -722,25 +733,29 @@ cudaError_t launch_hd(const CUtensorMap& q, const CUtensorMap& k, const CUtensor
   la[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = la;
   cfg.numAttrs = pdl_enabled() ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<HD, UPD>, q, k, v, k2, v2, p);
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel<HD, UPD, NT>, q, k, v, k2, v2, p);
 }
 
 }  // namespace
 
-int attention_kv_split(int B, int k_cap, int Nseq, int Hq) {
-  // few (sequence, head, pair) CTAs leave most SMs idle: share each pair's keys
-  // among up to 8 CTAs, at least two K/V tiles each
+int attention_kv_split(int B, int k_cap, int Nseq, int Hq, int NT) {
+  // few CTAs leave most SMs idle: share each CTA's keys among up to 8 CTAs (one
+  // CTA per SM with pairs of query tiles, whose two groups split a lone tile's
+  // keys again, so at least two K/V tiles per share; two per SM with one tile)
   const int T = (Nseq + BKV - 1) / BKV;
-  const int ctas = ((k_cap + NTILE * BT - 1) / (NTILE * BT)) * Hq * B;
-  if (ctas <= 0 || 2 * ctas > num_sms() || T < 4) return 1;
-  int S = std::max(1, std::min(std::min(8, T / 2), num_sms() / ctas));
+  const int ctas = ((k_cap + NT * BT - 1) / (NT * BT)) * Hq * B;
+  const int slots = (NT == 1 ? 2 : 1) * num_sms();  // resident CTAs
+  const int min_tiles = NT == 1 ? 1 : 2;
+  if (ctas <= 0 || 2 * ctas > slots || T < 2 * min_tiles) return 1;
+  int S = std::max(1, std::min(std::min(8, T / min_tiles), slots / ctas));
   while (S > 1 && (S - 1) * ((T + S - 1) / S) >= T) --S;  // every share holds keys
   return S;
 }
 
 size_t attention_part_bytes_bound(int cap, int Hq, int hd) {
   // a split launch has S * rows <= SMs * (rows of a pair) for any batch shape
-  const size_t rows = std::min((size_t)8 * cap * Hq, (size_t)num_sms() * NTILE * BT);
+  // (S x CTAs <= resident CTAs: SMs x 2 tiles of 128 rows either way)
+  const size_t rows = std::min((size_t)8 * cap * Hq, (size_t)num_sms() * 2 * BT);
   return rows * (hd + 2) * sizeof(float);
 }
 
@@ -761,17 +776,32 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
     return cudaErrorInvalidValue;
   if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
     return cudaErrorInvalidValue;
-  int S = part ? attention_kv_split(B, k_cap, Nseq, Hq) : 1;
+  // Query tiles per CTA.  A pair of tiles shares each K/V tile, but an odd tile
+  // count leaves a lone last tile whose CTA streams the keys again at half the
+  // work (32 x 308 rows, 1536 keys: 0.426 ms); one tile per CTA with two CTAs
+  // per SM avoids it (0.367 ms), at a cost where the tiles pair up evenly (256
+  // rows: 0.244 ms in pairs, 0.259 ms singly) or where long runs of pairs
+  // outweigh the one lone tile (estimated past 7 tiles).  With few tiles in all,
+  // one-tile CTAs also split the keys among twice as many CTAs.
+  const int tiles = (k_cap + BT - 1) / BT;
+  const int S1 = part ? attention_kv_split(B, k_cap, Nseq, Hq, 1) : 1;
+  const int NT = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3 && tiles <= 7)) ? 1 : 2;
+  int S = NT == 1 ? S1 : (part ? attention_kv_split(B, k_cap, Nseq, Hq, 2) : 1);
   if (S > 1 && attention_part_bytes(S, M_cap, Hq, hd) > part_bytes) S = 1;
   float* part_o = S > 1 ? part : nullptr;
   float* part_ml = S > 1 ? part + (size_t)S * M_cap * Hq * hd : nullptr;
   AttnParams p{row_off, o,      Nseq, Hq,      Hkv,    Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
                status,  st_m,   st_l, nullptr, 1,      S,       M_cap,
                part_o,  part_ml, nullptr};
-  dim3 grid(((k_cap + NTILE * BT - 1) / (NTILE * BT)) * S, Hq, B);
+  dim3 grid(((k_cap + NT * BT - 1) / (NT * BT)) * S, Hq, B);
   ProfScope prof("attention", s);
-  cudaError_t e = hd == 128 ? launch_hd<128, false>(tq, tk, tv, tk, tv, p, grid, s)
-                            : launch_hd<64, false>(tq, tk, tv, tk, tv, p, grid, s);
+  cudaError_t e;
+  if (NT == 1)
+    e = hd == 128 ? launch_hd<128, false, 1>(tq, tk, tv, tk, tv, p, grid, s)
+                  : launch_hd<64, false, 1>(tq, tk, tv, tk, tv, p, grid, s);
+  else
+    e = hd == 128 ? launch_hd<128, false, 2>(tq, tk, tv, tk, tv, p, grid, s)
+                  : launch_hd<64, false, 2>(tq, tk, tv, tk, tv, p, grid, s);
   if (e != cudaSuccess || S == 1) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((M_cap + 7) / 8, Hq);
@@ -808,7 +838,7 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
     return cudaErrorInvalidValue;
   // few changed keys make short key streams: a CTA takes several pairs of query
   // tiles of its (sequence, head) in turn, keeping about two CTAs per SM in flight
-  const int pairs = (r_cap + NTILE * BT - 1) / (NTILE * BT);
+  const int pairs = (r_cap + 2 * BT - 1) / (2 * BT);
   const int min_x = std::max(1, (2 * num_sms() + B * Hq - 1) / (B * Hq));
   const int ppc = std::max(1, (pairs + min_x - 1) / min_x);
   AttnParams p{r_off, o,    0,    Hq,   Hkv,   Hq * hd, 1.4426950408889634f / sqrtf((float)hd),
@@ -816,8 +846,8 @@ cudaError_t launch_attention_update(const __nv_bfloat16* q, int R_cap, __nv_bflo
                nullptr, nullptr, skip};
   dim3 grid((pairs + ppc - 1) / ppc, Hq, B);
   ProfScope prof("attention_update", s);
-  return hd == 128 ? launch_hd<128, true>(tq, tk, tv, tk2, tv2, p, grid, s)
-                   : launch_hd<64, true>(tq, tk, tv, tk2, tv2, p, grid, s);
+  return hd == 128 ? launch_hd<128, true, 2>(tq, tk, tv, tk2, tv2, p, grid, s)
+                   : launch_hd<64, true, 2>(tq, tk, tv, tk2, tv2, p, grid, s);
 }
 
 }  // namespace dllm

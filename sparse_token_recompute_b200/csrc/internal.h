@@ -154,9 +154,9 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
                                 int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
                                 cudaStream_t s, float* st_m = nullptr, float* st_l = nullptr,
                                 float* part = nullptr, size_t part_bytes = 0);
-// key shares per pair of query tiles the attention uses for this shape (1: none), and
+// key shares per CTA of NT query tiles the attention uses for this shape (1: none), and
 // the partial-output scratch (fp32) that launch_attention_tc then needs in `part`
-int attention_kv_split(int B, int k_cap, int Nseq, int Hq);
+int attention_kv_split(int B, int k_cap, int Nseq, int Hq, int NT);
 size_t attention_part_bytes(int S, int M_cap, int Hq, int hd);
 // scratch that covers the split of any launch over at most `cap` rows
 size_t attention_part_bytes_bound(int cap, int Hq, int hd);
