@@ -778,14 +778,14 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
     return cudaErrorInvalidValue;
   // Query tiles per CTA.  A pair of tiles shares each K/V tile, but an odd tile
   // count leaves a lone last tile whose CTA streams the keys again at half the
-  // work (32 x 308 rows, 1536 keys: 0.426 ms); one tile per CTA with two CTAs
-  // per SM avoids it (0.367 ms), at a cost where the tiles pair up evenly (256
-  // rows: 0.244 ms in pairs, 0.259 ms singly) or where long runs of pairs
-  // outweigh the one lone tile (estimated past 7 tiles).  With few tiles in all,
-  // one-tile CTAs also split the keys among twice as many CTAs.
+  // work; one tile per CTA with two CTAs per SM avoids it (32 sequences, 1536
+  // keys: 308 rows 0.426 -> 0.367 ms, 1152 rows 1.047 -> 1.029, 1664 rows
+  // 1.475 -> 1.455), at a cost where the tiles pair up evenly (256 rows: 0.244
+  // ms in pairs, 0.259 ms singly).  With few tiles in all, one-tile CTAs also
+  // split the keys among twice as many CTAs.
   const int tiles = (k_cap + BT - 1) / BT;
   const int S1 = part ? attention_kv_split(B, k_cap, Nseq, Hq, 1) : 1;
-  const int NT = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3 && tiles <= 7)) ? 1 : 2;
+  const int NT = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3)) ? 1 : 2;
   int S = NT == 1 ? S1 : (part ? attention_kv_split(B, k_cap, Nseq, Hq, 2) : 1);
   if (S > 1 && attention_part_bytes(S, M_cap, Hq, hd) > part_bytes) S = 1;
   float* part_o = S > 1 ? part : nullptr;
