@@ -538,6 +538,21 @@ dllm_status dllm_gemm_plan_info(int kind, int M, int K, const int32_t* seg_cols,
                                 int head_dim, int32_t* out);
 
 /*
+ * dllm_attention_plan_info - the launch plan of the exact partial attention
+ * (host only; with no device visible 148 SMs are assumed).  B sequences of N
+ * cached keys, at most k_cap selected query rows each, n_heads query heads of
+ * head_dim (64 or 128); in_step != 0 for the plan inside a step (whose layer
+ * workspace holds the key-split scratch), 0 for dllm_attention_bf16 alone.
+ * out (HOST, 3 int32): query tiles of 128 rows per CTA (2: a pair sharing every
+ * K/V tile, one CTA per SM; 1: two CTAs per SM, taken for an odd tile count of
+ * 3 or more and when keys are split), key shares per CTA's rows (1: none), CTAs
+ * launched.  DLLM_ERR_INVALID_ARG for non-positive sizes, another head_dim or
+ * a null out.
+ */
+dllm_status dllm_attention_plan_info(int B, int k_cap, int N, int n_heads, int head_dim,
+                                     int in_step, int32_t* out);
+
+/*
  * dllm_selftest_gemm_stall - failure-path check of the CTA-pair GEMM (256-row
  * tiles, tcgen05 cta_group::2): the same launch as dllm_gemm_bf16 (M >= 256,
  * N a multiple of 256, accumulate 0, no K split) with one signal withheld:

@@ -131,6 +131,7 @@ _gemm_ws = _sig("dllm_gemm_workspace_size", _sz, [_i, _i, _i, _i])
 _gemm = _sig("dllm_gemm_bf16", _i, [vp, vp, vp, _i, _i, _i, _i, _i, vp, _sz, vp])
 _gemm_stall = _sig("dllm_selftest_gemm_stall", _i, [vp, vp, vp, _i, _i, _i, vp, _sz, vp])
 _gemm_plan = _sig("dllm_gemm_plan_info", _i, [_i, _i, _i, vp, _i, _i, vp])
+_attn_plan = _sig("dllm_attention_plan_info", _i, [_i, _i, _i, _i, _i, _i, vp])
 _prof_enable = _sig("dllm_profile_enable", None, [_i])
 _prof_reset = _sig("dllm_profile_reset", None, [])
 _prof_read = _sig("dllm_profile_read", _sz, [C.c_char_p, _sz])
@@ -293,6 +294,16 @@ def dllm_gemm_plan_info(kind: str, M: int, K: int, seg_cols, head_dim: int = 0) 
                     int(head_dim), C.cast(out, C.c_void_p))
     _check(st, "dllm_gemm_plan_info")
     return {"bn": out[0], "splits": out[1], "tiles_n": out[2], "grid": out[3], "pair": out[4]}
+
+
+def dllm_attention_plan_info(B: int, k_cap: int, N: int, n_heads: int, head_dim: int,
+                             in_step: bool = True) -> Dict[str, int]:
+    """The host-side launch plan of the exact partial attention (no GPU work)."""
+    out = (C.c_int32 * 3)()
+    st = _attn_plan(int(B), int(k_cap), int(N), int(n_heads), int(head_dim), int(bool(in_step)),
+                    C.cast(out, C.c_void_p))
+    _check(st, "dllm_attention_plan_info")
+    return {"tiles_per_cta": out[0], "key_shares": out[1], "ctas": out[2]}
 
 
 def dllm_selftest_gemm_stall(A, Bm, Cm, ws: Workspace = None, stream=None):

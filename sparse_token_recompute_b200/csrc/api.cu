@@ -668,6 +668,21 @@ extern "C" dllm_status dllm_gemm_plan_info(int kind, int M, int K, const int32_t
   return DLLM_OK;
 }
 
+extern "C" dllm_status dllm_attention_plan_info(int B, int k_cap, int N, int n_heads,
+                                                int head_dim, int in_step, int32_t* out) {
+  if (B <= 0 || k_cap <= 0 || N <= 0 || n_heads <= 0 || !out ||
+      (head_dim != 64 && head_dim != 128))
+    return DLLM_ERR_INVALID_ARG;
+  // in a step the layer workspace carries the key-split scratch; the attention
+  // entry points alone have none
+  const size_t part = in_step ? attention_part_bytes_bound(B * N, n_heads, head_dim) : 0;
+  const AttnPlan pl = attention_plan(B, k_cap, N, n_heads, head_dim, B * k_cap, part);
+  out[0] = pl.nt;
+  out[1] = pl.shares;
+  out[2] = pl.ctas;
+  return DLLM_OK;
+}
+
 extern "C" dllm_status dllm_selftest_gemm_stall(const void* A, const void* Bm, void* C, int M,
                                                 int N, int K, void* ws, size_t ws_bytes,
                                                 dllm_stream_t stream) {

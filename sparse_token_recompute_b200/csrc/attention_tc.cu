@@ -763,6 +763,26 @@ size_t attention_part_bytes(int S, int M_cap, int Hq, int hd) {
   return S > 1 ? (size_t)S * M_cap * Hq * (hd + 2) * sizeof(float) : 0;
 }
 
+AttnPlan attention_plan(int B, int k_cap, int Nseq, int Hq, int hd, int M_cap,
+                        size_t part_bytes) {
+  // Query tiles per CTA.  A pair of tiles shares each K/V tile, but an odd tile
+  // count leaves a lone last tile whose CTA streams the keys again at half the
+  // work; one tile per CTA with two CTAs per SM avoids it (32 sequences, 1536
+  // keys: 308 rows 0.426 -> 0.367 ms, 1152 rows 1.047 -> 1.029, 1664 rows
+  // 1.475 -> 1.455), at a cost where the tiles pair up evenly (256 rows: 0.244
+  // ms in pairs, 0.259 ms singly).  With few tiles in all, one-tile CTAs also
+  // split the keys among twice as many CTAs (given scratch for the shares).
+  AttnPlan pl{};
+  const int tiles = (k_cap + BT - 1) / BT;
+  const int S1 = part_bytes ? attention_kv_split(B, k_cap, Nseq, Hq, 1) : 1;
+  pl.nt = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3)) ? 1 : 2;
+  pl.shares = pl.nt == 1 ? S1 : (part_bytes ? attention_kv_split(B, k_cap, Nseq, Hq, 2) : 1);
+  if (pl.shares > 1 && attention_part_bytes(pl.shares, M_cap, Hq, hd) > part_bytes)
+    pl.shares = 1;
+  pl.ctas = ((k_cap + pl.nt * BT - 1) / (pl.nt * BT)) * pl.shares * Hq * B;
+  return pl;
+}
+
 cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bfloat16* kc,
                                 const __nv_bfloat16* vc, __nv_bfloat16* o, const int* row_off,
                                 int B, int k_cap, int Nseq, int Hq, int Hkv, int hd, int* status,
@@ -776,18 +796,8 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
     return cudaErrorInvalidValue;
   if (!tmap_bf16_2d(&tv, vc, (uint64_t)B * Nseq, (uint64_t)Hkv * hd, BKV))
     return cudaErrorInvalidValue;
-  // Query tiles per CTA.  A pair of tiles shares each K/V tile, but an odd tile
-  // count leaves a lone last tile whose CTA streams the keys again at half the
-  // work; one tile per CTA with two CTAs per SM avoids it (32 sequences, 1536
-  // keys: 308 rows 0.426 -> 0.367 ms, 1152 rows 1.047 -> 1.029, 1664 rows
-  // 1.475 -> 1.455), at a cost where the tiles pair up evenly (256 rows: 0.244
-  // ms in pairs, 0.259 ms singly).  With few tiles in all, one-tile CTAs also
-  // split the keys among twice as many CTAs.
-  const int tiles = (k_cap + BT - 1) / BT;
-  const int S1 = part ? attention_kv_split(B, k_cap, Nseq, Hq, 1) : 1;
-  const int NT = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3)) ? 1 : 2;
-  int S = NT == 1 ? S1 : (part ? attention_kv_split(B, k_cap, Nseq, Hq, 2) : 1);
-  if (S > 1 && attention_part_bytes(S, M_cap, Hq, hd) > part_bytes) S = 1;
+  const AttnPlan pl = attention_plan(B, k_cap, Nseq, Hq, hd, M_cap, part ? part_bytes : 0);
+  const int NT = pl.nt, S = pl.shares;
   float* part_o = S > 1 ? part : nullptr;
   float* part_ml = S > 1 ? part + (size_t)S * M_cap * Hq * hd : nullptr;
   AttnParams p{row_off, o,      Nseq, Hq,      Hkv,    Hq * hd, 1.4426950408889634f / sqrtf((float)hd),

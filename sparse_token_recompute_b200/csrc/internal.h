@@ -157,6 +157,14 @@ cudaError_t launch_attention_tc(const __nv_bfloat16* q, int M_cap, const __nv_bf
 // key shares per CTA of NT query tiles the attention uses for this shape (1: none), and
 // the partial-output scratch (fp32) that launch_attention_tc then needs in `part`
 int attention_kv_split(int B, int k_cap, int Nseq, int Hq, int NT);
+// the exact attention's launch plan: query tiles per CTA (1: two CTAs per SM, 2:
+// a pair sharing each K/V tile), key shares per CTA's rows (needs part scratch of
+// part_bytes), CTAs launched
+struct AttnPlan {
+  int nt, shares, ctas;
+};
+AttnPlan attention_plan(int B, int k_cap, int Nseq, int Hq, int hd, int M_cap,
+                        size_t part_bytes);
 size_t attention_part_bytes(int S, int M_cap, int Hq, int hd);
 // scratch that covers the split of any launch over at most `cap` rows
 size_t attention_part_bytes_bound(int cap, int Hq, int hd);

@@ -113,6 +113,29 @@ def test_gemm_plans_of_the_benchmarked_shapes(lib):
             assert p["pair"] in (0, 1) and (not p["pair"] or p["grid"] % 2 == 0)
 
 
+def test_attention_plans_of_the_benchmarked_shapes(lib):
+    """The host-side attention plan (no GPU: 148 SMs assumed): one query tile per
+    CTA (two CTAs per SM) for an odd tile count of three or more and wherever the
+    keys are split among CTAs; pairs of tiles sharing each K/V tile otherwise."""
+    import sparse_token_recompute_b200 as S
+    P = S.dllm_attention_plan_info
+    plan = lambda *a, **kw: tuple(P(*a, **kw).values())
+    assert plan(32, 308, 1536, 32, 128) == (1, 1, 3072)      # the 32-sequence step: 3 tiles
+    assert plan(32, 308, 1536, 28, 128) == (1, 1, 2688)      # 7B GQA heads, 3 tiles
+    assert plan(32, 256, 1536, 32, 128) == (2, 1, 1024)      # 2 tiles: pairs
+    assert plan(32, 1536, 1536, 32, 128) == (2, 1, 6144)     # dense step: 12 tiles
+    assert plan(32, 640, 1536, 32, 128)[0] == 1              # 5 tiles
+    assert plan(1, 77, 768, 32, 128) == (1, 6, 192)          # one sequence: keys in 6 shares
+    assert plan(1, 192, 768, 32, 128) == (1, 3, 192)
+    assert plan(1, 77, 768, 32, 128, in_step=False) == (2, 1, 32)   # no scratch: no shares
+    # resident CTAs: one per SM with pairs, two per SM with one tile
+    for args in [(1, 77, 768, 32, 128), (1, 384, 768, 32, 128), (2, 300, 4096, 8, 64)]:
+        nt, shares, ctas = plan(*args)
+        assert ctas <= (2 if nt == 1 else 1) * 148 or shares == 1
+    with pytest.raises(RuntimeError):
+        P(1, 77, 768, 32, 96)
+
+
 def test_gemm_plan_rejects_bad_arguments(lib):
     import sparse_token_recompute_b200 as S
     segs = (C.c_int32 * 3)(4096, 4096, 4096)
