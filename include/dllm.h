@@ -545,7 +545,8 @@ dllm_status dllm_gemm_plan_info(int kind, int M, int K, const int32_t* seg_cols,
  * workspace holds the key-split scratch), 0 for dllm_attention_bf16 alone.
  * out (HOST, 3 int32): query tiles of 128 rows per CTA (2: a pair sharing every
  * K/V tile, one CTA per SM; 1: two CTAs per SM, taken for an odd tile count of
- * 3 or more and when keys are split), key shares per CTA's rows (1: none), CTAs
+ * 3 or more, when keys are split, and when one-tile CTAs fit one wave where
+ * pairs would need two), key shares per CTA's rows (1: none), CTAs
  * launched.  DLLM_ERR_INVALID_ARG for non-positive sizes, another head_dim or
  * a null out.
  */

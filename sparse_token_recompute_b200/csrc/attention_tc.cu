@@ -771,11 +771,16 @@ AttnPlan attention_plan(int B, int k_cap, int Nseq, int Hq, int hd, int M_cap,
   // keys: 308 rows 0.426 -> 0.367 ms, 1152 rows 1.047 -> 1.029, 1664 rows
   // 1.475 -> 1.455), at a cost where the tiles pair up evenly (256 rows: 0.244
   // ms in pairs, 0.259 ms singly).  With few tiles in all, one-tile CTAs also
-  // split the keys among twice as many CTAs (given scratch for the shares).
+  // split the keys among twice as many CTAs (given scratch for the shares), and
+  // fit one wave where pairs would need two (8 sequences x 28 heads, one tile
+  // each, 2048 keys: 0.057 -> 0.052 ms).
   AttnPlan pl{};
   const int tiles = (k_cap + BT - 1) / BT;
   const int S1 = part_bytes ? attention_kv_split(B, k_cap, Nseq, Hq, 1) : 1;
-  pl.nt = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3)) ? 1 : 2;
+  const long long ctas2 = (long long)((tiles + 1) / 2) * Hq * B;  // pairs, one per SM
+  const long long ctas1 = (long long)tiles * Hq * B;              // one tile, two per SM
+  const bool one_wave = ctas2 > num_sms() && ctas1 <= 2LL * num_sms();
+  pl.nt = (S1 > 1 || (tiles % 2 == 1 && tiles >= 3) || one_wave) ? 1 : 2;
   pl.shares = pl.nt == 1 ? S1 : (part_bytes ? attention_kv_split(B, k_cap, Nseq, Hq, 2) : 1);
   if (pl.shares > 1 && attention_part_bytes(pl.shares, M_cap, Hq, hd) > part_bytes)
     pl.shares = 1;

@@ -128,6 +128,8 @@ def test_attention_plans_of_the_benchmarked_shapes(lib):
     assert plan(1, 77, 768, 32, 128) == (1, 6, 192)          # one sequence: keys in 6 shares
     assert plan(1, 192, 768, 32, 128) == (1, 3, 192)
     assert plan(1, 77, 768, 32, 128, in_step=False) == (2, 1, 32)   # no scratch: no shares
+    assert plan(8, 103, 2048, 28, 128) == (1, 1, 224)       # one wave singly, two in pairs
+    assert plan(8, 205, 2048, 28, 128) == (2, 1, 224)
     # resident CTAs: one per SM with pairs, two per SM with one tile
     for args in [(1, 77, 768, 32, 128), (1, 384, 768, 32, 128), (2, 300, 4096, 8, 64)]:
         nt, shares, ctas = plan(*args)
