@@ -491,10 +491,11 @@ dllm_status dllm_attention_update_bf16(const void* q, void* o, float* m, float* 
  * the GPU (other streams, other host threads on the same device) race and
  * must be ordered by the caller.  Device-side faults are recorded in the
  * shared status word, which this entry point clears at the start of each call
- * and does not report.  It never splits one sequence's keys among several
- * CTAs (that needs a partial-output scratch far larger than the fixed array),
- * so with few query tiles (one or two sequences of a few hundred selected
- * rows) it runs fewer CTAs than dllm_attention_bf16 and can be slower.
+ * and does not report.  Like dllm_attention_bf16, it never splits one
+ * sequence's keys among several CTAs (that needs a partial-output scratch far
+ * larger than the fixed array); the attention inside dllm_step and
+ * dllm_partial_layer does, so with few query tiles (one or two sequences of a
+ * few hundred selected rows) it runs fewer CTAs than those and can be slower.
  */
 #define DLLM_NOALLOC_MAX_SEQS 4096
 dllm_status dllm_attention_bf16_noalloc(const void* q, const void* k_cache, const void* v_cache,

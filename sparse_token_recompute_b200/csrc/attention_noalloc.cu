@@ -19,10 +19,11 @@
 // cudaDeviceReset); later calls in the context reuse it.  Every call
 // shares the array, so calls that may overlap on the GPU (different streams,
 // or different host threads on one device) race on it and must be ordered by
-// the caller.  This entry point never splits a sequence's keys among CTAs (the
-// split needs a partial-output scratch far larger than the fixed array), so
-// with few query tiles -- one or two sequences of a few hundred selected rows --
-// it runs fewer CTAs than dllm_attention_bf16 and can be slower.
+// the caller.  Like dllm_attention_bf16, this entry point never splits a
+// sequence's keys among CTAs (the split needs a partial-output scratch far
+// larger than the fixed array); the attention inside a step does, so with few
+// query tiles -- one or two sequences of a few hundred selected rows -- it runs
+// fewer CTAs than the step's attention and can be slower.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
