@@ -44,6 +44,7 @@ constexpr int BT = 128;       // query rows per tile (= TMEM lanes)
 constexpr int BKV = 128;      // keys per K/V tile
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kSmemMax = 227 * 1024;  // dynamic shared memory a block may opt in to
+constexpr int kMaxShares = 8;         // key shares of a split exact attention, at most
 
 // NT query tiles per CTA: 2 (a pair sharing every K/V tile, one CTA per SM
 // holding all 512 TMEM columns) or 1 (one tile, 256 TMEM columns and under
@@ -689,19 +690,34 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const float* __restrict
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int h = blockIdx.y, lane = threadIdx.x & 31;
   if (r >= min(*M_dev, part_rows)) return;
+  // every share's (m, l) and output slice in flight at once (at most 8 shares)
+  float2 ml[kMaxShares];
+  float o[kMaxShares][PER];
+#pragma unroll
+  for (int sh = 0; sh < kMaxShares; ++sh) {
+    if (sh < S) {
+      const size_t base = ((size_t)sh * part_rows + r) * Hq + h;
+      ml[sh] = *reinterpret_cast<const float2*>(part_ml + base * 2);
+      const float* src = part_o + base * HD + lane * PER;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) o[sh][i] = src[i];
+    }
+  }
   float mx = -INFINITY;
-  for (int sh = 0; sh < S; ++sh)
-    mx = fmaxf(mx, part_ml[(((size_t)sh * part_rows + r) * Hq + h) * 2]);
+#pragma unroll
+  for (int sh = 0; sh < kMaxShares; ++sh)
+    if (sh < S) mx = fmaxf(mx, ml[sh].x);
   float acc[PER], L = 0.f;
 #pragma unroll
   for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-  for (int sh = 0; sh < S; ++sh) {
-    const size_t base = ((size_t)sh * part_rows + r) * Hq + h;
-    const float w = part_ml[base * 2 + 1] * ex2_approx(part_ml[base * 2] - mx);
-    L += w;
-    const float* src = part_o + base * HD + lane * PER;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, src[i], acc[i]);
+  for (int sh = 0; sh < kMaxShares; ++sh) {
+    if (sh < S) {
+      const float w = ml[sh].y * ex2_approx(ml[sh].x - mx);
+      L += w;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) acc[i] = fmaf(w, o[sh][i], acc[i]);
+    }
   }
   const float inv = 1.0f / L;
   __nv_bfloat16* dst = O + (size_t)r * ldo + h * HD + lane * PER;
@@ -747,7 +763,7 @@ int attention_kv_split(int B, int k_cap, int Nseq, int Hq, int NT) {
   const int slots = (NT == 1 ? 2 : 1) * num_sms();  // resident CTAs
   const int min_tiles = NT == 1 ? 1 : 2;
   if (ctas <= 0 || 2 * ctas > slots || T < 2 * min_tiles) return 1;
-  int S = std::max(1, std::min(std::min(8, T / min_tiles), slots / ctas));
+  int S = std::max(1, std::min(std::min(kMaxShares, T / min_tiles), slots / ctas));
   while (S > 1 && (S - 1) * ((T + S - 1) / S) >= T) --S;  // every share holds keys
   return S;
 }
@@ -755,7 +771,7 @@ int attention_kv_split(int B, int k_cap, int Nseq, int Hq, int NT) {
 size_t attention_part_bytes_bound(int cap, int Hq, int hd) {
   // a split launch has S * rows <= SMs * (rows of a pair) for any batch shape
   // (S x CTAs <= resident CTAs: SMs x 2 tiles of 128 rows either way)
-  const size_t rows = std::min((size_t)8 * cap * Hq, (size_t)num_sms() * 2 * BT);
+  const size_t rows = std::min((size_t)kMaxShares * cap * Hq, (size_t)num_sms() * 2 * BT);
   return rows * (hd + 2) * sizeof(float);
 }
 
