@@ -484,9 +484,18 @@ __global__ void __launch_bounds__(128) lm_merge_kernel(const float* __restrict__
   if (j >= *n_lm || j >= cap) return;
   const float* p = part + (size_t)j * tiles * 3;
   SoftStat st{-INFINITY, 0.f, 0x7fffffff};
-  for (int t = lane; t < tiles; t += 32) {
-    SoftStat y{p[3 * t], p[3 * t + 1], __float_as_int(p[3 * t + 2])};
-    st = soft_merge(st, y);
+  // each lane's tiles lane, lane + 32, ... in order; eight of them loaded at once
+  constexpr int U = 8;
+  for (int t0 = lane; t0 < tiles; t0 += 32 * U) {
+    SoftStat y[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = t0 + 32 * u;
+      if (t < tiles) y[u] = SoftStat{p[3 * t], p[3 * t + 1], __float_as_int(p[3 * t + 2])};
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (t0 + 32 * u < tiles) st = soft_merge(st, y[u]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
