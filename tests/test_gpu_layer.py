@@ -119,6 +119,14 @@ def test_layer_bf16_few_rows_split_keys(lib, B, N, counts):
     _run_layer(lib, shape, B=B, N=N, counts=counts, k_cap=max(counts))
 
 
+@pytest.mark.parametrize("B,N,counts", [(1, 1000, [77]), (2, 700, [300, 5])])
+def test_layer_bf16_few_rows_split_keys_hd64(lib, B, N, counts):
+    """The key split at head dim 64 (one query tile per CTA, two CTAs per SM)."""
+    shape = SY.with_(SY.TINY, dtype="bf16", d=512, n_heads=8, n_kv_heads=4, head_dim=64,
+                     ffn=1024, vocab=2048)
+    _run_layer(lib, shape, B=B, N=N, counts=counts, k_cap=max(counts))
+
+
 @pytest.mark.parametrize("heads,kv,hd", [(8, 8, 64), (8, 4, 128)])
 def test_layer_bf16_many_sequences_mixed_counts(lib, heads, kv, hd):
     """A grid several waves deep (76 sequences): row counts cover a lone first
